@@ -1,0 +1,471 @@
+#!/usr/bin/env python
+"""Benchmark of the MSA hot path (index select + sparse attention) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step is one pass of the whole path over one batch: msa_index_select
+(index scores with the fused causal block max pool, then top-k) followed by
+msa_sparse_attn on its ids, with inputs resident in HBM.  Decode workloads
+report algorithmic HBM GB/s (K_idx read once, the selected K/V blocks, q,
+q_idx and the output; scores, ids and partials are overhead, not credit);
+prefill workloads report effective TFLOP/s (2*d_idx per visible (query, group,
+key) for the index GEMM plus 4*d per selected visible (query head, key)).
+
+Multi-GPU (torchrun): every rank runs its own replica of the workload (weak
+scaling, no collective on the data path); the step time is the max over ranks.
+--impl reference runs the float64 CPU oracle on a bounded sample of the same
+workload on rank 0 (the other ranks exit).
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from block_sparse_gqa_03_b200.inputs import WORKLOADS, make_inputs  # noqa: E402
+
+METRIC = "MSA decode µs/step & HBM GB/s at 128K–1M ctx; prefill effective TFLOP/s"
+DEFAULT_WORKLOAD = "decode_128k"
+L2_BYTES = 126 * 2**20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# Per-launch DRAM traffic (read + write bytes) of the dominant kernel, from one ncu
+# capture of the same launch configuration (profiles/); None until captured or
+# after the kernel changed.
+TRAFFIC = {}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if args.impl == "ours" else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available() and args.impl == "ours":
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ----------------------------------------------------------------- work counts
+def positions(prob, seq_lens, device):
+    L = (torch.full((prob.batch,), prob.max_kv, device=device, dtype=torch.int64)
+         if seq_lens is None else seq_lens.to(torch.int64))
+    t = torch.arange(prob.n_q, device=device, dtype=torch.int64)
+    p = L[:, None] - prob.n_q + t[None, :]
+    lim = torch.minimum(L[:, None], p + 1) if prob.causal else L[:, None].expand(-1, prob.n_q)
+    return L, lim.clamp(min=0)  # lim[b, t]: visible tokens are j < lim
+
+
+def selected_visible_tokens(prob, ids, lim):
+    """Visible tokens in the selected blocks, per (b, t, g): [b, n_q, h] int64."""
+    idl = ids.to(torch.int64)
+    start = idl * prob.block
+    n = (lim[:, :, None, None] - start).clamp(min=0, max=prob.block)
+    n = torch.where(idl >= 0, n, torch.zeros_like(n))
+    return n.sum(-1)
+
+
+def work_units(prob, x, ids):
+    """Algorithmic bytes (decode) or flops (prefill), split by stage."""
+    L, lim = positions(prob, x["seq_lens"], ids.device)
+    sel_tok = selected_visible_tokens(prob, ids, lim)  # [b, n_q, h]
+    if prob.is_decode:
+        kidx = int(L.sum()) * prob.d_idx * 2
+        qidx = prob.batch * prob.n_q * prob.h * prob.d_idx * 2
+        kv = int(sel_tok.sum()) * prob.d * 2 * 2
+        q_o = 2 * prob.batch * prob.n_q * prob.H * prob.d * 2
+        return {"select": kidx + qidx, "attn": kv + q_o}
+    index = 2 * prob.d_idx * prob.h * int(lim.sum())
+    attn = 4 * prob.d * prob.G * int(sel_tok.sum())
+    return {"select": index, "attn": attn}
+
+
+# ------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples (200 ms) while the timed region runs."""
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            q = ("index,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                 "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                 "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "--query-gpu=" + q, "--format=csv,noheader,nounits", "-lms", "200",
+                 "-f", self.path], stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self, uuid: str | None):
+        if self.proc is None or not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 10:
+                    continue
+                if uuid and parts[1] != uuid:
+                    continue
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        mx = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[6 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# --------------------------------------------------------------- oracle arm
+def oracle_sample(prob, x, budget_s: float, max_rows: int | None = None):
+    """Times the float64 oracle on a bounded sample: whole sequences for decode,
+    query rows for prefill.  Returns (units processed, seconds, description)."""
+    import numpy as np
+    import oracle
+
+    cfg1 = oracle.Config(1, prob.n_q, prob.max_kv, prob.H, prob.h, prob.d, prob.d_idx,
+                         prob.block, prob.topk, causal=prob.causal, force_own=prob.force_own)
+    units, secs, nseq, nrows = 0.0, 0.0, 0, 0
+    rng = np.random.default_rng(0)
+    for b in range(prob.batch):
+        sl = x["seq_lens"][b:b + 1].cpu() if x["seq_lens"] is not None else None
+        hb = {k: x[k][b:b + 1].cpu() for k in ("q", "k", "v", "q_idx", "k_idx")}
+        if prob.is_decode:
+            rows = [(0, 0)]
+        else:
+            n = max_rows or 64
+            rows = [(0, int(t)) for t in sorted(rng.choice(prob.n_q, size=n, replace=False))]
+        t0 = time.perf_counter()
+        ids, _, _ = oracle.forward(cfg1, hb["q"], hb["k"], hb["v"], hb["q_idx"], hb["k_idx"],
+                                   seq_lens=sl, rows=rows)
+        secs += time.perf_counter() - t0
+        # work of the sampled rows, counted like the GPU's
+        sub = prob.with_(batch=1)
+        ids_t = torch.as_tensor(ids)
+        if prob.is_decode:
+            w = work_units(sub, {"seq_lens": sl}, ids_t.view(1, 1, prob.h, prob.topk))
+            units += w["select"] + w["attn"]
+        else:
+            L, lim = positions(sub, sl, "cpu")
+            tt = torch.as_tensor([r[1] for r in rows])
+            lim_r = lim[0, tt]
+            sel = selected_visible_tokens(sub, ids_t.view(1, len(rows), prob.h, prob.topk),
+                                          lim_r.view(1, -1))
+            units += 2 * prob.d_idx * prob.h * int(lim_r.sum()) + 4 * prob.d * prob.G * int(sel.sum())
+        nseq += 1
+        nrows += len(rows)
+        if secs >= budget_s:
+            break
+    if prob.is_decode:
+        desc = "%d of %d sequences (all %d groups, %d heads), full context" % (
+            nseq, prob.batch, prob.h, prob.H)
+    else:
+        desc = "%d query rows (%d per sequence, %d sequences), all groups and heads" % (
+            nrows, nrows // max(1, nseq), nseq)
+    return units, secs, desc
+
+
+def unit_of(prob):
+    return ("GB/s", 1e9) if prob.is_decode else ("TFLOP/s", 1e12)
+
+
+def run_reference(args, prob, world, rank):
+    import oracle
+    if rank != 0:
+        return
+    # The oracle samples whole sequences (decode) or query rows (prefill) of the
+    # workload; drawing two sequences of it on the host is enough for that.
+    sub = prob.with_(batch=min(prob.batch, 2))
+    x = make_inputs(sub, device="cpu")
+    prob = sub
+    unit, scale = unit_of(prob)
+    budget = 2.0
+    for _ in range(args.warmup):
+        oracle_sample(prob, x, 0.0, max_rows=8)
+    units, secs = 0.0, 0.0
+    desc = ""
+    for _ in range(args.steps):
+        u, s, desc = oracle_sample(prob, x, budget)
+        units += u
+        secs += s
+    value = units / secs / scale
+    cores = oracle.num_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": unit, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,1), bf16 inputs widened to f64)",
+        "config": {"workload": prob.name, **workload_config(prob)},
+        "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle",
+                         "sample": "each step: " + desc},
+        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(prob):
+    c = {"batch": prob.batch, "n_q": prob.n_q, "context": prob.max_kv, "H": prob.H, "h": prob.h,
+         "d": prob.d, "d_idx": prob.d_idx, "block": prob.block, "topk": prob.topk,
+         "causal": prob.causal, "force_own_block": prob.force_own}
+    if prob.len_range:
+        c["seq_len_range"] = list(prob.len_range)
+    if prob.plant_frac:
+        c["planted_block_frac"] = prob.plant_frac
+    return c
+
+
+# ----------------------------------------------------------------- our arm
+def run_ours(args, prob, world, rank, local):
+    from block_sparse_gqa_03_b200 import msa
+
+    dev = torch.device("cuda", local if world > 1 else 0)
+    x = make_inputs(prob, device=dev, seed=prob.seed + rank)
+    sl = x["seq_lens"]
+    kw = dict(block=prob.block, causal=prob.causal, seq_lens=sl)
+    ids = torch.empty((prob.batch, prob.n_q, prob.h, prob.topk), dtype=torch.int32, device=dev)
+    out = torch.empty_like(x["q"])
+    ws = msa.Workspace(dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        msa.msa_index_select(x["q_idx"], x["k_idx"], topk=prob.topk,
+                             force_own_block=prob.force_own, block_ids=ids, workspace=ws, **kw)
+        msa.msa_sparse_attn(x["q"], x["k"], x["v"], ids, out=out, workspace=ws, **kw)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    assert msa.msa_get_device_status(ws) == msa.MSA_OK
+    units = work_units(prob, x, ids)
+    touched = units["select"] + units["attn"] if prob.is_decode else None
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    props = torch.cuda.get_device_properties(dev)
+    uuid = str(getattr(props, "uuid", "")) or None
+    if uuid and not uuid.startswith("GPU-"):
+        uuid = "GPU-" + uuid
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev.index) as clk:
+        t_start.record(stream)
+        for i in range(K):
+            ev[i][0].record(stream)
+            msa.msa_index_select(x["q_idx"], x["k_idx"], topk=prob.topk,
+                                 force_own_block=prob.force_own, block_ids=ids, workspace=ws, **kw)
+            ev[i][1].record(stream)
+            msa.msa_sparse_attn(x["q"], x["k"], x["v"], ids, out=out, workspace=ws, **kw)
+            ev[i][2].record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world)
+    total_ms = max_over_ranks(t_start.elapsed_time(t_end), world)
+    sel_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+    attn_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+    assert msa.msa_get_device_status(ws) == msa.MSA_OK
+    ms_per_step = total_ms / K
+    unit, scale = unit_of(prob)
+    total_units = (units["select"] + units["attn"]) * world
+    value = total_units / (ms_per_step * 1e-3) / scale
+
+    # End to end through the public API: inputs from pinned host memory, the
+    # result read back, every step.
+    e2e = run_e2e(args, prob, x, dev, world, msa, kw)
+
+    p_sel = msa.make_params(batch=prob.batch, n_q=prob.n_q, max_kv=prob.max_kv, H=prob.H,
+                            h=prob.h, d=prob.d, d_idx=prob.d_idx, block=prob.block,
+                            topk=prob.topk, causal=prob.causal, q=x["q"], k=x["k"], v=x["v"],
+                            q_idx=x["q_idx"], k_idx=x["k_idx"], out=out)
+    launches_per_step = (msa.msa_launch_count(p_sel, msa.MSA_OP_INDEX_SELECT)
+                         + msa.msa_launch_count(p_sel, msa.MSA_OP_SPARSE_ATTN))
+
+    peaks, peak_kind = load_peaks()
+    dom = "attn" if attn_ms >= sel_ms else "select"
+    dom_ms = attn_ms if dom == "attn" else sel_ms
+    kernel = {"attn": "sparse_attn_kernel (+combine)", "select": "index_scan_kernel (+topk)"}[dom]
+    if prob.is_decode:
+        roof = {"bound": "hbm", "achieved": units[dom] / (dom_ms * 1e-3) / 1e9,
+                "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+    else:
+        key = "bf16_tflops_sustained" if ms_per_step > 50 else "bf16_tflops"
+        roof = {"bound": "tensor", "achieved": units[dom] / (dom_ms * 1e-3) / 1e12,
+                "peak": peaks.get(key, FALLBACK_PEAKS[key]), "unit": "TFLOP/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = TRAFFIC.get((prob.name, dom))
+    roof["kernel"] = kernel
+    roof["peak_source"] = "of %s" % peak_kind
+
+    line = {
+        "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16%s)" % (", planted blocks" if prob.plant_frac else ""),
+        "config": {"workload": prob.name, **workload_config(prob),
+                   "l2": ("inputs larger than L2 (%.2f GB touched per step)" % (touched / 1e9)
+                          if touched else "inputs larger than L2"),
+                   "parallelism": "replicas" if world > 1 else "single GPU"},
+        "us_per_step": 1e3 * ms_per_step,
+        "stage_ms": {"index_select": sel_ms, "sparse_attn": attn_ms},
+        "roofline": roof,
+        "e2e": e2e,
+        "gpu_launches": launches_per_step * K,
+    }
+    if prob.is_decode:
+        line["tokens_per_s"] = prob.batch * world / (ms_per_step * 1e-3)
+    if rank == 0:
+        line["clocks"] = clk.summary(uuid)
+        if world == 1 and not args.no_cpu_baseline:
+            import oracle
+            u, s, desc = oracle_sample(prob, {k: v for k, v in x.items()}, args.cpu_budget)
+            line["cpu_baseline"] = {"value": u / s / scale, "unit": unit,
+                                    "cores": oracle.num_threads(), "kind": "oracle",
+                                    "sample": desc}
+        print(json.dumps(line), flush=True)
+
+
+def run_e2e(args, prob, x, dev, world, msa, kw):
+    """Same metric through msa_forward with host buffers: pinned host -> device copies
+    of the step's inputs, the call, and the output read back, inside the timed region."""
+    stream = torch.cuda.current_stream(dev)
+    if prob.is_decode:
+        # a decode step's inputs: the new token's queries, and its K/V/K_idx rows
+        # written into the resident cache at position L_b - 1
+        names = ["q", "q_idx"]
+        host = {n: x[n].cpu().pin_memory() for n in names}
+        L = (x["seq_lens"].cpu().tolist() if x["seq_lens"] is not None
+             else [prob.max_kv] * prob.batch)
+        rows = {n: torch.stack([x[n][b, L[b] - 1] for b in range(prob.batch)]).cpu().pin_memory()
+                for n in ("k", "v", "k_idx")}
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        h2d += sum(t.numel() * t.element_size() for t in rows.values())
+    else:
+        names = ["q", "k", "v", "q_idx", "k_idx"]
+        host = {n: x[n].cpu().pin_memory() for n in names}
+        rows, L = {}, None
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+    out_dev = torch.empty_like(x["q"])
+    out_host = torch.empty(out_dev.shape, dtype=out_dev.dtype, pin_memory=True)
+    d2h = out_host.numel() * out_host.element_size()
+    ws = msa.Workspace(dev)
+    nsteps = max(1, min(args.steps, 20))
+
+    def one():
+        for n in names:
+            x[n].copy_(host[n], non_blocking=True)
+        for n, t in rows.items():
+            for b in range(prob.batch):
+                x[n][b, L[b] - 1].copy_(t[b], non_blocking=True)
+        msa.msa_forward(x["q"], x["k"], x["v"], x["q_idx"], x["k_idx"], topk=prob.topk,
+                        force_own_block=prob.force_own, out=out_dev, workspace=ws, **kw)
+        out_host.copy_(out_dev, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    s0 = torch.cuda.Event(enable_timing=True)
+    s1 = torch.cuda.Event(enable_timing=True)
+    s0.record(stream)
+    for _ in range(nsteps):
+        one()
+    s1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    ms = max_over_ranks(s0.elapsed_time(s1), world) / nsteps
+    ids = torch.empty((prob.batch, prob.n_q, prob.h, prob.topk), dtype=torch.int32, device=dev)
+    msa.msa_index_select(x["q_idx"], x["k_idx"], topk=prob.topk, force_own_block=prob.force_own,
+                         block_ids=ids, workspace=ws, **kw)
+    u = work_units(prob, x, ids)
+    unit, scale = unit_of(prob)
+    return {"value": (u["select"] + u["attn"]) * world / (ms * 1e-3) / scale, "unit": unit,
+            "ms_per_step": ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default=DEFAULT_WORKLOAD)
+    ap.add_argument("--cpu-budget", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    prob = WORKLOADS[args.workload]
+    world, rank, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            run_reference(args, prob, world, rank)
+        else:
+            run_ours(args, prob, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

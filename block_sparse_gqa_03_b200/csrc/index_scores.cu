@@ -1,0 +1,211 @@
+// Index branch, part 1: index scores with Block Max Pool fused into the epilogue.
+//
+// "MiniMax goes sparse" (atlascloud.ai), section 1, step 1: one index query per
+// GQA group is scored against a single-head index key shared by all heads
+// (Q_idx . K_idx^T), and Block Max Pool compresses the token scores to block
+// scores.  "MiniMax M3 的 MSA ..." (ai.air7.fun), first layer, says the same.
+// The causal mask is applied to token scores before pooling, so a query's own
+// block pools only tokens at or before its position; token scores never leave
+// the registers.
+//
+// Mapping.  The contraction is [tokens x d_idx] . [d_idx x columns], where a
+// column is one (query, group) index vector.  It runs on the warp-level bf16
+// tensor-core MMA (m16n8k16): rows are tokens, so the block max over tokens is
+// a max over accumulator rows (in-thread, then across the 8 row-lanes).  The
+// decode scan streams K_idx from HBM exactly once with 16-byte coalesced loads
+// straight into MMA fragments: each thread loads 8 consecutive dims of a token
+// row, and the same dim permutation is applied to the index-query fragments,
+// which leaves the dot products unchanged.
+#include "kernels.h"
+
+namespace msa {
+namespace {
+
+struct ScanArgs {
+  const uint16_t* q_idx;
+  const uint16_t* k_idx;
+  int64_t qi_s0, qi_s1, qi_s2, ki_s0, ki_s1;
+  const int32_t* seq_lens;
+  int n_q, max_kv, h, block, nblk, causal, qt, ntiles;
+  float* scores;
+  int fill_tail;
+  DeviceStatus* st;
+};
+
+constexpr int kScanWarps = 8;
+
+template <int DI, int NT>
+__global__ void __launch_bounds__(kScanWarps * 32) index_scan_kernel(ScanArgs a) {
+  constexpr int KC = DI / 32;  // 32-dim chunks of the index head dim
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int r = lane >> 2, q = lane & 3;
+  const int tile = blockIdx.x % a.ntiles;
+  const int b = blockIdx.x / a.ntiles;
+  const int t0 = tile * a.qt;
+  const int L = kv_length(a.seq_lens, b, a.max_kv, a.st);
+  const int ncols = a.qt * a.h;
+
+  // B fragments: column c = nt*8 + r; dims [32kc + 8q, 32kc + 8q + 8) of its index query.
+  uint4 bq[NT][KC];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    const int c = nt * 8 + r;
+    const int t = t0 + c / a.h, g = c % a.h;
+    const bool ok = c < ncols && t < a.n_q;
+    const uint16_t* src = a.q_idx + b * a.qi_s0 + (int64_t)t * a.qi_s1 + g * a.qi_s2 + 8 * q;
+#pragma unroll
+    for (int kc = 0; kc < KC; ++kc) bq[nt][kc] = ok ? ld_u4(src + 32 * kc) : make_uint4(0, 0, 0, 0);
+  }
+  // Accumulator columns of this lane: c = nt*8 + 2q + e.  Visible tokens j < lim.
+  int lim[NT][2];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int c = nt * 8 + 2 * q + e;
+      const int t = t0 + c / a.h;
+      const int p = L - a.n_q + t;
+      lim[nt][e] = a.causal ? min(L, p + 1) : L;
+    }
+
+  const int t_last = min(t0 + a.qt, a.n_q) - 1;
+  const int p_last = L - a.n_q + t_last;
+  const int nb_b = (L + a.block - 1) / a.block;
+  const int F = a.causal ? (p_last < 0 ? 0 : min(nb_b, p_last / a.block + 1)) : nb_b;
+
+  const int nw = gridDim.y * kScanWarps;
+  const int wid = blockIdx.y * kScanWarps + warp;
+  const uint16_t* kb = a.k_idx + b * a.ki_s0 + 8 * q;
+  const int nmt = a.block / 16;
+  const float ninf = -__int_as_float(0x7f800000);
+
+  for (int beta = wid; beta < F; beta += nw) {
+    float cm[NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) cm[nt][0] = cm[nt][1] = ninf;
+#pragma unroll 2
+    for (int mt = 0; mt < nmt; ++mt) {
+      const int jl = beta * a.block + mt * 16 + r, jh = jl + 8;
+      uint4 X[KC], Y[KC];
+#pragma unroll
+      for (int kc = 0; kc < KC; ++kc) {
+        X[kc] = jl < L ? ld_stream_u4(kb + (int64_t)jl * a.ki_s1 + 32 * kc) : make_uint4(0, 0, 0, 0);
+        Y[kc] = jh < L ? ld_stream_u4(kb + (int64_t)jh * a.ki_s1 + 32 * kc) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int kc = 0; kc < KC; ++kc) {
+          mma_bf16_16816(acc, X[kc].x, Y[kc].x, X[kc].y, Y[kc].y, bq[nt][kc].x, bq[nt][kc].y);
+          mma_bf16_16816(acc, X[kc].z, Y[kc].z, X[kc].w, Y[kc].w, bq[nt][kc].z, bq[nt][kc].w);
+        }
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          cm[nt][e] = fmaxf(cm[nt][e], jl < lim[nt][e] ? acc[e] : ninf);
+          cm[nt][e] = fmaxf(cm[nt][e], jh < lim[nt][e] ? acc[2 + e] : ninf);
+        }
+      }
+    }
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        float v = cm[nt][e];
+        v = warp_max_xor(v, 4);
+        v = warp_max_xor(v, 8);
+        v = warp_max_xor(v, 16);
+        cm[nt][e] = v;
+      }
+    if (r == 0) {
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int c = nt * 8 + 2 * q + e;
+          const int t = t0 + c / a.h, g = c % a.h;
+          if (c < ncols && t < a.n_q)
+            a.scores[(((int64_t)b * a.n_q + t) * a.h + g) * a.nblk + beta] = cm[nt][e];
+        }
+    }
+  }
+  if (a.fill_tail && r == 0) {
+    for (int beta = F + wid; beta < a.nblk; beta += nw) {
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int c = nt * 8 + 2 * q + e;
+          const int t = t0 + c / a.h, g = c % a.h;
+          if (c < ncols && t < a.n_q)
+            a.scores[(((int64_t)b * a.n_q + t) * a.h + g) * a.nblk + beta] = ninf;
+        }
+    }
+  }
+}
+
+template <int DI, int NT>
+cudaError_t run_scan(const ScanArgs& a, int batch, cudaStream_t stream) {
+  const int ctas_per_row = a.ntiles * batch;
+  // Spread the block range of each query tile over enough warps to fill the
+  // GPU a few times over; each warp then walks its blocks with a stride.
+  const int want = num_sms() * 4;
+  int split = (want + ctas_per_row - 1) / ctas_per_row;
+  const int max_split = (a.nblk + kScanWarps - 1) / kScanWarps;
+  split = max(1, min(split, max_split));
+  dim3 grid(ctas_per_row, split);
+  index_scan_kernel<DI, NT><<<grid, kScanWarps * 32, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_index_scores(const Shape& s, const uint16_t* q_idx, const uint16_t* k_idx,
+                                float* scores, bool fill_tail, DeviceStatus* st,
+                                cudaStream_t stream) {
+  ScanArgs a;
+  a.q_idx = q_idx;
+  a.k_idx = k_idx;
+  a.qi_s0 = s.qi_s[0];
+  a.qi_s1 = s.qi_s[1];
+  a.qi_s2 = s.qi_s[2];
+  a.ki_s0 = s.ki_s[0];
+  a.ki_s1 = s.ki_s[1];
+  a.seq_lens = s.seq_lens;
+  a.n_q = s.n_q;
+  a.max_kv = s.max_kv;
+  a.h = s.h;
+  a.block = s.block;
+  a.nblk = s.nblk;
+  a.causal = s.causal;
+  a.scores = scores;
+  a.fill_tail = fill_tail ? 1 : 0;
+  a.st = st;
+  // Columns per warp: all h groups of one query in decode; in prefill a tile of
+  // queries whose columns fill four 8-wide MMA tiles.
+  int nt;
+  if (s.n_q == 1) {
+    nt = (s.h + 7) / 8;
+    a.qt = 1;
+  } else {
+    nt = 4;
+    a.qt = max(1, 32 / s.h);
+  }
+  a.ntiles = (s.n_q + a.qt - 1) / a.qt;
+  const int B = s.batch;
+#define MSA_SCAN_CASE(DI_, NT_) \
+  if (s.d_idx == DI_ && nt == NT_) return run_scan<DI_, NT_>(a, B, stream);
+  MSA_SCAN_CASE(32, 1)
+  MSA_SCAN_CASE(32, 2)
+  MSA_SCAN_CASE(32, 4)
+  MSA_SCAN_CASE(64, 1)
+  MSA_SCAN_CASE(64, 2)
+  MSA_SCAN_CASE(64, 4)
+  MSA_SCAN_CASE(128, 1)
+  MSA_SCAN_CASE(128, 2)
+  MSA_SCAN_CASE(128, 4)
+#undef MSA_SCAN_CASE
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace msa

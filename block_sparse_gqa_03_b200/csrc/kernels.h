@@ -1,0 +1,44 @@
+// Launchers of the MSA kernels, called by the C-ABI layer (msa_api.cu).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace msa {
+
+// Problem description after validation; strides in elements.
+struct Shape {
+  int batch, n_q, max_kv, H, h, G, d, d_idx, block, topk, nblk;
+  int causal, force_own;
+  float scale;
+  const int32_t* seq_lens;
+  int64_t q_s[3], k_s[3], v_s[3], qi_s[3], ki_s[2], o_s[3];
+};
+
+// Stage 1a/1b: block-max-pooled index scores, fp32 [batch, n_q, h, nblk].
+// Blocks past a row's frontier are written -inf only when fill_tail is set.
+cudaError_t launch_index_scores(const Shape& s, const uint16_t* q_idx, const uint16_t* k_idx,
+                                float* scores, bool fill_tail, DeviceStatus* st,
+                                cudaStream_t stream);
+
+// Stage 1c: top-k block ids, int32 [batch, n_q, h, topk], from the scores.
+cudaError_t launch_topk(const Shape& s, const float* scores, int32_t* ids, DeviceStatus* st,
+                        cudaStream_t stream);
+
+// Stage 2: workspace bytes for the split-KV partials, then the attention.
+size_t attn_partial_bytes(const Shape& s);
+int attn_launches(const Shape& s);
+cudaError_t launch_sparse_attn(const Shape& s, const uint16_t* q, const uint16_t* k,
+                               const uint16_t* v, const int32_t* ids, uint16_t* out, float* lse,
+                               void* partials, size_t partial_bytes, DeviceStatus* st,
+                               cudaStream_t stream);
+
+// Test hook: one bounded wait that runs out and records kErrTimeout.
+cudaError_t launch_wait_timeout_probe(DeviceStatus* st, uint64_t wait_ns, cudaStream_t stream);
+
+int num_sms();
+
+}  // namespace msa

@@ -1,0 +1,284 @@
+"""Thin ctypes binding of ``libmsa.so`` (C ABI declared in ``include/msa.h``).
+
+Argument marshalling only: every step of MSA runs in the library's CUDA kernels.
+torch tensors provide device memory and the current stream.  The names follow
+the C ABI: ``msa_index_select``, ``msa_sparse_attn``, ``msa_forward``,
+``msa_workspace_size``, ``msa_get_device_status``, ``msa_workspace_init``,
+``msa_selftest_wait_timeout``, ``msa_status_string``.
+
+There is no fallback: if ``libmsa.so`` has not been built, or no CUDA device is
+present, these functions raise.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmsa.so")
+
+MSA_OK = 0
+MSA_ERR_INVALID_ARG = 1
+MSA_ERR_UNSUPPORTED = 2
+MSA_ERR_WORKSPACE = 3
+MSA_ERR_CUDA = 4
+MSA_ERR_TIMEOUT = 5
+MSA_ERR_DEVICE_ASSERT = 6
+
+MSA_OP_INDEX_SELECT = 0
+MSA_OP_SPARSE_ATTN = 1
+MSA_OP_FORWARD = 2
+
+EXPORTED = ("msa_workspace_size", "msa_index_select", "msa_sparse_attn", "msa_forward",
+            "msa_get_device_status", "msa_workspace_init", "msa_selftest_wait_timeout",
+            "msa_launch_count", "msa_status_string")
+
+
+class MsaError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__("%s failed: %s (status %d)" % (what, msa_status_string(code), code))
+        self.code = code
+
+
+class Params(ctypes.Structure):
+    """Mirror of ``msa_params_t``."""
+
+    _fields_ = [(n, ctypes.c_int32) for n in (
+        "batch", "n_q", "max_kv", "H", "h", "d", "d_idx", "block", "topk", "causal",
+        "force_own_block")] + [
+        ("softmax_scale", ctypes.c_float),
+        ("seq_lens", ctypes.c_void_p),
+        ("q_strides", ctypes.c_int64 * 3),
+        ("k_strides", ctypes.c_int64 * 3),
+        ("v_strides", ctypes.c_int64 * 3),
+        ("qi_strides", ctypes.c_int64 * 3),
+        ("ki_strides", ctypes.c_int64 * 2),
+        ("o_strides", ctypes.c_int64 * 3),
+    ]
+
+
+_lib = None
+_lib_lock = threading.Lock()
+
+
+def load_library():
+    """Load ``libmsa.so``; raises if it has not been built."""
+    global _lib
+    with _lib_lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError("libmsa.so is not built (run __graft_entry__.build() or "
+                                   "python -m block_sparse_gqa_03_b200.build)")
+            lib = ctypes.CDLL(LIB_PATH)
+            P, S, I = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
+            lib.msa_workspace_size.argtypes = [P, I]
+            lib.msa_workspace_size.restype = S
+            lib.msa_index_select.argtypes = [P, P, P, P, P, P, S, P]
+            lib.msa_index_select.restype = I
+            lib.msa_sparse_attn.argtypes = [P, P, P, P, P, P, P, P, S, P]
+            lib.msa_sparse_attn.restype = I
+            lib.msa_forward.argtypes = [P, P, P, P, P, P, P, P, P, P, P, S, P]
+            lib.msa_forward.restype = I
+            lib.msa_get_device_status.argtypes = [P, P]
+            lib.msa_get_device_status.restype = I
+            lib.msa_workspace_init.argtypes = [P, S, P]
+            lib.msa_workspace_init.restype = I
+            lib.msa_selftest_wait_timeout.argtypes = [P, S, ctypes.c_uint64, P]
+            lib.msa_selftest_wait_timeout.restype = I
+            lib.msa_launch_count.argtypes = [P, I]
+            lib.msa_launch_count.restype = I
+            lib.msa_status_string.argtypes = [I]
+            lib.msa_status_string.restype = ctypes.c_char_p
+            _lib = lib
+    return _lib
+
+
+def msa_status_string(code: int) -> str:
+    return load_library().msa_status_string(int(code)).decode()
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream=None) -> int | None:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream or None
+
+
+def _outer(t: torch.Tensor, n: int):
+    if t.stride(-1) != 1:
+        raise ValueError("innermost axis must be contiguous")
+    return list(t.stride()[:n])
+
+
+def make_params(*, batch, n_q, max_kv, H, h, d, d_idx, block, topk, causal=True,
+                force_own_block=False, softmax_scale=0.0, seq_lens=None, q=None, k=None, v=None,
+                q_idx=None, k_idx=None, out=None) -> Params:
+    p = Params()
+    p.batch, p.n_q, p.max_kv, p.H, p.h = batch, n_q, max_kv, H, h
+    p.d, p.d_idx, p.block, p.topk = d, d_idx, block, topk
+    p.causal, p.force_own_block = int(bool(causal)), int(bool(force_own_block))
+    p.softmax_scale = float(softmax_scale)
+    p.seq_lens = _ptr(seq_lens)
+    if q is not None:
+        p.q_strides[:] = _outer(q, 3)
+    if k is not None:
+        p.k_strides[:] = _outer(k, 3)
+    if v is not None:
+        p.v_strides[:] = _outer(v, 3)
+    if q_idx is not None:
+        p.qi_strides[:] = _outer(q_idx, 3)
+    if k_idx is not None:
+        p.ki_strides[:] = _outer(k_idx, 2)
+    if out is not None:
+        p.o_strides[:] = _outer(out, 3)
+    return p
+
+
+class Workspace:
+    """A device buffer for the library's workspace, grown on demand."""
+
+    def __init__(self, device=None):
+        self.device = torch.device(device or "cuda")
+        self.buf = None
+
+    def get(self, nbytes: int) -> torch.Tensor:
+        if self.buf is None or self.buf.numel() < nbytes:
+            self.buf = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=self.device)
+            rc = load_library().msa_workspace_init(self.buf.data_ptr(), self.buf.numel(), _stream())
+            if rc != MSA_OK:
+                raise MsaError(rc, "msa_workspace_init")
+        return self.buf
+
+
+_default_ws: dict = {}
+
+
+def _workspace(ws: Workspace | None, device) -> Workspace:
+    if ws is not None:
+        return ws
+    key = torch.device(device).index
+    if key not in _default_ws:
+        _default_ws[key] = Workspace(device)
+    return _default_ws[key]
+
+
+def msa_workspace_size(params: Params, op: int) -> int:
+    return int(load_library().msa_workspace_size(ctypes.byref(params), int(op)))
+
+
+def msa_launch_count(params: Params, op: int) -> int:
+    return int(load_library().msa_launch_count(ctypes.byref(params), int(op)))
+
+
+def msa_get_device_status(workspace: Workspace | torch.Tensor, stream=None) -> int:
+    buf = workspace.buf if isinstance(workspace, Workspace) else workspace
+    return int(load_library().msa_get_device_status(buf.data_ptr(), _stream(stream)))
+
+
+def msa_workspace_init(buf: torch.Tensor, stream=None) -> int:
+    return int(load_library().msa_workspace_init(buf.data_ptr(), buf.numel(), _stream(stream)))
+
+
+def msa_selftest_wait_timeout(buf: torch.Tensor, wait_ns: int, stream=None) -> int:
+    return int(load_library().msa_selftest_wait_timeout(buf.data_ptr(), buf.numel(), int(wait_ns),
+                                                        _stream(stream)))
+
+
+def _check(rc: int, what: str):
+    if rc != MSA_OK:
+        raise MsaError(rc, what)
+
+
+def msa_index_select(q_idx, k_idx, *, block, topk, causal=True, force_own_block=False,
+                     seq_lens=None, return_scores=False, block_ids=None, block_scores=None,
+                     workspace: Workspace | None = None, stream=None):
+    """Stage 1: block ids int32 [b, n_q, h, topk] (and fp32 block scores if asked)."""
+    b, n_q, h, d_idx = q_idx.shape
+    max_kv = k_idx.shape[1]
+    nblk = (max_kv + block - 1) // block
+    p = make_params(batch=b, n_q=n_q, max_kv=max_kv, H=h, h=h, d=64, d_idx=d_idx, block=block,
+                    topk=topk, causal=causal, force_own_block=force_own_block,
+                    seq_lens=seq_lens, q_idx=q_idx, k_idx=k_idx)
+    dev = q_idx.device
+    if block_ids is None:
+        block_ids = torch.empty((b, n_q, h, topk), dtype=torch.int32, device=dev)
+    if return_scores and block_scores is None:
+        block_scores = torch.empty((b, n_q, h, nblk), dtype=torch.float32, device=dev)
+    need = msa_workspace_size(p, MSA_OP_INDEX_SELECT)
+    if need == 0:
+        raise MsaError(MSA_ERR_INVALID_ARG, "msa_workspace_size")
+    ws = _workspace(workspace, dev).get(need)
+    _check(load_library().msa_index_select(ctypes.byref(p), _ptr(q_idx), _ptr(k_idx),
+                                           _ptr(block_ids), _ptr(block_scores), ws.data_ptr(),
+                                           ws.numel(), _stream(stream)), "msa_index_select")
+    return (block_ids, block_scores) if return_scores else block_ids
+
+
+def msa_sparse_attn(q, k, v, block_ids, *, block, causal=True, seq_lens=None, softmax_scale=0.0,
+                    return_lse=False, out=None, lse=None, workspace: Workspace | None = None,
+                    stream=None):
+    """Stage 2: bf16 output [b, n_q, H, d] (and fp32 lse [b, n_q, H] if asked)."""
+    b, n_q, H, d = q.shape
+    max_kv, h = k.shape[1], k.shape[2]
+    topk = block_ids.shape[-1]
+    if out is None:
+        out = torch.empty_like(q)
+    if return_lse and lse is None:
+        lse = torch.empty((b, n_q, H), dtype=torch.float32, device=q.device)
+    p = make_params(batch=b, n_q=n_q, max_kv=max_kv, H=H, h=h, d=d, d_idx=32, block=block,
+                    topk=topk, causal=causal, softmax_scale=softmax_scale, seq_lens=seq_lens,
+                    q=q, k=k, v=v, out=out)
+    need = msa_workspace_size(p, MSA_OP_SPARSE_ATTN)
+    if need == 0:
+        raise MsaError(MSA_ERR_INVALID_ARG, "msa_workspace_size")
+    ws = _workspace(workspace, q.device).get(need)
+    _check(load_library().msa_sparse_attn(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v),
+                                          _ptr(block_ids), _ptr(out), _ptr(lse), ws.data_ptr(),
+                                          ws.numel(), _stream(stream)), "msa_sparse_attn")
+    return (out, lse) if return_lse else out
+
+
+def msa_forward(q, k, v, q_idx, k_idx, *, block, topk, causal=True, force_own_block=False,
+                seq_lens=None, softmax_scale=0.0, out=None, block_ids=None, block_scores=None,
+                lse=None, return_ids=False, return_scores=False, return_lse=False,
+                workspace: Workspace | None = None, stream=None, params: Params | None = None):
+    """Both stages; returns out, plus (ids, scores, lse) when asked, in that order."""
+    b, n_q, H, d = q.shape
+    max_kv, h = k.shape[1], k.shape[2]
+    d_idx = q_idx.shape[-1]
+    nblk = (max_kv + block - 1) // block
+    dev = q.device
+    if out is None:
+        out = torch.empty_like(q)
+    if return_ids and block_ids is None:
+        block_ids = torch.empty((b, n_q, h, topk), dtype=torch.int32, device=dev)
+    if return_scores and block_scores is None:
+        block_scores = torch.empty((b, n_q, h, nblk), dtype=torch.float32, device=dev)
+    if return_lse and lse is None:
+        lse = torch.empty((b, n_q, H), dtype=torch.float32, device=dev)
+    p = params or make_params(batch=b, n_q=n_q, max_kv=max_kv, H=H, h=h, d=d, d_idx=d_idx,
+                              block=block, topk=topk, causal=causal,
+                              force_own_block=force_own_block, softmax_scale=softmax_scale,
+                              seq_lens=seq_lens, q=q, k=k, v=v, q_idx=q_idx, k_idx=k_idx, out=out)
+    need = msa_workspace_size(p, MSA_OP_FORWARD)
+    if need == 0:
+        raise MsaError(MSA_ERR_INVALID_ARG, "msa_workspace_size")
+    ws = _workspace(workspace, dev).get(need)
+    _check(load_library().msa_forward(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(q_idx),
+                                      _ptr(k_idx), _ptr(out), _ptr(block_ids), _ptr(block_scores),
+                                      _ptr(lse), ws.data_ptr(), ws.numel(), _stream(stream)),
+           "msa_forward")
+    res = [out]
+    if return_ids:
+        res.append(block_ids)
+    if return_scores:
+        res.append(block_scores)
+    if return_lse:
+        res.append(lse)
+    return res[0] if len(res) == 1 else tuple(res)

@@ -1,0 +1,168 @@
+/*
+ * msa.h - C ABI of libmsa.so: MiniMax Sparse Attention (MSA) on B200 (sm_100a).
+ *
+ * MSA is two-stage block-sparse GQA attention:
+ *   stage 1, the index branch: one index query per GQA group is scored against a
+ *     single-head index key shared by all heads; token scores are max-pooled into
+ *     per-block scores under the causal mask, and a top-k picks the KV blocks of
+ *     each (query, group).  Sources: "MiniMax goes sparse" (atlascloud.ai),
+ *     section 1, step 1; "MiniMax M3 的 MSA 与阶跃 Step 3.7 Flash 的 MFA"
+ *     (ai.air7.fun), section "MSA：稀疏注意力的一种极简实现", first layer.
+ *   stage 2, the sparse branch: exact softmax attention over the raw K/V of only
+ *     the selected blocks; all query heads of a group share the group's
+ *     selection.  Sources: the same sections, step 2 / second layer.
+ *
+ * Shapes and notation
+ *   batch         number of sequences b
+ *   n_q           query tokens per sequence (n_q = 1 is one decode step)
+ *   max_kv        token capacity of the K/V buffers (allocated length)
+ *   seq_lens[b]   KV length L_b of sequence b (device int32; NULL: all = max_kv)
+ *   H, h          query heads and KV heads; h is also the number of index groups;
+ *                 G = H / h heads per group, head hq belongs to group hq / G
+ *   d, d_idx      head dim of q/k/v and of q_idx/k_idx
+ *   block         tokens per KV block B; nblk = ceil(max_kv / B)
+ *   topk          blocks kept per (query, group)
+ *   Query t of sequence b sits at absolute position p = L_b - n_q + t.
+ *
+ * Tensor layouts (element strides given in msa_params_t; the innermost axis is
+ * always contiguous):
+ *   q      bf16 [batch, n_q, H, d]          k, v   bf16 [batch, max_kv, h, d]
+ *   q_idx  bf16 [batch, n_q, h, d_idx]      k_idx  bf16 [batch, max_kv, d_idx]
+ *   out    bf16 [batch, n_q, H, d]
+ *   block_ids    int32 [batch, n_q, h, topk]   dense, row-major
+ *   block_scores fp32  [batch, n_q, h, nblk]   dense, row-major
+ *   lse          fp32  [batch, n_q, H]         dense, row-major (natural log)
+ *
+ * Supported sizes: d in {64, 128}; d_idx in {32, 64, 128}; block in {16, 32, 64,
+ * 128}; 1 <= G <= 16; 1 <= topk <= 4096; h <= 16; n_q <= max_kv; all base pointers
+ * 16-byte aligned and every outer stride a multiple of 8 elements.  Anything else
+ * returns MSA_ERR_UNSUPPORTED (or MSA_ERR_INVALID_ARG for inconsistent input).
+ * There is no CPU fallback.
+ *
+ * Ownership and execution
+ *   The caller owns every buffer, the workspace included; the library allocates
+ *   no memory and keeps no state between calls.  All pointers except `params`
+ *   are device pointers.  Calls are asynchronous on `stream`: argument errors
+ *   return before anything is launched, launch failures return MSA_ERR_CUDA, and
+ *   errors found on the device (a bounded wait that ran out, an id out of range)
+ *   are recorded in a sticky word at the start of the workspace that
+ *   msa_get_device_status() reads.  Calls that share a workspace must be ordered
+ *   on one stream.
+ */
+#ifndef MSA_H_
+#define MSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define MSA_API __attribute__((visibility("default")))
+#else
+#define MSA_API
+#endif
+
+typedef uint16_t msa_bf16_t;          /* raw bf16 bits */
+typedef struct CUstream_st* msa_stream_t; /* same handle as cudaStream_t; NULL = legacy default */
+
+typedef enum msa_status {
+  MSA_OK = 0,
+  MSA_ERR_INVALID_ARG = 1,   /* null pointer, inconsistent shape, bad stride */
+  MSA_ERR_UNSUPPORTED = 2,   /* a size outside the supported set above */
+  MSA_ERR_WORKSPACE = 3,     /* workspace null, misaligned or smaller than msa_workspace_size() */
+  MSA_ERR_CUDA = 4,          /* a CUDA runtime call or kernel launch failed */
+  MSA_ERR_TIMEOUT = 5,       /* device: a bounded wait in a kernel ran out */
+  MSA_ERR_DEVICE_ASSERT = 6  /* device: an input broke a precondition (e.g. block id >= nblk) */
+} msa_status_t;
+
+typedef enum msa_op {
+  MSA_OP_INDEX_SELECT = 0,
+  MSA_OP_SPARSE_ATTN = 1,
+  MSA_OP_FORWARD = 2
+} msa_op_t;
+
+typedef struct msa_params {
+  int32_t batch, n_q, max_kv, H, h, d, d_idx, block, topk;
+  int32_t causal;          /* 1: query at p sees tokens j <= p; 0: all j < L_b */
+  int32_t force_own_block; /* 1: the block holding p is always selected */
+  float softmax_scale;     /* <= 0 selects 1/sqrt(d) */
+  const int32_t* seq_lens; /* device [batch]; NULL means every L_b = max_kv */
+  int64_t q_strides[3];    /* q:     [b, t, head]  strides in elements */
+  int64_t k_strides[3];    /* k:     [b, token, kv head] */
+  int64_t v_strides[3];    /* v:     [b, token, kv head] */
+  int64_t qi_strides[3];   /* q_idx: [b, t, group] */
+  int64_t ki_strides[2];   /* k_idx: [b, token] */
+  int64_t o_strides[3];    /* out:   [b, t, head] */
+} msa_params_t;
+
+/* Bytes of workspace `op` needs for these shapes (0 on invalid params).  The
+ * workspace must be 256-byte aligned.  It holds the sticky device status word,
+ * and, when the caller does not supply them, block scores and block ids, plus
+ * the split-KV partial results of the attention. */
+MSA_API size_t msa_workspace_size(const msa_params_t* params, msa_op_t op);
+
+/* Stage 1 (index branch).  For every (b, t, g):
+ *   S[beta] = max over visible tokens j of block beta of <q_idx[b,t,g,:], k_idx[b,j,:]>
+ *   (unscaled fp32 dot products of bf16 inputs; visible = j < L_b and, when causal,
+ *   j <= p; blocks with no visible token score -inf), then the top-k blocks by
+ *   (score descending, block id ascending), the own block first when forced.
+ *   block_ids receives min(topk, F) ids in ascending order followed by -1 padding,
+ *   F being the number of blocks with a visible token.
+ *   block_scores (nullable) receives S for every block (-inf past the frontier).
+ * Sources: "MiniMax goes sparse" section 1 step 1; "MiniMax M3 的 MSA ..." first layer. */
+MSA_API msa_status_t msa_index_select(const msa_params_t* params, const msa_bf16_t* q_idx,
+                              const msa_bf16_t* k_idx, int32_t* block_ids,
+                              float* block_scores, void* workspace, size_t workspace_bytes,
+                              msa_stream_t stream);
+
+/* Stage 2 (sparse branch).  For every (b, t, hq) with g = hq / G:
+ *   keys J = tokens j of the blocks in block_ids[b,t,g,:] (entries < 0 are empty
+ *   slots, any order, no repeats) with j < L_b and, when causal, j <= p;
+ *   out = softmax(scale * q . k_J^T) v_J  (fp32 softmax and accumulation, bf16 out),
+ *   lse (nullable) = log sum_j exp(scale * q . k_j); rows with no key get out = 0,
+ *   lse = -inf.  Ids >= nblk are skipped and flagged MSA_ERR_DEVICE_ASSERT.
+ * Works for prefill (n_q > 1) and decode (n_q = 1).
+ * Sources: "MiniMax goes sparse" section 1 step 2; "MiniMax M3 的 MSA ..." second layer. */
+MSA_API msa_status_t msa_sparse_attn(const msa_params_t* params, const msa_bf16_t* q,
+                             const msa_bf16_t* k, const msa_bf16_t* v,
+                             const int32_t* block_ids, msa_bf16_t* out, float* lse,
+                             void* workspace, size_t workspace_bytes, msa_stream_t stream);
+
+/* Both stages in one call: msa_index_select followed by msa_sparse_attn on its ids.
+ * block_ids, block_scores and lse are optional outputs (nullable). */
+MSA_API msa_status_t msa_forward(const msa_params_t* params, const msa_bf16_t* q, const msa_bf16_t* k,
+                         const msa_bf16_t* v, const msa_bf16_t* q_idx, const msa_bf16_t* k_idx,
+                         msa_bf16_t* out, int32_t* block_ids, float* block_scores, float* lse,
+                         void* workspace, size_t workspace_bytes, msa_stream_t stream);
+
+/* Synchronises `stream`, returns the first error a kernel recorded in this
+ * workspace since the last reset (MSA_OK if none) and clears it. */
+MSA_API msa_status_t msa_get_device_status(void* workspace, msa_stream_t stream);
+
+/* Zeroes the workspace's status word, asynchronously on `stream`.  Call it once
+ * on every new workspace before its first use (the word is sticky: kernels only
+ * ever set it, msa_get_device_status() clears it). */
+MSA_API msa_status_t msa_workspace_init(void* workspace, size_t workspace_bytes, msa_stream_t stream);
+
+/* Self-test of the device error path: launches one tiny kernel that waits, with
+ * a bound of `wait_ns` nanoseconds, on a barrier that nothing completes, so the
+ * wait runs out and records MSA_ERR_TIMEOUT in the workspace; nothing faults or
+ * hangs.  Read the result with msa_get_device_status(). */
+MSA_API msa_status_t msa_selftest_wait_timeout(void* workspace, size_t workspace_bytes, uint64_t wait_ns,
+                                       msa_stream_t stream);
+
+/* Number of kernel launches `op` makes on the stream for these shapes (its
+ * plan depends on the current device's SM count); -1 on invalid params. */
+MSA_API int msa_launch_count(const msa_params_t* params, msa_op_t op);
+
+/* A static description of a status code. */
+MSA_API const char* msa_status_string(msa_status_t status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MSA_H_ */

@@ -1,0 +1,113 @@
+"""The C ABI on a machine without a GPU: the library loads, exports every entry
+point ``include/msa.h`` declares, and rejects bad arguments on the host before
+anything is launched.  No compute call is made here."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from block_sparse_gqa_03_b200 import build as msa_build
+from block_sparse_gqa_03_b200 import msa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "msa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    msa_build.build()
+    return msa.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return re.findall(r"MSA_API\s+[\w\s\*]+?\b(msa_\w+)\s*\(", text)
+
+
+def test_header_declares_the_binding_names():
+    names = declared_functions()
+    assert sorted(names) == sorted(msa.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    for code in range(7):
+        assert msa.msa_status_string(code)
+    assert msa.msa_status_string(99) == "unknown status"
+
+
+def valid_params(**kw):
+    base = dict(batch=1, n_q=1024, max_kv=1024, H=6, h=2, d=64, d_idx=32, block=64, topk=4)
+    base.update(kw)
+    p = msa.make_params(**base)
+    p.q_strides[:] = [1024 * 6 * 64, 6 * 64, 64]
+    p.k_strides[:] = [1024 * 2 * 64, 2 * 64, 64]
+    p.v_strides[:] = [1024 * 2 * 64, 2 * 64, 64]
+    p.o_strides[:] = [1024 * 6 * 64, 6 * 64, 64]
+    p.qi_strides[:] = [1024 * 2 * 32, 2 * 32, 32]
+    p.ki_strides[:] = [1024 * 32, 32]
+    return p
+
+
+def test_workspace_size_host_only(lib):
+    p = valid_params()
+    sel = msa.msa_workspace_size(p, msa.MSA_OP_INDEX_SELECT)
+    fwd = msa.msa_workspace_size(p, msa.MSA_OP_FORWARD)
+    # status word + fp32 block scores [1, 1024, 2, 16] (+ ids for forward)
+    assert sel >= 256 + 1024 * 2 * 16 * 4
+    assert fwd >= sel + 1024 * 2 * 4 * 4
+    assert msa.msa_workspace_size(p, 7) == 0
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(H=7), msa.MSA_ERR_INVALID_ARG),          # H % h != 0
+    (dict(d=96), msa.MSA_ERR_UNSUPPORTED),
+    (dict(d_idx=48), msa.MSA_ERR_UNSUPPORTED),
+    (dict(block=48), msa.MSA_ERR_UNSUPPORTED),
+    (dict(topk=0), msa.MSA_ERR_INVALID_ARG),
+    (dict(topk=5000), msa.MSA_ERR_UNSUPPORTED),
+    (dict(n_q=2048), msa.MSA_ERR_INVALID_ARG),     # n_q > max_kv
+    (dict(H=34, h=2), msa.MSA_ERR_UNSUPPORTED),    # G = 17
+])
+def test_bad_params_rejected_before_launch(lib, bad, code):
+    p = valid_params(**bad)
+    fake = 1 << 20  # never dereferenced: validation fails first
+    rc = lib.msa_forward(ctypes.byref(p), fake, fake, fake, fake, fake, fake, None, None, None,
+                         fake, 1 << 30, None)
+    assert rc == code
+    assert msa.msa_workspace_size(p, msa.MSA_OP_FORWARD) == 0
+
+
+def test_bad_pointers_and_workspace_rejected(lib):
+    p = valid_params()
+    fake = 1 << 20
+    # null q
+    assert lib.msa_forward(ctypes.byref(p), None, fake, fake, fake, fake, fake, None, None, None,
+                           fake, 1 << 30, None) == msa.MSA_ERR_INVALID_ARG
+    # misaligned k_idx
+    assert lib.msa_index_select(ctypes.byref(p), fake, fake + 2, fake, None, fake, 1 << 30,
+                                None) == msa.MSA_ERR_INVALID_ARG
+    # workspace too small, or misaligned
+    assert lib.msa_index_select(ctypes.byref(p), fake, fake, fake, None, fake, 512,
+                                None) == msa.MSA_ERR_WORKSPACE
+    assert lib.msa_index_select(ctypes.byref(p), fake, fake, fake, None, fake + 16, 1 << 30,
+                                None) == msa.MSA_ERR_WORKSPACE
+    # stride not a multiple of 8 elements
+    p.k_strides[1] = 130
+    assert lib.msa_sparse_attn(ctypes.byref(p), fake, fake, fake, fake, fake, None, fake, 1 << 30,
+                               None) == msa.MSA_ERR_INVALID_ARG
+    assert lib.msa_selftest_wait_timeout(None, 4096, 1000, None) == msa.MSA_ERR_WORKSPACE
+    assert lib.msa_selftest_wait_timeout(fake, 4096, 0, None) == msa.MSA_ERR_INVALID_ARG
+
+
+def test_binding_fails_loudly_without_library(monkeypatch):
+    monkeypatch.setattr(msa, "LIB_PATH", "/nonexistent/libmsa.so")
+    monkeypatch.setattr(msa, "_lib", None)
+    with pytest.raises(RuntimeError, match="not built"):
+        msa.load_library()
