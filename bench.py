@@ -23,9 +23,7 @@ import argparse
 import json
 import os
 import statistics
-import subprocess
 import sys
-import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -123,57 +121,68 @@ def work_units(prob, x, ids):
 
 # ------------------------------------------------------------------- clocks
 class ClockSampler:
-    """nvidia-smi samples (200 ms) while the timed region runs."""
+    """Polls the GPU's SM clock and clock-event reasons through NVML every ~2 ms on a
+    background thread; summary() keeps the samples taken inside the timed window."""
 
-    def __init__(self, device_index: int):
-        self.idx = device_index
-        self.proc = None
-        self.path = None
+    # NVML clock-event reason bits (nvml.h)
+    REASONS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+               "hw_thermal_slowdown": 0x40}
+
+    def __init__(self, uuid: str | None):
+        self.uuid = uuid
+        self.samples = []
+        self.window = None
+        self.err = None
+        self._stop = False
+        self._thread = None
 
     def __enter__(self):
+        import threading
         try:
-            fd, self.path = tempfile.mkstemp(suffix=".csv")
-            os.close(fd)
-            q = ("index,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-                 "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-                 "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "--query-gpu=" + q, "--format=csv,noheader,nounits", "-lms", "200",
-                 "-f", self.path], stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
-        except Exception:
-            self.proc = None
+            import pynvml
+            pynvml.nvmlInit()
+            h = (pynvml.nvmlDeviceGetHandleByUUID(self.uuid) if self.uuid
+                 else pynvml.nvmlDeviceGetHandleByIndex(0))
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            reasons_fn = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+        except Exception as e:  # no NVML: report it, do not guess
+            self.err = "nvml unavailable: %s" % e
+            return self
+
+        def poll():
+            while not self._stop:
+                try:
+                    self.samples.append((time.perf_counter(),
+                                         pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM),
+                                         reasons_fn(h)))
+                except Exception as e:
+                    self.err = str(e)
+                    return
+                time.sleep(0.002)
+
+        self._thread = threading.Thread(target=poll, daemon=True)
+        self._thread.start()
         return self
 
-    def __exit__(self, *exc):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except Exception:
-                self.proc.kill()
+    def mark(self, t0, t1):
+        self.window = (t0, t1)
 
-    def summary(self, uuid: str | None):
-        if self.proc is None or not self.path or not os.path.exists(self.path):
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        rows = []
-        with open(self.path) as f:
-            for line in f:
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) < 10:
-                    continue
-                if uuid and parts[1] != uuid:
-                    continue
-                rows.append(parts)
-        os.unlink(self.path)
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        sm = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
-        mx = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[6 + i] == "Active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
-                "samples": len(rows)}
+    def __exit__(self, *exc):
+        self._stop = True
+        if self._thread is not None:
+            self._thread.join(timeout=2)
+
+    def summary(self):
+        if self.err and not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [self.err]}
+        t0, t1 = self.window or (float("-inf"), float("inf"))
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        used = inside or self.samples[-3:]
+        reasons = sorted({n for _, _, r in used for n, bit in self.REASONS.items() if r & bit})
+        return {"sm_mhz": statistics.median(s[1] for s in used) if used else None,
+                "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(inside),
+                "source": "nvml, 2 ms polling, samples inside the timed region"}
 
 
 # --------------------------------------------------------------- oracle arm
@@ -309,7 +318,8 @@ def run_ours(args, prob, world, rank, local):
         uuid = "GPU-" + uuid
     barrier(world)
     torch.cuda.synchronize(dev)
-    with ClockSampler(dev.index) as clk:
+    with ClockSampler(uuid) as clk:
+        h0 = time.perf_counter()
         t_start.record(stream)
         for i in range(K):
             ev[i][0].record(stream)
@@ -320,6 +330,7 @@ def run_ours(args, prob, world, rank, local):
             ev[i][2].record(stream)
         t_end.record(stream)
         torch.cuda.synchronize(dev)
+        clk.mark(h0, time.perf_counter())
     barrier(world)
     total_ms = max_over_ranks(t_start.elapsed_time(t_end), world)
     sel_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
@@ -375,7 +386,7 @@ def run_ours(args, prob, world, rank, local):
     if prob.is_decode:
         line["tokens_per_s"] = prob.batch * world / (ms_per_step * 1e-3)
     if rank == 0:
-        line["clocks"] = clk.summary(uuid)
+        line["clocks"] = clk.summary()
         if world == 1 and not args.no_cpu_baseline:
             import oracle
             u, s, desc = oracle_sample(prob, {k: v for k, v in x.items()}, args.cpu_budget)
@@ -445,7 +456,7 @@ def run_e2e(args, prob, x, dev, world, msa, kw):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default=DEFAULT_WORKLOAD)

@@ -301,3 +301,55 @@ const char* msa_status_string(msa_status_t status) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// msa_sparse_attn_noalloc: the sparse branch for callers that cannot allocate
+// device memory.  Its split-KV partial results live in one fixed array in the
+// library's own device memory instead of a caller-provided workspace.
+namespace {
+
+// Scratch for the split-KV partials of msa_sparse_attn_noalloc.  Every GPU that
+// loads this library holds these bytes until the process exits.
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;
+__device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of g_noalloc_scratch per device.  In host code the array's
+// name is only a host-side stand-in, so the address is looked up once per
+// device (with that device current) and cached.
+void* g_noalloc_ptr[64] = {nullptr};
+
+msa_status_t noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MSA_ERR_CUDA;
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+      return MSA_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return MSA_OK;
+}
+
+}  // namespace
+
+extern "C" msa_status_t msa_sparse_attn_noalloc(const msa_params_t* params, const msa_bf16_t* q,
+                                                const msa_bf16_t* k, const msa_bf16_t* v,
+                                                const int32_t* block_ids, msa_bf16_t* out,
+                                                float* lse, msa_stream_t stream) {
+  Shape s;
+  msa_status_t rc = make_shape(params, &s);
+  if (rc != MSA_OK) return rc;
+  if ((rc = check_attn_args(s, q, k, v, out)) != MSA_OK) return rc;
+  if (block_ids == nullptr) return MSA_ERR_INVALID_ARG;
+  const size_t need = msa::attn_partial_bytes(s);
+  if (need > kNoAllocScratchBytes) return MSA_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  if ((rc = noalloc_scratch(&scratch)) != MSA_OK) return rc;
+  // The partials need no clearing: each (query, head, split) slot is written by
+  // its CTA before the combine reads it.  No status word: device-side errors are
+  // skipped, not recorded.
+  return cuda_status(msa::launch_sparse_attn(s, q, k, v, block_ids, out, lse, scratch,
+                                             kNoAllocScratchBytes, nullptr,
+                                             reinterpret_cast<cudaStream_t>(stream)));
+}

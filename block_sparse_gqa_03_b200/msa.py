@@ -35,7 +35,7 @@ MSA_OP_FORWARD = 2
 
 EXPORTED = ("msa_workspace_size", "msa_index_select", "msa_sparse_attn", "msa_forward",
             "msa_get_device_status", "msa_workspace_init", "msa_selftest_wait_timeout",
-            "msa_launch_count", "msa_status_string")
+            "msa_launch_count", "msa_sparse_attn_noalloc", "msa_status_string")
 
 
 class MsaError(RuntimeError):
@@ -89,6 +89,8 @@ def load_library():
             lib.msa_workspace_init.restype = I
             lib.msa_selftest_wait_timeout.argtypes = [P, S, ctypes.c_uint64, P]
             lib.msa_selftest_wait_timeout.restype = I
+            lib.msa_sparse_attn_noalloc.argtypes = [P, P, P, P, P, P, P, P]
+            lib.msa_sparse_attn_noalloc.restype = I
             lib.msa_launch_count.argtypes = [P, I]
             lib.msa_launch_count.restype = I
             lib.msa_status_string.argtypes = [I]
@@ -242,6 +244,24 @@ def msa_sparse_attn(q, k, v, block_ids, *, block, causal=True, seq_lens=None, so
                                           _ptr(block_ids), _ptr(out), _ptr(lse), ws.data_ptr(),
                                           ws.numel(), _stream(stream)), "msa_sparse_attn")
     return (out, lse) if return_lse else out
+
+
+def msa_sparse_attn_noalloc(q, k, v, block_ids, *, block, causal=True, seq_lens=None,
+                            softmax_scale=0.0, out=None, lse=None, stream=None):
+    """Stage 2 without a workspace (the library's fixed device scratch holds the
+    split-KV partials); for callers that cannot allocate device memory.  ``out``
+    (and ``lse``, if wanted) should be preallocated by such callers."""
+    b, n_q, H, d = q.shape
+    max_kv, h = k.shape[1], k.shape[2]
+    if out is None:
+        out = torch.empty_like(q)
+    p = make_params(batch=b, n_q=n_q, max_kv=max_kv, H=H, h=h, d=d, d_idx=32, block=block,
+                    topk=block_ids.shape[-1], causal=causal, softmax_scale=softmax_scale,
+                    seq_lens=seq_lens, q=q, k=k, v=v, out=out)
+    _check(load_library().msa_sparse_attn_noalloc(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v),
+                                                  _ptr(block_ids), _ptr(out), _ptr(lse),
+                                                  _stream(stream)), "msa_sparse_attn_noalloc")
+    return out
 
 
 def msa_forward(q, k, v, q_idx, k_idx, *, block, topk, causal=True, force_own_block=False,

@@ -154,6 +154,30 @@ MSA_API msa_status_t msa_workspace_init(void* workspace, size_t workspace_bytes,
 MSA_API msa_status_t msa_selftest_wait_timeout(void* workspace, size_t workspace_bytes, uint64_t wait_ns,
                                        msa_stream_t stream);
 
+/* msa_sparse_attn without a workspace, for callers that cannot allocate device
+ * memory: code running where an allocation is forbidden or would stall the GPU
+ * (an inference engine's enqueue path, a real-time loop, a host framework that
+ * owns every allocation), which therefore cannot provide the workspace that
+ * msa_sparse_attn needs for its split-KV partial results.  This entry point has
+ * no counterpart in the pages; it is a deployment convenience.
+ *   - Same arguments and results as msa_sparse_attn, minus the workspace.  The
+ *     caller still passes inputs and outputs.
+ *   - The partials live in one fixed 16 MiB array in the library's own device
+ *     memory (every GPU that loads libmsa.so holds it until the process exits).
+ *     Shapes whose partials do not fit (batch * n_q * H * splits * (d + 1) * 4
+ *     bytes) return MSA_ERR_WORKSPACE; problems that run in one split (prefill)
+ *     need none.
+ *   - All calls share that array: calls whose work overlaps on the GPU (two
+ *     streams, or two host threads) race and must be serialised by the caller.
+ *   - The first call on a device looks up the array's device address; make that
+ *     first call before any stream capture.
+ *   - Device-side precondition failures (ids >= nblk, lengths outside
+ *     [0, max_kv]) are skipped but not recorded, as there is no status word. */
+MSA_API msa_status_t msa_sparse_attn_noalloc(const msa_params_t* params, const msa_bf16_t* q,
+                                             const msa_bf16_t* k, const msa_bf16_t* v,
+                                             const int32_t* block_ids, msa_bf16_t* out,
+                                             float* lse, msa_stream_t stream);
+
 /* Number of kernel launches `op` makes on the stream for these shapes (its
  * plan depends on the current device's SM count); -1 on invalid params. */
 MSA_API int msa_launch_count(const msa_params_t* params, msa_op_t op);

@@ -1,0 +1,63 @@
+"""msa_sparse_attn_noalloc: the sparse branch for callers that cannot allocate
+device memory (the split-KV partials live in the library's fixed device array).
+
+Checked through the C ABI against msa_sparse_attn (which takes a caller
+workspace) on a decode problem that runs in several KV splits, so the fixed
+scratch is really used, on two calls in a row.  This file is collected last.
+"""
+
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_gqa_03_b200 import msa
+from block_sparse_gqa_03_b200.inputs import Problem, make_inputs
+from msa_check import OUT_MAX_ABS, OUT_MEAN_ABS
+
+pytestmark = pytest.mark.gpu
+
+
+def test_noalloc_matches_workspace_entry_point_twice():
+    prob = Problem("noalloc", batch=4, n_q=1, max_kv=65536, H=64, h=8, d=128, d_idx=128,
+                   block=64, topk=256, causal=True, seed=120, len_range=(30000, 65536))
+    x = make_inputs(prob, device="cuda")
+    kw = dict(block=prob.block, causal=True, seq_lens=x["seq_lens"])
+    ids = msa.msa_index_select(x["q_idx"], x["k_idx"], topk=prob.topk, **kw)
+    ref, ref_lse = msa.msa_sparse_attn(x["q"], x["k"], x["v"], ids, return_lse=True, **kw)
+    p = msa.make_params(batch=prob.batch, n_q=1, max_kv=prob.max_kv, H=prob.H, h=prob.h,
+                        d=prob.d, d_idx=prob.d_idx, block=prob.block, topk=prob.topk,
+                        seq_lens=x["seq_lens"], q=x["q"], k=x["k"], v=x["v"], out=ref)
+    assert msa.msa_launch_count(p, msa.MSA_OP_SPARSE_ATTN) == 2  # split KV + combine
+    lib = msa.load_library()
+    stream = torch.cuda.current_stream().cuda_stream or None
+    for _ in range(2):
+        out = torch.full_like(ref, float("nan"))
+        lse = torch.full_like(ref_lse, float("nan"))
+        rc = lib.msa_sparse_attn_noalloc(ctypes.byref(p), x["q"].data_ptr(), x["k"].data_ptr(),
+                                         x["v"].data_ptr(), ids.data_ptr(), out.data_ptr(),
+                                         lse.data_ptr(), stream)
+        assert rc == msa.MSA_OK, msa.msa_status_string(rc)
+        torch.cuda.synchronize()
+        err = (out.float() - ref.float()).abs()
+        assert float(err.max()) <= OUT_MAX_ABS and float(err.mean()) <= OUT_MEAN_ABS
+        assert np.allclose(lse.cpu().numpy(), ref_lse.cpu().numpy(), atol=2e-3)
+
+
+def test_noalloc_rejects_partials_beyond_its_scratch():
+    # topk = 4096 forces at least 8 KV splits; 64 sequences x 256 heads x 8 splits
+    # x 129 floats is about 67 MB of partials, beyond the fixed 16 MiB.  The shape
+    # is rejected on the host, before any launch.
+    B, L, H, h, d = 64, 4096, 256, 16, 128
+    p = msa.make_params(batch=B, n_q=1, max_kv=L, H=H, h=h, d=d, d_idx=128, block=64, topk=4096)
+    p.q_strides[:] = [H * d, H * d, d]
+    p.k_strides[:] = [L * h * d, h * d, d]
+    p.v_strides[:] = [L * h * d, h * d, d]
+    p.o_strides[:] = [H * d, H * d, d]
+    assert msa.msa_launch_count(p, msa.MSA_OP_SPARSE_ATTN) == 2
+    fake = torch.empty(16, device="cuda")
+    rc = msa.load_library().msa_sparse_attn_noalloc(ctypes.byref(p), fake.data_ptr(),
+                                                    fake.data_ptr(), fake.data_ptr(),
+                                                    fake.data_ptr(), fake.data_ptr(), None, None)
+    assert rc == msa.MSA_ERR_WORKSPACE
