@@ -343,7 +343,7 @@ def run_ours(args, prob, world, rank, local):
 
     # End to end through the public API: inputs from pinned host memory, the
     # result read back, every step.
-    e2e = run_e2e(args, prob, x, dev, world, msa, kw)
+    e2e = None if args.no_e2e else run_e2e(args, prob, x, dev, world, msa, kw)
 
     p_sel = msa.make_params(batch=prob.batch, n_q=prob.n_q, max_kv=prob.max_kv, H=prob.H,
                             h=prob.h, d=prob.d, d_idx=prob.d_idx, block=prob.block,
@@ -462,10 +462,15 @@ def main():
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default=DEFAULT_WORKLOAD)
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="override the workload's batch (for small profiling captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     prob = WORKLOADS[args.workload]
+    if args.batch:
+        prob = prob.with_(batch=args.batch)
     world, rank, local = dist_setup(args)
     try:
         if args.impl == "reference":

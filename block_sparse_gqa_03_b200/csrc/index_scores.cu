@@ -26,7 +26,7 @@ struct ScanArgs {
   const uint16_t* k_idx;
   int64_t qi_s0, qi_s1, qi_s2, ki_s0, ki_s1;
   const int32_t* seq_lens;
-  int n_q, max_kv, h, block, nblk, causal, qt, ntiles;
+  int batch, n_q, max_kv, h, block, nblk, causal, qt, ntiles;
   float* scores;
   int fill_tail;
   DeviceStatus* st;
@@ -34,19 +34,12 @@ struct ScanArgs {
 
 constexpr int kScanWarps = 8;
 
+// Loads the B fragments (index-query columns) of this lane: column c = nt*8 + r,
+// dims [32kc + 8q, 32kc + 8q + 8).  Columns past `ncols` or t >= n_q are zero.
 template <int DI, int NT>
-__global__ void __launch_bounds__(kScanWarps * 32) index_scan_kernel(ScanArgs a) {
-  constexpr int KC = DI / 32;  // 32-dim chunks of the index head dim
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int r = lane >> 2, q = lane & 3;
-  const int tile = blockIdx.x % a.ntiles;
-  const int b = blockIdx.x / a.ntiles;
-  const int t0 = tile * a.qt;
-  const int L = kv_length(a.seq_lens, b, a.max_kv, a.st);
+__device__ __forceinline__ void load_columns(const ScanArgs& a, int b, int t0, int r, int q,
+                                             uint4 (&bq)[NT][DI / 32]) {
   const int ncols = a.qt * a.h;
-
-  // B fragments: column c = nt*8 + r; dims [32kc + 8q, 32kc + 8q + 8) of its index query.
-  uint4 bq[NT][KC];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
     const int c = nt * 8 + r;
@@ -54,9 +47,107 @@ __global__ void __launch_bounds__(kScanWarps * 32) index_scan_kernel(ScanArgs a)
     const bool ok = c < ncols && t < a.n_q;
     const uint16_t* src = a.q_idx + b * a.qi_s0 + (int64_t)t * a.qi_s1 + g * a.qi_s2 + 8 * q;
 #pragma unroll
-    for (int kc = 0; kc < KC; ++kc) bq[nt][kc] = ok ? ld_u4(src + 32 * kc) : make_uint4(0, 0, 0, 0);
+    for (int kc = 0; kc < DI / 32; ++kc)
+      bq[nt][kc] = ok ? ld_u4(src + 32 * kc) : make_uint4(0, 0, 0, 0);
   }
-  // Accumulator columns of this lane: c = nt*8 + 2q + e.  Visible tokens j < lim.
+}
+
+// Block max of the visible token scores of block `beta` for this lane's
+// accumulator columns (c = nt*8 + 2q + e, visible tokens j < lim[nt][e]),
+// reduced over the warp: every lane returns the maxima of its own columns.
+template <int DI, int NT>
+__device__ __forceinline__ void block_max(const ScanArgs& a, const uint16_t* kb, int L, int beta,
+                                          int r, const uint4 (&bq)[NT][DI / 32],
+                                          const int (&lim)[NT][2], float (&cm)[NT][2]) {
+  constexpr int KC = DI / 32;
+  const float ninf = -__int_as_float(0x7f800000);
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) cm[nt][0] = cm[nt][1] = ninf;
+  const int nmt = a.block / 16;
+#pragma unroll 2
+  for (int mt = 0; mt < nmt; ++mt) {
+    const int jl = beta * a.block + mt * 16 + r, jh = jl + 8;
+    uint4 X[KC], Y[KC];
+#pragma unroll
+    for (int kc = 0; kc < KC; ++kc) {
+      X[kc] = jl < L ? ld_stream_u4(kb + (int64_t)jl * a.ki_s1 + 32 * kc) : make_uint4(0, 0, 0, 0);
+      Y[kc] = jh < L ? ld_stream_u4(kb + (int64_t)jh * a.ki_s1 + 32 * kc) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int kc = 0; kc < KC; ++kc) {
+        mma_bf16_16816(acc, X[kc].x, Y[kc].x, X[kc].y, Y[kc].y, bq[nt][kc].x, bq[nt][kc].y);
+        mma_bf16_16816(acc, X[kc].z, Y[kc].z, X[kc].w, Y[kc].w, bq[nt][kc].z, bq[nt][kc].w);
+      }
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        cm[nt][e] = fmaxf(cm[nt][e], jl < lim[nt][e] ? acc[e] : ninf);
+        cm[nt][e] = fmaxf(cm[nt][e], jh < lim[nt][e] ? acc[2 + e] : ninf);
+      }
+    }
+  }
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      float v = cm[nt][e];
+      v = warp_max_xor(v, 4);
+      v = warp_max_xor(v, 8);
+      v = warp_max_xor(v, 16);
+      cm[nt][e] = v;
+    }
+}
+
+// Decode (one query per sequence): one warp per (sequence, block) item, so the
+// grid is many short CTAs and no wave leaves the GPU half idle.  The columns are
+// the h groups of the sequence's query.
+template <int DI, int NT>
+__global__ void __launch_bounds__(kScanWarps * 32) index_scan_decode_kernel(ScanArgs a) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int r = lane >> 2, q = lane & 3;
+  const int64_t item = (int64_t)blockIdx.x * kScanWarps + warp;
+  const int b = (int)(item / a.nblk), beta = (int)(item % a.nblk);
+  if (b >= a.batch) return;
+  const int L = kv_length(a.seq_lens, b, a.max_kv, a.st);
+  const int nb_b = (L + a.block - 1) / a.block;
+  const float ninf = -__int_as_float(0x7f800000);
+  if (beta >= nb_b) {
+    if (a.fill_tail && lane < a.h) a.scores[((int64_t)b * a.h + lane) * a.nblk + beta] = ninf;
+    return;
+  }
+  uint4 bq[NT][DI / 32];
+  load_columns<DI, NT>(a, b, 0, r, q, bq);
+  int lim[NT][2];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) lim[nt][0] = lim[nt][1] = L;  // p = L - 1: all j < L visible
+  float cm[NT][2];
+  block_max<DI, NT>(a, a.k_idx + b * a.ki_s0 + 8 * q, L, beta, r, bq, lim, cm);
+  if (r == 0) {
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int g = nt * 8 + 2 * q + e;
+        if (g < a.h) a.scores[((int64_t)b * a.h + g) * a.nblk + beta] = cm[nt][e];
+      }
+  }
+}
+
+// Prefill: a CTA per (sequence, tile of queries); the columns are the tile's
+// (query, group) pairs and each warp walks the blocks up to the tile's frontier.
+template <int DI, int NT>
+__global__ void __launch_bounds__(kScanWarps * 32) index_scan_kernel(ScanArgs a) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int r = lane >> 2, q = lane & 3;
+  const int tile = blockIdx.x % a.ntiles;
+  const int b = blockIdx.x / a.ntiles;
+  const int t0 = tile * a.qt;
+  const int L = kv_length(a.seq_lens, b, a.max_kv, a.st);
+  const int ncols = a.qt * a.h;
+  uint4 bq[NT][DI / 32];
+  load_columns<DI, NT>(a, b, t0, r, q, bq);
   int lim[NT][2];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt)
@@ -67,56 +158,17 @@ __global__ void __launch_bounds__(kScanWarps * 32) index_scan_kernel(ScanArgs a)
       const int p = L - a.n_q + t;
       lim[nt][e] = a.causal ? min(L, p + 1) : L;
     }
-
   const int t_last = min(t0 + a.qt, a.n_q) - 1;
   const int p_last = L - a.n_q + t_last;
   const int nb_b = (L + a.block - 1) / a.block;
   const int F = a.causal ? (p_last < 0 ? 0 : min(nb_b, p_last / a.block + 1)) : nb_b;
-
   const int nw = gridDim.y * kScanWarps;
   const int wid = blockIdx.y * kScanWarps + warp;
   const uint16_t* kb = a.k_idx + b * a.ki_s0 + 8 * q;
-  const int nmt = a.block / 16;
   const float ninf = -__int_as_float(0x7f800000);
-
   for (int beta = wid; beta < F; beta += nw) {
     float cm[NT][2];
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) cm[nt][0] = cm[nt][1] = ninf;
-#pragma unroll 2
-    for (int mt = 0; mt < nmt; ++mt) {
-      const int jl = beta * a.block + mt * 16 + r, jh = jl + 8;
-      uint4 X[KC], Y[KC];
-#pragma unroll
-      for (int kc = 0; kc < KC; ++kc) {
-        X[kc] = jl < L ? ld_stream_u4(kb + (int64_t)jl * a.ki_s1 + 32 * kc) : make_uint4(0, 0, 0, 0);
-        Y[kc] = jh < L ? ld_stream_u4(kb + (int64_t)jh * a.ki_s1 + 32 * kc) : make_uint4(0, 0, 0, 0);
-      }
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int kc = 0; kc < KC; ++kc) {
-          mma_bf16_16816(acc, X[kc].x, Y[kc].x, X[kc].y, Y[kc].y, bq[nt][kc].x, bq[nt][kc].y);
-          mma_bf16_16816(acc, X[kc].z, Y[kc].z, X[kc].w, Y[kc].w, bq[nt][kc].z, bq[nt][kc].w);
-        }
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          cm[nt][e] = fmaxf(cm[nt][e], jl < lim[nt][e] ? acc[e] : ninf);
-          cm[nt][e] = fmaxf(cm[nt][e], jh < lim[nt][e] ? acc[2 + e] : ninf);
-        }
-      }
-    }
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        float v = cm[nt][e];
-        v = warp_max_xor(v, 4);
-        v = warp_max_xor(v, 8);
-        v = warp_max_xor(v, 16);
-        cm[nt][e] = v;
-      }
+    block_max<DI, NT>(a, kb, L, beta, r, bq, lim, cm);
     if (r == 0) {
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt)
@@ -146,6 +198,12 @@ __global__ void __launch_bounds__(kScanWarps * 32) index_scan_kernel(ScanArgs a)
 
 template <int DI, int NT>
 cudaError_t run_scan(const ScanArgs& a, int batch, cudaStream_t stream) {
+  if (a.n_q == 1) {
+    const int64_t items = (int64_t)batch * a.nblk;
+    index_scan_decode_kernel<DI, NT>
+        <<<(unsigned)((items + kScanWarps - 1) / kScanWarps), kScanWarps * 32, 0, stream>>>(a);
+    return cudaGetLastError();
+  }
   const int ctas_per_row = a.ntiles * batch;
   // Spread the block range of each query tile over enough warps to fill the
   // GPU a few times over; each warp then walks its blocks with a stride.
@@ -172,6 +230,7 @@ cudaError_t launch_index_scores(const Shape& s, const uint16_t* q_idx, const uin
   a.ki_s0 = s.ki_s[0];
   a.ki_s1 = s.ki_s[1];
   a.seq_lens = s.seq_lens;
+  a.batch = s.batch;
   a.n_q = s.n_q;
   a.max_kv = s.max_kv;
   a.h = s.h;

@@ -310,7 +310,7 @@ namespace {
 
 // Scratch for the split-KV partials of msa_sparse_attn_noalloc.  Every GPU that
 // loads this library holds these bytes until the process exits.
-constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;
 __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 // Device address of g_noalloc_scratch per device.  In host code the array's
@@ -346,9 +346,9 @@ extern "C" msa_status_t msa_sparse_attn_noalloc(const msa_params_t* params, cons
   if (need > kNoAllocScratchBytes) return MSA_ERR_WORKSPACE;
   void* scratch = nullptr;
   if ((rc = noalloc_scratch(&scratch)) != MSA_OK) return rc;
-  // The partials need no clearing: each (query, head, split) slot is written by
-  // its CTA before the combine reads it.  No status word: device-side errors are
-  // skipped, not recorded.
+  // The per-row merge counters inside the scratch are zeroed on the stream before
+  // every launch; the partials themselves are always written before they are
+  // read.  No status word: device-side errors are skipped, not recorded.
   return cuda_status(msa::launch_sparse_attn(s, q, k, v, block_ids, out, lse, scratch,
                                              kNoAllocScratchBytes, nullptr,
                                              reinterpret_cast<cudaStream_t>(stream)));

@@ -6,21 +6,28 @@
 // group's top-k selection, so one load of a block serves the whole group
 // ("MiniMax M3 的 MSA ...", second layer).
 //
-// Kernel design (one CTA per (query, group, KV split)):
-//  * warp 4 is the producer: one lane streams the selected blocks' K and V tiles
-//    into a ring of shared-memory stages with TMA (4-D tensor maps over
-//    [batch, token, kv head, dim], 128-byte swizzle), completion tracked by
-//    mbarriers (bounded waits: a wait that runs out records an error and the
-//    kernel returns, it never hangs);
-//  * warps 0-3 consume: the group's G query heads are the 16 rows of a bf16
-//    tensor-core MMA tile (rows >= G are zero), S = Q K^T and O += P V run on
-//    m16n8k16 MMAs fed by ldmatrix from the swizzled tiles, with an fp32 online
-//    softmax in the exp2 domain.  Each warp takes 16-token slices of the blocks in
-//    turn and keeps its own running max / sum / output; the four are merged at
-//    the end through shared memory;
-//  * with one split the CTA writes bf16 output and the log-sum-exp; with several
-//    (decode, where a row has few queries but many blocks) it writes fp32
-//    partials that a combine kernel merges by log-sum-exp weights.
+// A "row" is one (sequence, query, group); its G query heads are the 16 rows of
+// a bf16 m16n8k16 tensor-core tile (rows >= G are zero).  Both kernels below
+// share the same engine:
+//  * one producer warp streams each selected block's K and V tiles into a ring of
+//    shared-memory stages with TMA (4-D tensor maps over [batch, token, kv head,
+//    dim], 128-byte swizzle), completion tracked by mbarriers whose waits are
+//    bounded (a wait that runs out records an error; nothing hangs);
+//  * consumer warps take 16-token slices of the blocks in turn: S = Q K^T and
+//    O += P V on MMAs fed by ldmatrix from the swizzled tiles, with an fp32
+//    online softmax in the exp2 domain; each warp keeps its own running max, sum
+//    and output, and the warps' states are merged through shared memory.
+//
+// sparse_attn_rows_kernel: one CTA per row (prefill: many rows, each with a
+// modest block list).  Writes bf16 output and the log-sum-exp directly.
+//
+// sparse_attn_stream_kernel: decode-style work, few rows with long block lists.
+// A persistent grid of one CTA per SM splits the flattened (row, slot) list into
+// equal contiguous ranges, so every SM streams the same number of blocks through
+// one pipeline that never drains.  At each row boundary the consumers merge their
+// states; a row covered by several CTAs gets one fp32 partial per CTA, and the
+// last CTA to finish the row (a per-row counter, zeroed before the launch)
+// merges them by log-sum-exp weights.
 #include "kernels.h"
 
 namespace msa {
@@ -33,117 +40,68 @@ struct AttnArgs {
   const int32_t* seq_lens;
   int n_q, max_kv, H, h, G, topk, block, nblk, causal;
   float scale_log2;
-  int splits, chunk, stages;
-  uint32_t stage_bytes, region_bytes;
+  int stages;
+  uint32_t stage_bytes, region_bytes, merge_off;
+  int list_cap;
+  // stream kernel only
+  int64_t total_slots;
+  int per, smax;
+  float* part_o;
+  float* part_lse;
+  int* counters;
   uint16_t* out;
   int64_t o_s0, o_s1, o_s2;
   float* lse;
-  float* part_o;
-  float* part_lse;
   DeviceStatus* st;
   uint64_t wait_ns;
 };
 
-constexpr int kConsumerWarps = 4;
-constexpr int kAttnThreads = (kConsumerWarps + 1) * 32;
+constexpr float kLn2 = 0.69314718055994531f;
+constexpr float kLog2e = 1.4426950408889634f;
 
 __device__ __forceinline__ uint32_t ld_b32(const uint16_t* p) {
   return *reinterpret_cast<const uint32_t*>(p);
 }
 
+__device__ __forceinline__ float neg_inf() { return -__int_as_float(0x7f800000); }
+
+// Geometry of one row: sequence b, query t, group g, and the visible-token bound.
+struct RowGeo {
+  int b, t, g, bt, lim;
+};
+
+__device__ __forceinline__ RowGeo row_geo(const AttnArgs& a, int64_t rowg) {
+  RowGeo r;
+  r.g = (int)(rowg % a.h);
+  r.bt = (int)(rowg / a.h);
+  r.t = r.bt % a.n_q;
+  r.b = r.bt / a.n_q;
+  const int L = kv_length(a.seq_lens, r.b, a.max_kv, a.st);
+  const int p = L - a.n_q + r.t;
+  r.lim = a.causal ? min(L, p + 1) : L;  // visible tokens: j < lim
+  return r;
+}
+
+// Running softmax state of one warp: rows r and r + 8 of the 16-row tile.
 template <int D>
-__global__ void __launch_bounds__(kAttnThreads, 1)
-    sparse_attn_kernel(const __grid_constant__ CUtensorMap tmk,
-                       const __grid_constant__ CUtensorMap tmv, AttnArgs a) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
-  const uint32_t sbase = smem_u32(smem);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + a.region_bytes);
-  int32_t* list = reinterpret_cast<int32_t*>(bars + 2 * a.stages);
-  int32_t* n_list = list + a.chunk;
-  const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + a.stages);
-
-  // After a timed-out wait anywhere in this launch, the remaining CTAs stop early.
-  if (status_failed(a.st)) return;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int rowg = blockIdx.x;  // ((b * n_q) + t) * h + g
-  const int g = rowg % a.h;
-  const int bt = rowg / a.h;
-  const int t = bt % a.n_q, b = bt / a.n_q;
-  const int split = blockIdx.y;
-  const int BLK = a.block;
-  const int L = kv_length(a.seq_lens, b, a.max_kv, a.st);
-  const int p = L - a.n_q + t;
-  const int lim = a.causal ? min(L, p + 1) : L;  // visible tokens: j < lim
-  const int nsub = BLK / 16;
-  const uint32_t half_bytes = (uint32_t)BLK * 128u;
-  constexpr int NH = D / 64;  // 128-byte halves of a row
-
-  if (tid == 0) {
-    for (int s = 0; s < a.stages; ++s) {
-      mbar_init(full0 + 8 * s, 1);
-      mbar_init(empty0 + 8 * s, min(kConsumerWarps, nsub));
-    }
-    fence_mbar_init();
-  }
-  if (warp == kConsumerWarps) {
-    // Compact this split's slots into the list of blocks that hold a visible token.
-    const int s0 = split * a.chunk, s1 = min(a.topk, s0 + a.chunk);
-    const int32_t* row_ids = a.ids + (int64_t)rowg * a.topk;
-    const unsigned lt = (1u << lane) - 1u;
-    int n = 0;
-    for (int base = s0; base < s1; base += 32) {
-      const int i = base + lane;
-      const int beta = i < s1 ? row_ids[i] : -1;
-      const bool bad = beta >= a.nblk;
-      if (bad) record_error(a.st, kErrDeviceAssert, (uint32_t)rowg);
-      const bool keep = beta >= 0 && !bad && (int64_t)beta * BLK < lim;
-      const unsigned msk = __ballot_sync(0xffffffffu, keep);
-      if (keep) list[n + __popc(msk & lt)] = beta;
-      n += __popc(msk);
-    }
-    if (lane == 0) *n_list = n;
-  }
-  __syncthreads();
-  const int n = *n_list;
-
-  if (warp == kConsumerWarps) {
-    if (lane == 0 && n > 0) {
-      prefetch_tensormap(&tmk);
-      prefetch_tensormap(&tmv);
-      int issued = 0;
-      for (int i = 0; i < n; ++i) {
-        const int s = i % a.stages;
-        if (i >= a.stages &&
-            !mbar_wait_bounded(empty0 + 8 * s, ((i / a.stages) - 1) & 1, a.st, 1u, a.wait_ns))
-          break;
-        const uint32_t full = full0 + 8 * s;
-        mbar_arrive_expect_tx(full, a.stage_bytes);
-        const uint32_t kdst = sbase + (uint32_t)s * a.stage_bytes;
-        const uint32_t vdst = kdst + NH * half_bytes;
-        const int tok = list[i] * BLK;
-#pragma unroll
-        for (int hh = 0; hh < NH; ++hh) {
-          tma_load_4d(kdst + hh * half_bytes, &tmk, full, hh * 64, g, tok, b);
-          tma_load_4d(vdst + hh * half_bytes, &tmv, full, hh * 64, g, tok, b);
-        }
-        ++issued;
-      }
-      // Drain: make sure no copy into this CTA's shared memory is in flight at exit.
-      for (int i = max(0, issued - a.stages); i < issued; ++i)
-        mbar_wait_bounded(full0 + 8 * (i % a.stages), (i / a.stages) & 1, a.st, 2u, a.wait_ns);
-    }
-    return;
-  }
-
-  // ------------------------------------------------------------ consumers
-  const int r = lane >> 2, q4 = lane & 3;
-  const float ninf = -__int_as_float(0x7f800000);
+struct WarpState {
   uint32_t qa[D / 16][4];
-  {
+  float o[D / 8][4];
+  float m_a, m_b, l_a, l_b;
+
+  __device__ __forceinline__ void reset() {
+#pragma unroll
+    for (int i = 0; i < D / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+    m_a = m_b = neg_inf();
+    l_a = l_b = 0.f;
+  }
+
+  // A-operand fragments of the group's G query heads (rows >= G are zero).
+  __device__ __forceinline__ void load_q(const AttnArgs& a, const RowGeo& rg, int lane) {
+    const int r = lane >> 2, q4 = lane & 3;
     const bool vlo = r < a.G, vhi = r + 8 < a.G;
-    const uint16_t* qb = a.q + b * a.q_s0 + (int64_t)t * a.q_s1 + (int64_t)(g * a.G) * a.q_s2 + 2 * q4;
+    const uint16_t* qb = a.q + rg.b * a.q_s0 + (int64_t)rg.t * a.q_s1 +
+                         (int64_t)(rg.g * a.G) * a.q_s2 + 2 * q4;
     const uint16_t* qlo = qb + (int64_t)r * a.q_s2;
     const uint16_t* qhi = qb + (int64_t)(r + 8) * a.q_s2;
 #pragma unroll
@@ -154,206 +112,442 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       qa[kk][3] = vhi ? ld_b32(qhi + 16 * kk + 8) : 0u;
     }
   }
-  float o[D / 8][4];
-#pragma unroll
-  for (int i = 0; i < D / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
-  float m_a = ninf, m_b = ninf, l_a = 0.f, l_b = 0.f;
 
-  for (int i = 0; i < n; ++i) {
-    const int u0 = i * nsub;
-    const int st0 = (warp - (u0 & 3) + 4) & 3;  // first slice of block i owned by this warp
-    if (st0 >= nsub) continue;
-    const int s = i % a.stages;
-    if (!mbar_wait_bounded(full0 + 8 * s, (i / a.stages) & 1, a.st, 3u, a.wait_ns)) break;
-    const uint32_t kbase = sbase + (uint32_t)s * a.stage_bytes;
-    const uint32_t vbase = kbase + NH * half_bytes;
-    const int beta = list[i];
-    bool wrote_smem = false;
-    for (int st = st0; st < nsub; st += kConsumerWarps) {
-      const int j0 = beta * BLK + st * 16;
-      if (j0 >= lim) continue;
-      const int tok = st * 16;
-      if (j0 + 16 > lim) {
-        // Tokens j >= lim of this slice may be uninitialised memory: zero their V rows.
-        const int r0 = lim - j0;
-        const int cnt = (16 - r0) * 8 * NH;
-        uint8_t* vrow = smem + (vbase - sbase);
-        for (int x = lane; x < cnt; x += 32) {
-          const int hh = x / ((16 - r0) * 8);
-          const int rem = x % ((16 - r0) * 8);
-          const int row = tok + r0 + rem / 8;
-          *reinterpret_cast<uint4*>(vrow + hh * half_bytes + row * 128 + (rem % 8) * 16) =
-              make_uint4(0, 0, 0, 0);
-        }
-        wrote_smem = true;
-        __syncwarp();
+  // One 16-token slice (rows `tok`.. of the stage tiles, absolute first token j0).
+  __device__ __forceinline__ void attend(const AttnArgs& a, uint8_t* smem, uint32_t sbase,
+                                         uint32_t kbase, uint32_t vbase, uint32_t half_bytes,
+                                         int tok, int j0, int lim, int lane, bool& wrote_smem) {
+    constexpr int NH = D / 64;
+    const int q4 = lane & 3;
+    const float ninf = neg_inf();
+    if (j0 + 16 > lim) {
+      // Tokens j >= lim of this slice may be uninitialised memory: zero their V rows
+      // so that a zero probability never meets a non-finite value.
+      const int r0 = lim - j0;
+      const int per_h = (16 - r0) * 8;
+      uint8_t* vrow = smem + (vbase - sbase);
+      for (int x = lane; x < per_h * NH; x += 32) {
+        const int hh = x / per_h, rem = x % per_h;
+        const int row = tok + r0 + rem / 8;
+        *reinterpret_cast<uint4*>(vrow + hh * half_bytes + row * 128 + (rem % 8) * 16) =
+            make_uint4(0, 0, 0, 0);
       }
-      float sc[2][4];
+      wrote_smem = true;
+      __syncwarp();
+    }
+    float sc[2][4];
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
-      {
-        const int mi = lane >> 3, rr = lane & 7;
-        const uint32_t row = tok + (mi >> 1) * 8 + rr;
+    for (int nt = 0; nt < 2; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+    {
+      const int mi = lane >> 3, rr = lane & 7;
+      const uint32_t row = tok + (mi >> 1) * 8 + rr;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t chunk = (kk & 3) * 2 + (mi & 1);
-          uint32_t k0, k1, k2, k3;
-          ldmatrix_x4(kbase + (kk >> 2) * half_bytes + swz128(row, chunk), k0, k1, k2, k3);
-          mma_bf16_16816(sc[0], qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3], k0, k1);
-          mma_bf16_16816(sc[1], qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3], k2, k3);
-        }
-      }
-      float mx_a = ninf, mx_b = ninf;
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const bool ok = j0 + nt * 8 + 2 * q4 + e < lim;
-          sc[nt][e] = ok ? sc[nt][e] * a.scale_log2 : ninf;
-          sc[nt][2 + e] = ok ? sc[nt][2 + e] * a.scale_log2 : ninf;
-          mx_a = fmaxf(mx_a, sc[nt][e]);
-          mx_b = fmaxf(mx_b, sc[nt][2 + e]);
-        }
-      mx_a = warp_max_xor(warp_max_xor(mx_a, 1), 2);
-      mx_b = warp_max_xor(warp_max_xor(mx_b, 1), 2);
-      const float mn_a = fmaxf(m_a, mx_a), mn_b = fmaxf(m_b, mx_b);
-      const float c_a = exp2f(m_a - mn_a), c_b = exp2f(m_b - mn_b);
-      m_a = mn_a;
-      m_b = mn_b;
-      float ps_a = 0.f, ps_b = 0.f;
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          sc[nt][e] = exp2f(sc[nt][e] - mn_a);
-          sc[nt][2 + e] = exp2f(sc[nt][2 + e] - mn_b);
-          ps_a += sc[nt][e];
-          ps_b += sc[nt][2 + e];
-        }
-      l_a = l_a * c_a + ps_a;
-      l_b = l_b * c_b + ps_b;
-#pragma unroll
-      for (int i2 = 0; i2 < D / 8; ++i2) {
-        o[i2][0] *= c_a;
-        o[i2][1] *= c_a;
-        o[i2][2] *= c_b;
-        o[i2][3] *= c_b;
-      }
-      const uint32_t pa0 = pack_bf16(sc[0][0], sc[0][1]);
-      const uint32_t pa1 = pack_bf16(sc[0][2], sc[0][3]);
-      const uint32_t pa2 = pack_bf16(sc[1][0], sc[1][1]);
-      const uint32_t pa3 = pack_bf16(sc[1][2], sc[1][3]);
-      {
-        const int mi = lane >> 3, rr = lane & 7;
-        const uint32_t row = tok + (mi & 1) * 8 + rr;
-#pragma unroll
-        for (int c2 = 0; c2 < D / 16; ++c2) {
-          const uint32_t chunk = (c2 & 3) * 2 + (mi >> 1);
-          uint32_t v0, v1, v2, v3;
-          ldmatrix_x4_trans(vbase + (c2 >> 2) * half_bytes + swz128(row, chunk), v0, v1, v2, v3);
-          mma_bf16_16816(o[2 * c2], pa0, pa1, pa2, pa3, v0, v1);
-          mma_bf16_16816(o[2 * c2 + 1], pa0, pa1, pa2, pa3, v2, v3);
-        }
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t chunk = (kk & 3) * 2 + (mi & 1);
+        uint32_t k0, k1, k2, k3;
+        ldmatrix_x4(kbase + (kk >> 2) * half_bytes + swz128(row, chunk), k0, k1, k2, k3);
+        mma_bf16_16816(sc[0], qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3], k0, k1);
+        mma_bf16_16816(sc[1], qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3], k2, k3);
       }
     }
-    if (wrote_smem) fence_proxy_async_smem();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(empty0 + 8 * s);
+    float mx_a = ninf, mx_b = ninf;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const bool ok = j0 + nt * 8 + 2 * q4 + e < lim;
+        sc[nt][e] = ok ? sc[nt][e] * a.scale_log2 : ninf;
+        sc[nt][2 + e] = ok ? sc[nt][2 + e] * a.scale_log2 : ninf;
+        mx_a = fmaxf(mx_a, sc[nt][e]);
+        mx_b = fmaxf(mx_b, sc[nt][2 + e]);
+      }
+    mx_a = warp_max_xor(warp_max_xor(mx_a, 1), 2);
+    mx_b = warp_max_xor(warp_max_xor(mx_b, 1), 2);
+    const float mn_a = fmaxf(m_a, mx_a), mn_b = fmaxf(m_b, mx_b);
+    const float c_a = exp2f(m_a - mn_a), c_b = exp2f(m_b - mn_b);
+    m_a = mn_a;
+    m_b = mn_b;
+    float ps_a = 0.f, ps_b = 0.f;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        sc[nt][e] = exp2f(sc[nt][e] - mn_a);
+        sc[nt][2 + e] = exp2f(sc[nt][2 + e] - mn_b);
+        ps_a += sc[nt][e];
+        ps_b += sc[nt][2 + e];
+      }
+    l_a = l_a * c_a + ps_a;
+    l_b = l_b * c_b + ps_b;
+#pragma unroll
+    for (int i2 = 0; i2 < D / 8; ++i2) {
+      o[i2][0] *= c_a;
+      o[i2][1] *= c_a;
+      o[i2][2] *= c_b;
+      o[i2][3] *= c_b;
+    }
+    const uint32_t pa0 = pack_bf16(sc[0][0], sc[0][1]);
+    const uint32_t pa1 = pack_bf16(sc[0][2], sc[0][3]);
+    const uint32_t pa2 = pack_bf16(sc[1][0], sc[1][1]);
+    const uint32_t pa3 = pack_bf16(sc[1][2], sc[1][3]);
+    const int mi = lane >> 3, rr = lane & 7;
+    const uint32_t row = tok + (mi & 1) * 8 + rr;
+#pragma unroll
+    for (int c2 = 0; c2 < D / 16; ++c2) {
+      const uint32_t chunk = (c2 & 3) * 2 + (mi >> 1);
+      uint32_t v0, v1, v2, v3;
+      ldmatrix_x4_trans(vbase + (c2 >> 2) * half_bytes + swz128(row, chunk), v0, v1, v2, v3);
+      mma_bf16_16816(o[2 * c2], pa0, pa1, pa2, pa3, v0, v1);
+      mma_bf16_16816(o[2 * c2 + 1], pa0, pa1, pa2, pa3, v2, v3);
+    }
   }
-  l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
-  l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
-  l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
-  l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
 
-  // ------------------------------------------- merge the four warps' states
-  asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
-  float* mo = reinterpret_cast<float*>(smem);           // [4][16][D]
-  float* mm = mo + kConsumerWarps * 16 * D;              // [4][16]
-  float* ml = mm + kConsumerWarps * 16;                  // [4][16]
-  {
+  // Stores this warp's state in the merge buffer: o [16][D], m [16], l [16].
+  __device__ __forceinline__ void stash(float* mo, float* mm, float* ml, int warp, int lane) {
+    const int r = lane >> 2, q4 = lane & 3;
+    float la = l_a, lb = l_b;
+    la += __shfl_xor_sync(0xffffffffu, la, 1);
+    la += __shfl_xor_sync(0xffffffffu, la, 2);
+    lb += __shfl_xor_sync(0xffffffffu, lb, 1);
+    lb += __shfl_xor_sync(0xffffffffu, lb, 2);
     float* mw = mo + warp * 16 * D;
 #pragma unroll
     for (int nt = 0; nt < D / 8; ++nt) {
       const int c = nt * 8 + 2 * q4;
-      mw[r * D + c] = o[nt][0];
-      mw[r * D + c + 1] = o[nt][1];
-      mw[(r + 8) * D + c] = o[nt][2];
-      mw[(r + 8) * D + c + 1] = o[nt][3];
+      *reinterpret_cast<float2*>(mw + r * D + c) = make_float2(o[nt][0], o[nt][1]);
+      *reinterpret_cast<float2*>(mw + (r + 8) * D + c) = make_float2(o[nt][2], o[nt][3]);
     }
     if (q4 == 0) {
       mm[warp * 16 + r] = m_a;
       mm[warp * 16 + r + 8] = m_b;
-      ml[warp * 16 + r] = l_a;
-      ml[warp * 16 + r + 8] = l_b;
+      ml[warp * 16 + r] = la;
+      ml[warp * 16 + r + 8] = lb;
     }
   }
-  asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
-  const float kLn2 = 0.69314718055994531f;
-  for (int x = tid; x < a.G * D; x += kConsumerWarps * 32) {
-    const int row = x / D, dim = x % D;
-    float M = ninf;
+};
+
+// Merge of NC warp states for tile row `row` and dim `dim`: normalised output
+// and natural-log LSE (-inf and 0 when no key was seen).
+template <int D, int NC>
+__device__ __forceinline__ void merge_warps(const float* mo, const float* mm, const float* ml,
+                                            int row, int dim, float& val, float& lsev) {
+  const float ninf = neg_inf();
+  float M = ninf;
 #pragma unroll
-    for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, mm[w * 16 + row]);
-    float val = 0.f, lsev = ninf;
-    if (M != ninf) {
-      float wsum = 0.f, acc = 0.f;
+  for (int w = 0; w < NC; ++w) M = fmaxf(M, mm[w * 16 + row]);
+  val = 0.f;
+  lsev = ninf;
+  if (M == ninf) return;
+  float wsum = 0.f, acc = 0.f;
 #pragma unroll
-      for (int w = 0; w < kConsumerWarps; ++w) {
-        const float f = exp2f(mm[w * 16 + row] - M);
-        wsum += f * ml[w * 16 + row];
-        acc += f * mo[(w * 16 + row) * D + dim];
+  for (int w = 0; w < NC; ++w) {
+    const float f = exp2f(mm[w * 16 + row] - M);
+    wsum += f * ml[w * 16 + row];
+    acc += f * mo[(w * 16 + row) * D + dim];
+  }
+  val = acc / wsum;
+  lsev = (M + log2f(wsum)) * kLn2;
+}
+
+__device__ __forceinline__ void consumer_sync(int nthreads) {
+  asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
+}
+
+// Producer: streams the K and V tiles of list entries [0, n) into the stage ring.
+// Each entry is (block id in the low 16 bits, row offset in the high bits); the
+// row supplies the sequence and the KV head.  Waits are bounded; before leaving,
+// the producer waits for its copies still in flight.
+template <int D>
+__device__ __forceinline__ void produce(const AttnArgs& a, const CUtensorMap* tmk,
+                                        const CUtensorMap* tmv, const int32_t* list, int n,
+                                        int64_t row0, uint32_t sbase, uint32_t full0,
+                                        uint32_t empty0) {
+  constexpr int NH = D / 64;
+  const uint32_t half_bytes = (uint32_t)a.block * 128u;
+  prefetch_tensormap(tmk);
+  prefetch_tensormap(tmv);
+  int issued = 0;
+  for (int i = 0; i < n; ++i) {
+    const int s = i % a.stages;
+    if (i >= a.stages &&
+        !mbar_wait_bounded(empty0 + 8 * s, ((i / a.stages) - 1) & 1, a.st, 1u, a.wait_ns))
+      break;
+    const uint32_t full = full0 + 8 * s;
+    mbar_arrive_expect_tx(full, a.stage_bytes);
+    const uint32_t kdst = sbase + (uint32_t)s * a.stage_bytes;
+    const uint32_t vdst = kdst + NH * half_bytes;
+    const int e = list[i];
+    const int64_t rowg = row0 + (e >> 16);
+    const int g = (int)(rowg % a.h);
+    const int b = (int)(rowg / a.h) / a.n_q;
+    const int tok = (e & 0xffff) * a.block;
+#pragma unroll
+    for (int hh = 0; hh < NH; ++hh) {
+      tma_load_4d(kdst + hh * half_bytes, tmk, full, hh * 64, g, tok, b);
+      tma_load_4d(vdst + hh * half_bytes, tmv, full, hh * 64, g, tok, b);
+    }
+    ++issued;
+  }
+  for (int i = max(0, issued - a.stages); i < issued; ++i)
+    mbar_wait_bounded(full0 + 8 * (i % a.stages), (i / a.stages) & 1, a.st, 2u, a.wait_ns);
+}
+
+// Compacts slots [s0, s1) of the flattened id array into the entry list: only
+// blocks holding a visible token are kept.  Run by one full warp; returns the count.
+__device__ __forceinline__ int compact_ids(const AttnArgs& a, int64_t s0, int64_t s1,
+                                           int64_t row0, int32_t* list, int lane) {
+  const unsigned lt = (1u << lane) - 1u;
+  int n = 0;
+  int64_t cached_row = -1;
+  int lim = 0;
+  for (int64_t base = s0; base < s1; base += 32) {
+    const int64_t i = base + lane;
+    int beta = -1;
+    int64_t rowg = row0;
+    if (i < s1) {
+      beta = a.ids[i];
+      rowg = i / a.topk;
+      if (rowg != cached_row) {
+        lim = row_geo(a, rowg).lim;
+        cached_row = rowg;
       }
-      val = acc / wsum;
-      lsev = (M + log2f(wsum)) * kLn2;
     }
-    const int hq = g * a.G + row;
-    if (a.splits == 1) {
-      a.out[b * a.o_s0 + (int64_t)t * a.o_s1 + (int64_t)hq * a.o_s2 + dim] =
-          __bfloat16_as_ushort(__float2bfloat16_rn(val));
-      if (dim == 0 && a.lse) a.lse[(int64_t)bt * a.H + hq] = lsev;
-    } else {
-      const int64_t pr = ((int64_t)bt * a.H + hq) * a.splits + split;
-      a.part_o[pr * D + dim] = val;
-      if (dim == 0) a.part_lse[pr] = lsev;
+    const bool bad = beta >= a.nblk;
+    if (bad) record_error(a.st, kErrDeviceAssert, (uint32_t)rowg);
+    const bool keep = beta >= 0 && !bad && (int64_t)beta * a.block < lim;
+    const unsigned msk = __ballot_sync(0xffffffffu, keep);
+    if (keep) list[n + __popc(msk & lt)] = beta | (int)((rowg - row0) << 16);
+    n += __popc(msk);
+  }
+  return n;
+}
+
+// ------------------------------------------------------- one CTA per row
+template <int D>
+__global__ void __launch_bounds__(5 * 32, 1)
+    sparse_attn_rows_kernel(const __grid_constant__ CUtensorMap tmk,
+                            const __grid_constant__ CUtensorMap tmv, AttnArgs a) {
+  constexpr int NC = 4;
+  if (status_failed(a.st)) return;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + a.region_bytes);
+  int32_t* list = reinterpret_cast<int32_t*>(bars + 2 * a.stages);
+  int32_t* n_list = list + a.list_cap;
+  const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + a.stages);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t rowg = blockIdx.x;
+  const int nsub = a.block / 16;
+  const uint32_t half_bytes = (uint32_t)a.block * 128u;
+
+  if (tid == 0) {
+    for (int s = 0; s < a.stages; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, min(NC, nsub));
     }
+    fence_mbar_init();
+  }
+  if (warp == NC) {
+    const int n = compact_ids(a, rowg * a.topk, (rowg + 1) * a.topk, rowg, list, lane);
+    if (lane == 0) *n_list = n;
+  }
+  __syncthreads();
+  const int n = *n_list;
+  if (warp == NC) {
+    if (lane == 0 && n > 0) produce<D>(a, &tmk, &tmv, list, n, rowg, sbase, full0, empty0);
+    return;
+  }
+  const RowGeo rg = row_geo(a, rowg);
+  WarpState<D> ws;
+  ws.reset();
+  ws.load_q(a, rg, lane);
+  for (int i = 0; i < n; ++i) {
+    const int u0 = i * nsub;
+    const int st0 = (warp - (u0 % NC) + NC) % NC;  // first slice of block i owned by this warp
+    if (st0 >= nsub) continue;
+    const int s = i % a.stages;
+    if (!mbar_wait_bounded(full0 + 8 * s, (i / a.stages) & 1, a.st, 3u, a.wait_ns)) break;
+    const uint32_t kbase = sbase + (uint32_t)s * a.stage_bytes;
+    const uint32_t vbase = kbase + (D / 64) * half_bytes;
+    const int beta = list[i] & 0xffff;
+    bool wrote = false;
+    for (int st = st0; st < nsub; st += NC) {
+      const int j0 = beta * a.block + st * 16;
+      if (j0 < rg.lim) ws.attend(a, smem, sbase, kbase, vbase, half_bytes, st * 16, j0, rg.lim, lane, wrote);
+    }
+    if (wrote) fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty0 + 8 * s);
+  }
+  // Merge the warps' states (the stages are free: every load was consumed).
+  consumer_sync(NC * 32);
+  float* mo = reinterpret_cast<float*>(smem);
+  float* mm = mo + NC * 16 * D;
+  float* ml = mm + NC * 16;
+  ws.stash(mo, mm, ml, warp, lane);
+  consumer_sync(NC * 32);
+  for (int x = tid; x < a.G * D; x += NC * 32) {
+    const int row = x / D, dim = x % D;
+    float val, lsev;
+    merge_warps<D, NC>(mo, mm, ml, row, dim, val, lsev);
+    const int hq = rg.g * a.G + row;
+    a.out[rg.b * a.o_s0 + (int64_t)rg.t * a.o_s1 + (int64_t)hq * a.o_s2 + dim] =
+        __bfloat16_as_ushort(__float2bfloat16_rn(val));
+    if (dim == 0 && a.lse) a.lse[(int64_t)rg.bt * a.H + hq] = lsev;
   }
 }
 
-// Log-sum-exp merge of the split partials of one (query, head) per CTA.
-__global__ void __launch_bounds__(128) combine_kernel(const float* part_o, const float* part_lse,
-                                                      int splits, int D, int H, int n_q,
-                                                      uint16_t* out, int64_t o_s0, int64_t o_s1,
-                                                      int64_t o_s2, float* lse) {
-  const int64_t rh = blockIdx.x;  // bt * H + hq
-  const int hq = (int)(rh % H);
-  const int64_t bt = rh / H;
-  const int t = (int)(bt % n_q);
-  const int64_t b = bt / n_q;
-  const float* pl = part_lse + rh * splits;
-  const float ninf = -__int_as_float(0x7f800000);
-  float M = ninf;
-  for (int s = 0; s < splits; ++s) M = fmaxf(M, pl[s]);
-  for (int dim = threadIdx.x; dim < D; dim += blockDim.x) {
-    float val = 0.f;
-    if (M != ninf) {
-      float den = 0.f, acc = 0.f;
-      for (int s = 0; s < splits; ++s) {
-        const float w = __expf(pl[s] - M);
-        den += w;
-        acc += w * part_o[(rh * splits + s) * D + dim];
-      }
-      val = acc / den;
+// ----------------------------------------- persistent, balanced streaming
+template <int D, int NC>
+__global__ void __launch_bounds__((NC + 1) * 32, 1)
+    sparse_attn_stream_kernel(const __grid_constant__ CUtensorMap tmk,
+                              const __grid_constant__ CUtensorMap tmv, AttnArgs a) {
+  if (status_failed(a.st)) return;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  float* mo = reinterpret_cast<float*>(smem + a.merge_off);  // [NC][16][D]
+  float* mm = mo + NC * 16 * D;                               // [NC][16]
+  float* ml = mm + NC * 16;                                   // [NC][16]
+  int* flag = reinterpret_cast<int*>(ml + NC * 16);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + a.region_bytes);
+  int32_t* list = reinterpret_cast<int32_t*>(bars + 2 * a.stages);
+  int32_t* n_list = list + a.list_cap;
+  const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + a.stages);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nsub = a.block / 16;
+  const uint32_t half_bytes = (uint32_t)a.block * 128u;
+  const int64_t c = blockIdx.x;
+  const int64_t s0 = c * a.per;
+  const int64_t s1 = min(s0 + a.per, a.total_slots);
+  if (s0 >= s1) return;
+  const int64_t r0 = s0 / a.topk, r1 = (s1 - 1) / a.topk;
+
+  if (tid == 0) {
+    for (int s = 0; s < a.stages; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, min(NC, nsub));
     }
-    out[b * o_s0 + t * o_s1 + hq * o_s2 + dim] = __bfloat16_as_ushort(__float2bfloat16_rn(val));
+    fence_mbar_init();
   }
-  if (threadIdx.x == 0 && lse) {
-    float l = ninf;
-    if (M != ninf) {
-      float den = 0.f;
-      for (int s = 0; s < splits; ++s) den += __expf(pl[s] - M);
-      l = M + __logf(den);
+  if (warp == NC) {
+    const int n = compact_ids(a, s0, s1, r0, list, lane);
+    if (lane == 0) *n_list = n;
+  }
+  __syncthreads();
+  const int n = *n_list;
+  if (warp == NC) {
+    if (lane == 0 && n > 0) produce<D>(a, &tmk, &tmv, list, n, r0, sbase, full0, empty0);
+    return;
+  }
+
+  WarpState<D> ws;
+  bool failed = false;
+  int64_t cur = r0;
+  RowGeo rg = row_geo(a, cur);
+  ws.reset();
+  ws.load_q(a, rg, lane);
+
+  // Ends the segment of row `cur` held by this CTA: merge the warps, then write
+  // the output (row entirely in this CTA) or a partial (and merge the row's
+  // partials if this CTA is the last of the row to finish).
+  auto flush = [&]() {
+    ws.stash(mo, mm, ml, warp, lane);
+    consumer_sync(NC * 32);
+    const int64_t c_first = (cur * a.topk) / a.per;
+    const int64_t c_last = ((cur + 1) * a.topk - 1) / a.per;
+    const int nseg = (int)(c_last - c_first + 1);
+    const int seg = (int)(c - c_first);
+    for (int x = tid; x < a.G * D; x += NC * 32) {
+      const int row = x / D, dim = x % D;
+      float val, lsev;
+      merge_warps<D, NC>(mo, mm, ml, row, dim, val, lsev);
+      const int hq = rg.g * a.G + row;
+      if (nseg == 1) {
+        a.out[rg.b * a.o_s0 + (int64_t)rg.t * a.o_s1 + (int64_t)hq * a.o_s2 + dim] =
+            __bfloat16_as_ushort(__float2bfloat16_rn(val));
+        if (dim == 0 && a.lse) a.lse[(int64_t)rg.bt * a.H + hq] = lsev;
+      } else {
+        const int64_t pr = ((int64_t)rg.bt * a.H + hq) * a.smax + seg;
+        a.part_o[pr * D + dim] = val;
+        if (dim == 0) a.part_lse[pr] = lsev;
+      }
     }
-    lse[rh] = l;
+    if (nseg > 1) {
+      __threadfence();
+      consumer_sync(NC * 32);
+      if (tid == 0) *flag = atomicAdd(&a.counters[cur], 1);
+      consumer_sync(NC * 32);
+      if (*flag == nseg - 1) {
+        __threadfence();
+        for (int x = tid; x < a.G * D; x += NC * 32) {
+          const int row = x / D, dim = x % D;
+          const int hq = rg.g * a.G + row;
+          const int64_t pr0 = ((int64_t)rg.bt * a.H + hq) * a.smax;
+          const float ninf = neg_inf();
+          float M = ninf;
+          for (int sp = 0; sp < nseg; ++sp) M = fmaxf(M, __ldcg(a.part_lse + pr0 + sp));
+          float val = 0.f, lsev = ninf;
+          if (M != ninf) {
+            float den = 0.f, acc = 0.f;
+            for (int sp = 0; sp < nseg; ++sp) {
+              const float w = exp2f((__ldcg(a.part_lse + pr0 + sp) - M) * kLog2e);
+              den += w;
+              acc += w * __ldcg(a.part_o + (pr0 + sp) * D + dim);
+            }
+            val = acc / den;
+            lsev = M + log2f(den) * kLn2;
+          }
+          a.out[rg.b * a.o_s0 + (int64_t)rg.t * a.o_s1 + (int64_t)hq * a.o_s2 + dim] =
+              __bfloat16_as_ushort(__float2bfloat16_rn(val));
+          if (dim == 0 && a.lse) a.lse[(int64_t)rg.bt * a.H + hq] = lsev;
+        }
+      }
+    }
+    consumer_sync(NC * 32);  // the merge buffer is free again
+  };
+
+  for (int i = 0; i < n; ++i) {
+    const int e = list[i];
+    const int64_t row = r0 + (e >> 16);
+    while (cur < row) {
+      flush();
+      ++cur;
+      rg = row_geo(a, cur);
+      ws.reset();
+      ws.load_q(a, rg, lane);
+    }
+    const int u0 = i * nsub;
+    const int st0 = (warp - (u0 % NC) + NC) % NC;
+    if (st0 >= nsub || failed) continue;
+    const int s = i % a.stages;
+    // After a wait runs out this warp stops computing but keeps walking the list,
+    // so that every consumer warp still reaches the same row-boundary barriers.
+    if (!mbar_wait_bounded(full0 + 8 * s, (i / a.stages) & 1, a.st, 3u, a.wait_ns)) {
+      failed = true;
+      continue;
+    }
+    const uint32_t kbase = sbase + (uint32_t)s * a.stage_bytes;
+    const uint32_t vbase = kbase + (D / 64) * half_bytes;
+    const int beta = e & 0xffff;
+    bool wrote = false;
+    for (int st = st0; st < nsub; st += NC) {
+      const int j0 = beta * a.block + st * 16;
+      if (j0 < rg.lim) ws.attend(a, smem, sbase, kbase, vbase, half_bytes, st * 16, j0, rg.lim, lane, wrote);
+    }
+    if (wrote) fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty0 + 8 * s);
+  }
+  while (true) {
+    flush();
+    if (cur >= r1) break;
+    ++cur;
+    rg = row_geo(a, cur);
+    ws.reset();
   }
 }
 
@@ -393,39 +587,62 @@ bool make_kv_map(CUtensorMap* map, const uint16_t* base, const Shape& s, const i
          CUDA_SUCCESS;
 }
 
+constexpr int kStreamNC = 4;       // consumer warps of the streaming kernel
+constexpr int kMaxList = 4096;     // entries a streaming CTA compacts up front
+constexpr uint32_t kSmemCap = 227u * 1024u;
+
 struct AttnPlan {
-  int splits, chunk, stages;
-  uint32_t stage_bytes, region_bytes;
+  bool stream;
+  int stages, ctas, per, smax, list_cap;
+  int64_t total;
+  uint32_t stage_bytes, region_bytes, merge_off;
   size_t smem_bytes;
 };
+
+// Stage count that keeps every block of a stage on the same warps (a warp waits
+// only on the stages of blocks it processes): with fewer 16-token slices per
+// block than consumer warps, a multiple of the warp cycle.
+int stage_count(int want, int nsub, int nc) {
+  const int cycle = nsub >= nc ? 1 : nc / nsub;
+  want = max(2, min(8, want));
+  return max(cycle, want - want % cycle);
+}
 
 AttnPlan plan_attn(const Shape& s) {
   AttnPlan pl;
   pl.stage_bytes = 4u * s.d * s.block;  // K and V tiles of one block, bf16
-  // Two CTAs per SM when the stages allow it, otherwise one with deeper buffering.
-  int stages = (int)((100u * 1024u) / pl.stage_bytes);
-  if (stages < 2) stages = min(4, (int)((200u * 1024u) / pl.stage_bytes));
-  stages = max(2, min(8, stages));
-  // A warp waits only on the stages of the blocks it processes, so every block
-  // that lands in a given stage must be processed by the same warps: with fewer
-  // than four 16-token slices per block, the stage count is a multiple of the
-  // warp cycle (4 / slices).
   const int nsub = s.block / 16;
-  const int cycle = nsub >= kConsumerWarps ? 1 : kConsumerWarps / nsub;
-  stages = max(cycle, stages - stages % cycle);
-  pl.stages = stages;
-  const uint32_t merge_bytes = kConsumerWarps * 16 * (s.d + 2) * 4;
-  pl.region_bytes = max(pl.stages * pl.stage_bytes, merge_bytes);
   const int64_t rows_g = (int64_t)s.batch * s.n_q * s.h;
-  const int ctas_per_sm = (pl.region_bytes <= 100u * 1024u) ? 2 : 1;
-  const int64_t want = (int64_t)num_sms() * ctas_per_sm * 2;
-  const int64_t by_fill = (want + rows_g - 1) / rows_g;
-  int splits = (int)(by_fill < (s.topk + 3) / 4 ? by_fill : (s.topk + 3) / 4);
-  splits = max(splits, (s.topk + 511) / 512);
-  pl.splits = max(1, splits);
-  pl.chunk = (s.topk + pl.splits - 1) / pl.splits;
-  pl.splits = (s.topk + pl.chunk - 1) / pl.chunk;
-  pl.smem_bytes = 1024 + pl.region_bytes + 16 * pl.stages + 4 * (pl.chunk + 1);
+  pl.total = rows_g * s.topk;
+  const uint32_t merge_bytes = (uint32_t)kStreamNC * 16 * (s.d + 2) * 4 + 16;
+  // Few rows with many blocks (decode): the persistent streaming kernel.
+  pl.stream = rows_g < 4LL * num_sms();
+  if (pl.stream) {
+    pl.stages = stage_count((int)((160u * 1024u) / pl.stage_bytes), nsub, kStreamNC);
+    pl.region_bytes = pl.stages * pl.stage_bytes + ((merge_bytes + 1023) & ~1023u);
+    pl.merge_off = pl.stages * pl.stage_bytes;
+    pl.ctas = num_sms();
+    pl.per = (int)((pl.total + pl.ctas - 1) / pl.ctas);
+    if (pl.per > kMaxList) {
+      pl.per = kMaxList;
+      pl.ctas = (int)((pl.total + kMaxList - 1) / kMaxList);
+    }
+    pl.ctas = (int)((pl.total + pl.per - 1) / pl.per);
+    pl.smax = (s.topk - 1) / pl.per + 2;
+    pl.list_cap = pl.per;
+  } else {
+    // Two CTAs per SM when the stages allow it, else one with deeper buffering.
+    int want = (int)((100u * 1024u) / pl.stage_bytes);
+    if (want < 2) want = min(4, (int)((200u * 1024u) / pl.stage_bytes));
+    pl.stages = stage_count(want, nsub, 4);
+    pl.region_bytes = max(pl.stages * pl.stage_bytes, merge_bytes);
+    pl.merge_off = 0;
+    pl.ctas = (int)rows_g;
+    pl.per = s.topk;
+    pl.smax = 1;
+    pl.list_cap = s.topk;
+  }
+  pl.smem_bytes = 1024 + pl.region_bytes + 16 * pl.stages + 4 * (pl.list_cap + 1);
   return pl;
 }
 
@@ -433,18 +650,20 @@ AttnPlan plan_attn(const Shape& s) {
 
 size_t attn_partial_bytes(const Shape& s) {
   const AttnPlan pl = plan_attn(s);
-  if (pl.splits <= 1) return 0;
-  const size_t n = (size_t)s.batch * s.n_q * s.H * pl.splits;
-  return n * (size_t)(s.d + 1) * sizeof(float) + 256;
+  if (!pl.stream) return 0;
+  const size_t n = (size_t)s.batch * s.n_q * s.H * pl.smax;
+  const size_t rows_g = (size_t)s.batch * s.n_q * s.h;
+  return n * (size_t)(s.d + 1) * sizeof(float) + rows_g * sizeof(int) + 512;
 }
 
-int attn_launches(const Shape& s) { return plan_attn(s).splits > 1 ? 2 : 1; }
+int attn_launches(const Shape&) { return 1; }
 
 cudaError_t launch_sparse_attn(const Shape& s, const uint16_t* q, const uint16_t* k,
                                const uint16_t* v, const int32_t* ids, uint16_t* out, float* lse,
                                void* partials, size_t partial_bytes, DeviceStatus* st,
                                cudaStream_t stream) {
   const AttnPlan pl = plan_attn(s);
+  if (pl.smem_bytes > kSmemCap) return cudaErrorInvalidValue;
   CUtensorMap tmk, tmv;
   if (!make_kv_map(&tmk, k, s, s.k_s) || !make_kv_map(&tmv, v, s, s.v_s))
     return cudaErrorInvalidValue;
@@ -464,12 +683,18 @@ cudaError_t launch_sparse_attn(const Shape& s, const uint16_t* q, const uint16_t
   a.block = s.block;
   a.nblk = s.nblk;
   a.causal = s.causal;
-  a.scale_log2 = s.scale * 1.4426950408889634f;
-  a.splits = pl.splits;
-  a.chunk = pl.chunk;
+  a.scale_log2 = s.scale * kLog2e;
   a.stages = pl.stages;
   a.stage_bytes = pl.stage_bytes;
   a.region_bytes = pl.region_bytes;
+  a.merge_off = pl.merge_off;
+  a.list_cap = pl.list_cap;
+  a.total_slots = pl.total;
+  a.per = pl.per;
+  a.smax = pl.smax;
+  a.part_o = nullptr;
+  a.part_lse = nullptr;
+  a.counters = nullptr;
   a.out = out;
   a.o_s0 = s.o_s[0];
   a.o_s1 = s.o_s[1];
@@ -477,32 +702,43 @@ cudaError_t launch_sparse_attn(const Shape& s, const uint16_t* q, const uint16_t
   a.lse = lse;
   a.st = st;
   a.wait_ns = 500000000ull;  // 0.5 s; a healthy wait takes microseconds
-  a.part_o = nullptr;
-  a.part_lse = nullptr;
-  const size_t nrow_h = (size_t)s.batch * s.n_q * s.H;
-  if (pl.splits > 1) {
-    if (partials == nullptr || partial_bytes < attn_partial_bytes(s)) return cudaErrorInvalidValue;
-    a.part_o = reinterpret_cast<float*>(partials);
-    a.part_lse = a.part_o + nrow_h * pl.splits * s.d;
-  }
-  const dim3 grid((unsigned)((int64_t)s.batch * s.n_q * s.h), pl.splits);
   cudaError_t err;
-  if (s.d == 128) {
-    err = cudaFuncSetAttribute(sparse_attn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)pl.smem_bytes);
-    if (err != cudaSuccess) return err;
-    sparse_attn_kernel<128><<<grid, kAttnThreads, pl.smem_bytes, stream>>>(tmk, tmv, a);
-  } else {
-    err = cudaFuncSetAttribute(sparse_attn_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)pl.smem_bytes);
-    if (err != cudaSuccess) return err;
-    sparse_attn_kernel<64><<<grid, kAttnThreads, pl.smem_bytes, stream>>>(tmk, tmv, a);
+  if (!pl.stream) {
+    const dim3 grid((unsigned)pl.ctas);
+    if (s.d == 128) {
+      err = cudaFuncSetAttribute(sparse_attn_rows_kernel<128>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem_bytes);
+      if (err != cudaSuccess) return err;
+      sparse_attn_rows_kernel<128><<<grid, 5 * 32, pl.smem_bytes, stream>>>(tmk, tmv, a);
+    } else {
+      err = cudaFuncSetAttribute(sparse_attn_rows_kernel<64>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem_bytes);
+      if (err != cudaSuccess) return err;
+      sparse_attn_rows_kernel<64><<<grid, 5 * 32, pl.smem_bytes, stream>>>(tmk, tmv, a);
+    }
+    return cudaGetLastError();
   }
-  err = cudaGetLastError();
-  if (err != cudaSuccess || pl.splits == 1) return err;
-  combine_kernel<<<(unsigned)nrow_h, 128, 0, stream>>>(a.part_o, a.part_lse, pl.splits, s.d, s.H,
-                                                       s.n_q, out, s.o_s[0], s.o_s[1], s.o_s[2],
-                                                       lse);
+  const size_t nrow_h = (size_t)s.batch * s.n_q * s.H;
+  if (partials == nullptr || partial_bytes < attn_partial_bytes(s)) return cudaErrorInvalidValue;
+  a.part_o = reinterpret_cast<float*>(partials);
+  a.part_lse = a.part_o + nrow_h * pl.smax * s.d;
+  a.counters = reinterpret_cast<int*>(
+      (reinterpret_cast<uintptr_t>(a.part_lse + nrow_h * pl.smax) + 255) & ~uintptr_t(255));
+  err = cudaMemsetAsync(a.counters, 0, (size_t)s.batch * s.n_q * s.h * sizeof(int), stream);
+  if (err != cudaSuccess) return err;
+  const dim3 grid((unsigned)pl.ctas);
+  constexpr int NT = (kStreamNC + 1) * 32;
+  if (s.d == 128) {
+    err = cudaFuncSetAttribute(sparse_attn_stream_kernel<128, kStreamNC>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem_bytes);
+    if (err != cudaSuccess) return err;
+    sparse_attn_stream_kernel<128, kStreamNC><<<grid, NT, pl.smem_bytes, stream>>>(tmk, tmv, a);
+  } else {
+    err = cudaFuncSetAttribute(sparse_attn_stream_kernel<64, kStreamNC>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem_bytes);
+    if (err != cudaSuccess) return err;
+    sparse_attn_stream_kernel<64, kStreamNC><<<grid, NT, pl.smem_bytes, stream>>>(tmk, tmv, a);
+  }
   return cudaGetLastError();
 }
 

@@ -99,24 +99,22 @@ __global__ void __launch_bounds__(256) topk_warp_kernel(TopkArgs a) {
   for (int i = m + lane; i < a.topk; i += 32) out[i] = -1;
 }
 
-constexpr int kCtaThreads = 1024;
-constexpr int kCtaWarps = kCtaThreads / 32;
-
-// Sum over the CTA; `buf` alternates between calls so one barrier suffices.
-__device__ __forceinline__ unsigned cta_sum(unsigned v, unsigned (*red)[kCtaWarps], int& buf) {
+// Sum over the CTA (NW warps); `buf` alternates between calls so one barrier
+// per call suffices.  Each warp reads the NW partial sums with one load per lane.
+template <int NW>
+__device__ __forceinline__ unsigned cta_sum(unsigned v, unsigned (*red)[32], int& buf) {
+  const int lane = threadIdx.x & 31;
   v = __reduce_add_sync(0xffffffffu, v);
-  if ((threadIdx.x & 31) == 0) red[buf][threadIdx.x >> 5] = v;
+  if (lane == 0) red[buf][threadIdx.x >> 5] = v;
   __syncthreads();
-  unsigned tot = 0;
-#pragma unroll 8
-  for (int w = 0; w < kCtaWarps; ++w) tot += red[buf][w];
+  const unsigned tot = __reduce_add_sync(0xffffffffu, lane < NW ? red[buf][lane] : 0u);
   buf ^= 1;
   return tot;
 }
 
-// Exclusive prefix over the CTA in thread order; returns the prefix, sets `total`.
-__device__ __forceinline__ unsigned cta_exclusive_scan(unsigned v, unsigned* wsum,
-                                                       unsigned& total) {
+// Exclusive prefix over the CTA in thread order.
+template <int NW>
+__device__ __forceinline__ unsigned cta_exclusive_scan(unsigned v, unsigned* wsum) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   unsigned inc = v;
 #pragma unroll
@@ -126,22 +124,18 @@ __device__ __forceinline__ unsigned cta_exclusive_scan(unsigned v, unsigned* wsu
   }
   if (lane == 31) wsum[warp] = inc;
   __syncthreads();
-  unsigned before = 0;
-  total = 0;
-  for (int w = 0; w < kCtaWarps; ++w) {
-    const unsigned x = wsum[w];
-    if (w < warp) before += x;
-    total += x;
-  }
+  const unsigned x = lane < NW ? wsum[lane] : 0u;
+  const unsigned before = __reduce_add_sync(0xffffffffu, lane < warp ? x : 0u);
   __syncthreads();
   return before + inc - v;
 }
 
-// One CTA per row; thread i holds elements [i*E, i*E + E).
-template <int E>
-__global__ void __launch_bounds__(kCtaThreads) topk_cta_kernel(TopkArgs a) {
-  __shared__ unsigned red[2][kCtaWarps];
-  __shared__ unsigned wsum[kCtaWarps];
+// One CTA of NT threads per row; thread i holds elements [i*E, i*E + E).
+template <int NT, int E>
+__global__ void __launch_bounds__(NT) topk_cta_kernel(TopkArgs a) {
+  constexpr int NW = NT / 32;
+  __shared__ unsigned red[2][32];
+  __shared__ unsigned wsum[32];
   const int row = blockIdx.x;
   const RowInfo ri = row_info(a, row);
   const float* s = a.scores + (int64_t)row * a.nblk;
@@ -163,7 +157,7 @@ __global__ void __launch_bounds__(kCtaThreads) topk_cta_kernel(TopkArgs a) {
       unsigned cnt = 0;
 #pragma unroll
       for (int e = 0; e < E; ++e) cnt += key[e] >= cand;
-      if ((int)cta_sum(cnt, red, buf) >= m) T = cand;
+      if ((int)cta_sum<NW>(cnt, red, buf) >= m) T = cand;
     }
     unsigned gt = 0, eq = 0;
 #pragma unroll
@@ -171,9 +165,8 @@ __global__ void __launch_bounds__(kCtaThreads) topk_cta_kernel(TopkArgs a) {
       gt += key[e] > T;
       eq += key[e] == T;
     }
-    const int need = m - (int)cta_sum(gt, red, buf);
-    unsigned tot;
-    unsigned eqr = cta_exclusive_scan(eq, wsum, tot);
+    const int need = m - (int)cta_sum<NW>(gt, red, buf);
+    unsigned eqr = cta_exclusive_scan<NW>(eq, wsum);
     unsigned nsel = 0;
     bool sel[E];
 #pragma unroll
@@ -183,12 +176,12 @@ __global__ void __launch_bounds__(kCtaThreads) topk_cta_kernel(TopkArgs a) {
       eqr += is_eq;
       nsel += sel[e];
     }
-    unsigned pos = cta_exclusive_scan(nsel, wsum, tot);
+    unsigned pos = cta_exclusive_scan<NW>(nsel, wsum);
 #pragma unroll
     for (int e = 0; e < E; ++e)
       if (sel[e]) out[pos++] = i0 + e;
   }
-  for (int i = m + threadIdx.x; i < a.topk; i += kCtaThreads) out[i] = -1;
+  for (int i = m + threadIdx.x; i < a.topk; i += NT) out[i] = -1;
 }
 
 }  // namespace
@@ -226,17 +219,17 @@ cudaError_t launch_topk(const Shape& s, const float* scores, int32_t* ids, Devic
 #undef MSA_TOPK_WARP
   }
   const dim3 grid(a.rows);
-#define MSA_TOPK_CTA(E_)                                                 \
-  if (n <= kCtaThreads * E_) {                                           \
-    topk_cta_kernel<E_><<<grid, kCtaThreads, 0, stream>>>(a);            \
-    return cudaGetLastError();                                           \
+#define MSA_TOPK_CTA(NT_, E_)                                      \
+  if (n <= NT_ * E_) {                                             \
+    topk_cta_kernel<NT_, E_><<<grid, NT_, 0, stream>>>(a);         \
+    return cudaGetLastError();                                     \
   }
-  MSA_TOPK_CTA(2)
-  MSA_TOPK_CTA(4)
-  MSA_TOPK_CTA(8)
-  MSA_TOPK_CTA(16)
-  MSA_TOPK_CTA(32)
-  MSA_TOPK_CTA(64)
+  MSA_TOPK_CTA(256, 8)
+  MSA_TOPK_CTA(256, 16)
+  MSA_TOPK_CTA(512, 16)
+  MSA_TOPK_CTA(1024, 16)
+  MSA_TOPK_CTA(1024, 32)
+  MSA_TOPK_CTA(1024, 64)
 #undef MSA_TOPK_CTA
   return cudaErrorInvalidValue;
 }

@@ -162,7 +162,7 @@ MSA_API msa_status_t msa_selftest_wait_timeout(void* workspace, size_t workspace
  * no counterpart in the pages; it is a deployment convenience.
  *   - Same arguments and results as msa_sparse_attn, minus the workspace.  The
  *     caller still passes inputs and outputs.
- *   - The partials live in one fixed 16 MiB array in the library's own device
+ *   - The partials live in one fixed 8 MiB array in the library's own device
  *     memory (every GPU that loads libmsa.so holds it until the process exits).
  *     Shapes whose partials do not fit (batch * n_q * H * splits * (d + 1) * 4
  *     bytes) return MSA_ERR_WORKSPACE; problems that run in one split (prefill)
