@@ -1,0 +1,317 @@
+// Index branch for prefill on the fifth-generation tensor cores (tcgen05).
+//
+// "MiniMax goes sparse" (atlascloud.ai), section 1, step 1 and "MiniMax M3 的 MSA
+// ..." (ai.air7.fun), first layer: token scores Q_idx . K_idx^T (one index query
+// per GQA group, one index key shared by all heads), compressed by Block Max Pool.
+// In prefill this is a dense causal GEMM per group (the pages note that the index
+// branch still scans the whole length there), so it runs on tcgen05 MMAs with the
+// accumulators in tensor memory; the causal mask and the block max are applied in
+// the tensor-memory -> register epilogue, and only fp32 block scores reach HBM.
+//
+// One CTA per (sequence, pair of groups, tile of 128 queries).  Both groups share
+// every 128-token key tile, which TMA streams through a ring of shared-memory
+// stages; the two query tiles stay resident.  Warp roles:
+//   warp 0     TMA producer (query tiles once, then the key ring);
+//   warp 1     tensor-memory allocation, and one thread issuing the MMAs
+//              (M = 128 queries, N = 128 keys, K = 16 per instruction);
+//   warps 2-5  epilogue: each owns 32 tensor-memory lanes (= 32 query rows),
+//              masks invisible keys, takes the block maxima, stores them.
+// Accumulators are double-buffered (2 x 2 groups x 128 columns = 512 columns), so
+// the epilogue of one key tile overlaps the MMAs of the next.  Every mbarrier wait
+// is bounded and records an error instead of hanging.
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace msa {
+namespace {
+
+constexpr int kQT = 128;  // queries per tile (MMA M, tensor-memory lanes)
+constexpr int kKT = 128;  // keys per tile (MMA N)
+constexpr int kNG = 2;    // groups per CTA
+constexpr int kTcThreads = 6 * 32;
+constexpr uint32_t kTmemCols = 512;
+
+struct TcArgs {
+  int batch, n_q, max_kv, h, block, nblk, causal;
+  const int32_t* seq_lens;
+  int n_mtiles, n_gpairs, stages;
+  float* scores;
+  int fill_tail;
+  DeviceStatus* st;
+  uint64_t wait_ns;
+};
+
+template <int DI, int BLK>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    index_score_tc_kernel(const __grid_constant__ CUtensorMap tmq,
+                          const __grid_constant__ CUtensorMap tmk, TcArgs a) {
+  constexpr int NATOM = DI / 64;               // 128-byte K atoms per row
+  constexpr uint32_t ATOM = 128u * 128u;       // one atom of a 128-row tile
+  constexpr uint32_t Q_BYTES = NATOM * ATOM;   // one group's query tile
+  constexpr uint32_t K_BYTES = NATOM * ATOM;   // one key tile
+  if (status_failed(a.st)) return;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t q_base = smem_u32(smem);
+  const uint32_t k_base = q_base + kNG * Q_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kNG * Q_BYTES + a.stages * K_BYTES);
+  const uint32_t b_qfull = smem_u32(bars);
+  const uint32_t b_kfull = b_qfull + 8;
+  const uint32_t b_kempty = b_kfull + 8 * a.stages;
+  const uint32_t b_afull = b_kempty + 8 * a.stages;
+  const uint32_t b_aempty = b_afull + 16;
+  const uint32_t b_done = b_aempty + 16;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 1 + 2 * a.stages + 5);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int x = blockIdx.x;
+  const int mt = a.n_mtiles - 1 - (x % a.n_mtiles);  // late (long) query tiles first
+  x /= a.n_mtiles;
+  const int gp = x % a.n_gpairs;
+  const int b = x / a.n_gpairs;
+  const int t0 = mt * kQT;
+  const int ng_valid = min(kNG, a.h - gp * kNG);
+  const int L = kv_length(a.seq_lens, b, a.max_kv, a.st);
+  const int t_last = min(t0 + kQT, a.n_q) - 1;
+  const int p_last = L - a.n_q + t_last;
+  const int lim_last = max(0, a.causal ? min(L, p_last + 1) : L);
+  const int n_kt = (lim_last + kKT - 1) / kKT;  // key tiles holding a visible key
+
+  if (threadIdx.x == 0) {
+    mbar_init(b_qfull, 1);
+    for (int s = 0; s < a.stages; ++s) {
+      mbar_init(b_kfull + 8 * s, 1);
+      mbar_init(b_kempty + 8 * s, 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(b_afull + 8 * i, 1);
+      mbar_init(b_aempty + 8 * i, 4);
+    }
+    mbar_init(b_done, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0 && n_kt > 0) {
+      prefetch_tensormap(&tmq);
+      prefetch_tensormap(&tmk);
+      mbar_arrive_expect_tx(b_qfull, ng_valid * Q_BYTES);
+      for (int ng = 0; ng < ng_valid; ++ng)
+#pragma unroll
+        for (int at = 0; at < NATOM; ++at)
+          tma_load_4d(q_base + ng * Q_BYTES + at * ATOM, &tmq, b_qfull, at * 64, gp * kNG + ng,
+                      t0, b);
+      int issued = 0;
+      for (int kt = 0; kt < n_kt; ++kt) {
+        const int s = kt % a.stages;
+        if (kt >= a.stages &&
+            !mbar_wait_bounded(b_kempty + 8 * s, ((kt / a.stages) - 1) & 1, a.st, 0x101u,
+                               a.wait_ns))
+          break;
+        mbar_arrive_expect_tx(b_kfull + 8 * s, K_BYTES);
+#pragma unroll
+        for (int at = 0; at < NATOM; ++at)
+          tma_load_3d(k_base + s * K_BYTES + at * ATOM, &tmk, b_kfull + 8 * s, at * 64, kt * kKT,
+                      b);
+        ++issued;
+      }
+      // Drain: the last stages are released by the MMA commits, i.e. after their
+      // copies landed and were read.
+      for (int kt = max(0, issued - a.stages); kt < issued; ++kt)
+        mbar_wait_bounded(b_kempty + 8 * (kt % a.stages), (kt / a.stages) & 1, a.st, 0x102u,
+                          a.wait_ns);
+    }
+  } else if (warp == 1) {
+    // ----------------------------------------------------------- MMA issue
+    if (lane == 0 && n_kt > 0) {
+      const uint32_t idesc = tc::idesc_bf16(kQT, kKT, false);
+      bool ok = mbar_wait_bounded(b_qfull, 0, a.st, 0x103u, a.wait_ns);
+      for (int kt = 0; kt < n_kt && ok; ++kt) {
+        const int s = kt % a.stages, buf = kt & 1;
+        ok = mbar_wait_bounded(b_kfull + 8 * s, (kt / a.stages) & 1, a.st, 0x104u, a.wait_ns);
+        if (ok && kt >= 2)
+          ok = mbar_wait_bounded(b_aempty + 8 * buf, ((kt >> 1) - 1) & 1, a.st, 0x105u,
+                                 a.wait_ns);
+        if (!ok) break;
+        tc::fence_after_sync();
+        for (int ng = 0; ng < ng_valid; ++ng) {
+          const uint32_t d_tmem = tmem + (uint32_t)(buf * kNG * kKT + ng * kKT);
+#pragma unroll
+          for (int ks = 0; ks < DI / 16; ++ks) {
+            const uint32_t koff = (ks >> 2) * ATOM + (ks & 3) * 32;
+            tc::mma_bf16(d_tmem, tc::desc_k_sw128(q_base + ng * Q_BYTES + koff),
+                         tc::desc_k_sw128(k_base + s * K_BYTES + koff), idesc, ks > 0 ? 1u : 0u);
+          }
+        }
+        tc::commit(b_kempty + 8 * s);
+        tc::commit(b_afull + 8 * buf);
+      }
+      // Every MMA this thread issued has completed before tensor memory is freed.
+      tc::commit(b_done);
+      mbar_wait_bounded(b_done, 0, a.st, 0x107u, a.wait_ns);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int quarter = warp & 3;  // tensor-memory lanes [32q, 32q + 32)
+    const int row = quarter * 32 + lane;
+    const int t = t0 + row;
+    const bool row_ok = t < a.n_q;
+    const int p = L - a.n_q + t;
+    const int lim = row_ok ? max(0, a.causal ? min(L, p + 1) : L) : 0;
+    constexpr int bpt = kKT / BLK;  // blocks per key tile
+    const float ninf = -__int_as_float(0x7f800000);
+    const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+    float* srow = a.scores + ((int64_t)b * a.n_q + t) * a.h * (int64_t)a.nblk;
+    for (int kt = 0; kt < n_kt; ++kt) {
+      const int buf = kt & 1;
+      if (!mbar_wait_bounded(b_afull + 8 * buf, (kt >> 1) & 1, a.st, 0x106u, a.wait_ns)) break;
+      tc::fence_after_sync();
+      const int j0 = kt * kKT;
+      const int vis = lim - j0;  // columns [0, vis) of this tile are visible keys
+      for (int ng = 0; ng < ng_valid; ++ng) {
+        float bm[bpt];
+#pragma unroll
+        for (int k = 0; k < bpt; ++k) bm[k] = ninf;
+#pragma unroll
+        for (int c = 0; c < kKT / 32; ++c) {
+          float v[32];
+          tc::tmem_ld32(lane_base + (uint32_t)(buf * kNG * kKT + ng * kKT + c * 32), v);
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int col = c * 32 + i;
+            bm[col / BLK] = fmaxf(bm[col / BLK], col < vis ? v[i] : ninf);
+          }
+        }
+        if (row_ok) {
+          float* dst = srow + (int64_t)(gp * kNG + ng) * a.nblk + j0 / BLK;
+#pragma unroll
+          for (int k = 0; k < bpt; ++k)
+            if (j0 / BLK + k < a.nblk) dst[k] = bm[k];
+        }
+      }
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(b_aempty + 8 * buf);
+    }
+    if (a.fill_tail && row_ok) {
+      for (int ng = 0; ng < ng_valid; ++ng) {
+        float* dst = srow + (int64_t)(gp * kNG + ng) * a.nblk;
+        for (int beta = n_kt * bpt; beta < a.nblk; ++beta) dst[beta] = ninf;
+      }
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+template <int DI, int BLK>
+cudaError_t run_tc(const Shape& s, const uint16_t* q_idx, const uint16_t* k_idx, TcArgs& a,
+                   cudaStream_t stream) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return cudaErrorInvalidValue;
+  CUtensorMap tmq, tmk;
+  {
+    cuuint64_t dims[4] = {(cuuint64_t)s.d_idx, (cuuint64_t)s.h, (cuuint64_t)s.n_q,
+                          (cuuint64_t)s.batch};
+    cuuint64_t str[3] = {(cuuint64_t)s.qi_s[2] * 2, (cuuint64_t)s.qi_s[1] * 2,
+                         (cuuint64_t)s.qi_s[0] * 2};
+    cuuint32_t box[4] = {64, 1, (cuuint32_t)kQT, 1};
+    cuuint32_t es[4] = {1, 1, 1, 1};
+    if (enc(&tmq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<uint16_t*>(q_idx), dims, str,
+            box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  {
+    cuuint64_t dims[3] = {(cuuint64_t)s.d_idx, (cuuint64_t)s.max_kv, (cuuint64_t)s.batch};
+    cuuint64_t str[2] = {(cuuint64_t)s.ki_s[1] * 2, (cuuint64_t)s.ki_s[0] * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)kKT, 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    if (enc(&tmk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<uint16_t*>(k_idx), dims, str,
+            box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  constexpr uint32_t tile = (DI / 64) * 128u * 128u;
+  a.stages = DI == 128 ? 4 : 8;
+  const size_t smem = 1024 + kNG * tile + (size_t)a.stages * tile + 8 * (1 + 2 * a.stages + 5) + 16;
+  cudaError_t err = cudaFuncSetAttribute(index_score_tc_kernel<DI, BLK>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  const unsigned grid = (unsigned)((int64_t)s.batch * a.n_gpairs * a.n_mtiles);
+  index_score_tc_kernel<DI, BLK><<<grid, kTcThreads, smem, stream>>>(tmq, tmk, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool index_scores_tc_supported(const Shape& s) {
+  return s.n_q > 1 && (s.d_idx == 64 || s.d_idx == 128);
+}
+
+cudaError_t launch_index_scores_tc(const Shape& s, const uint16_t* q_idx, const uint16_t* k_idx,
+                                   float* scores, bool fill_tail, DeviceStatus* st,
+                                   cudaStream_t stream) {
+  TcArgs a;
+  a.batch = s.batch;
+  a.n_q = s.n_q;
+  a.max_kv = s.max_kv;
+  a.h = s.h;
+  a.block = s.block;
+  a.nblk = s.nblk;
+  a.causal = s.causal;
+  a.seq_lens = s.seq_lens;
+  a.n_mtiles = (s.n_q + kQT - 1) / kQT;
+  a.n_gpairs = (s.h + kNG - 1) / kNG;
+  a.scores = scores;
+  a.fill_tail = fill_tail ? 1 : 0;
+  a.st = st;
+  a.wait_ns = 500000000ull;
+#define MSA_TC_CASE(DI_, BLK_) \
+  if (s.d_idx == DI_ && s.block == BLK_) return run_tc<DI_, BLK_>(s, q_idx, k_idx, a, stream);
+  MSA_TC_CASE(128, 16)
+  MSA_TC_CASE(128, 32)
+  MSA_TC_CASE(128, 64)
+  MSA_TC_CASE(128, 128)
+  MSA_TC_CASE(64, 16)
+  MSA_TC_CASE(64, 32)
+  MSA_TC_CASE(64, 64)
+  MSA_TC_CASE(64, 128)
+#undef MSA_TC_CASE
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace msa

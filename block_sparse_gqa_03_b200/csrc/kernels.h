@@ -24,6 +24,12 @@ cudaError_t launch_index_scores(const Shape& s, const uint16_t* q_idx, const uin
                                 float* scores, bool fill_tail, DeviceStatus* st,
                                 cudaStream_t stream);
 
+// Stage 1a/1b for prefill on tcgen05 (d_idx 64 or 128, n_q > 1).
+bool index_scores_tc_supported(const Shape& s);
+cudaError_t launch_index_scores_tc(const Shape& s, const uint16_t* q_idx, const uint16_t* k_idx,
+                                   float* scores, bool fill_tail, DeviceStatus* st,
+                                   cudaStream_t stream);
+
 // Stage 1c: top-k block ids, int32 [batch, n_q, h, topk], from the scores.
 cudaError_t launch_topk(const Shape& s, const float* scores, int32_t* ids, DeviceStatus* st,
                         cudaStream_t stream);

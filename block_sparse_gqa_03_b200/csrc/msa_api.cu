@@ -178,8 +178,11 @@ msa_status_t run_select(const Shape& s, const msa_bf16_t* q_idx, const msa_bf16_
                         cudaStream_t stream) {
   msa::DeviceStatus* st = reinterpret_cast<msa::DeviceStatus*>(ws);
   float* scores = user_scores ? user_scores : reinterpret_cast<float*>(at(ws, l.scores_off));
-  cudaError_t e = msa::launch_index_scores(s, q_idx, k_idx, scores, user_scores != nullptr, st,
-                                           stream);
+  cudaError_t e = msa::index_scores_tc_supported(s)
+                      ? msa::launch_index_scores_tc(s, q_idx, k_idx, scores,
+                                                    user_scores != nullptr, st, stream)
+                      : msa::launch_index_scores(s, q_idx, k_idx, scores, user_scores != nullptr,
+                                                 st, stream);
   if (e != cudaSuccess) return MSA_ERR_CUDA;
   return cuda_status(msa::launch_topk(s, scores, ids, st, stream));
 }
