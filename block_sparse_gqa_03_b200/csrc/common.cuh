@@ -114,6 +114,15 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
   }
 }
 
+// Bounded wait taken by a whole warp: the result is the same on every lane (all
+// lanes succeed or all report failure), so that warp-collective instructions that
+// follow (ldmatrix, mma.sync, tcgen05.ld) never run on a diverged warp.
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, DeviceStatus* st,
+                                               uint32_t detail, uint64_t limit_ns) {
+  const bool ok = mbar_wait_bounded(bar, parity, st, detail, limit_ns);
+  return __all_sync(0xffffffffu, ok);
+}
+
 // -------------------------------------------------------------- TMA loads
 // 4-D tiled tensor load into shared memory, completion counted in bytes on an
 // mbarrier.  No cluster multicast.

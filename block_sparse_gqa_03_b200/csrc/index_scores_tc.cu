@@ -174,7 +174,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     float* srow = a.scores + ((int64_t)b * a.n_q + t) * a.h * (int64_t)a.nblk;
     for (int kt = 0; kt < n_kt; ++kt) {
       const int buf = kt & 1;
-      if (!mbar_wait_bounded(b_afull + 8 * buf, (kt >> 1) & 1, a.st, 0x106u, a.wait_ns)) break;
+      if (!mbar_wait_warp(b_afull + 8 * buf, (kt >> 1) & 1, a.st, 0x106u, a.wait_ns)) break;
       tc::fence_after_sync();
       const int j0 = kt * kKT;
       const int vis = lim - j0;  // columns [0, vis) of this tile are visible keys

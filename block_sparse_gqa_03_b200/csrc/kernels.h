@@ -42,6 +42,16 @@ cudaError_t launch_sparse_attn(const Shape& s, const uint16_t* q, const uint16_t
                                void* partials, size_t partial_bytes, DeviceStatus* st,
                                cudaStream_t stream);
 
+// Stage 2 for prefill, KV-major on tcgen05 (d 64/128, block 64/128, n_q > 1):
+// inverted index, tiles of gathered (query, head) rows per selected block,
+// partials merged by a combine kernel; processed in query chunks.
+bool kv_attn_supported(const Shape& s);
+size_t kv_workspace_bytes(const Shape& s);
+int kv_launches(const Shape& s);
+cudaError_t launch_kv_attn(const Shape& s, const CUtensorMap& tmk, const CUtensorMap& tmv,
+                           const uint16_t* q, const int32_t* ids, uint16_t* out, float* lse,
+                           void* ws, size_t ws_bytes, DeviceStatus* st, cudaStream_t stream);
+
 // Test hook: one bounded wait that runs out and records kErrTimeout.
 cudaError_t launch_wait_timeout_probe(DeviceStatus* st, uint64_t wait_ns, cudaStream_t stream);
 

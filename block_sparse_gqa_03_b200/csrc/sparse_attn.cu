@@ -368,7 +368,7 @@ __global__ void __launch_bounds__(5 * 32, 1)
     const int st0 = (warp - (u0 % NC) + NC) % NC;  // first slice of block i owned by this warp
     if (st0 >= nsub) continue;
     const int s = i % a.stages;
-    if (!mbar_wait_bounded(full0 + 8 * s, (i / a.stages) & 1, a.st, 3u, a.wait_ns)) break;
+    if (!mbar_wait_warp(full0 + 8 * s, (i / a.stages) & 1, a.st, 3u, a.wait_ns)) break;
     const uint32_t kbase = sbase + (uint32_t)s * a.stage_bytes;
     const uint32_t vbase = kbase + (D / 64) * half_bytes;
     const int beta = list[i] & 0xffff;
@@ -526,7 +526,7 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1)
     const int s = i % a.stages;
     // After a wait runs out this warp stops computing but keeps walking the list,
     // so that every consumer warp still reaches the same row-boundary barriers.
-    if (!mbar_wait_bounded(full0 + 8 * s, (i / a.stages) & 1, a.st, 3u, a.wait_ns)) {
+    if (!mbar_wait_warp(full0 + 8 * s, (i / a.stages) & 1, a.st, 3u, a.wait_ns)) {
       failed = true;
       continue;
     }
@@ -650,13 +650,16 @@ AttnPlan plan_attn(const Shape& s) {
 
 size_t attn_partial_bytes(const Shape& s) {
   const AttnPlan pl = plan_attn(s);
-  if (!pl.stream) return 0;
+  if (!pl.stream) return kv_attn_supported(s) ? kv_workspace_bytes(s) : 0;
   const size_t n = (size_t)s.batch * s.n_q * s.H * pl.smax;
   const size_t rows_g = (size_t)s.batch * s.n_q * s.h;
   return n * (size_t)(s.d + 1) * sizeof(float) + rows_g * sizeof(int) + 512;
 }
 
-int attn_launches(const Shape&) { return 1; }
+int attn_launches(const Shape& s) {
+  const AttnPlan pl = plan_attn(s);
+  return !pl.stream && kv_attn_supported(s) ? kv_launches(s) : 1;
+}
 
 cudaError_t launch_sparse_attn(const Shape& s, const uint16_t* q, const uint16_t* k,
                                const uint16_t* v, const int32_t* ids, uint16_t* out, float* lse,
@@ -703,6 +706,8 @@ cudaError_t launch_sparse_attn(const Shape& s, const uint16_t* q, const uint16_t
   a.st = st;
   a.wait_ns = 500000000ull;  // 0.5 s; a healthy wait takes microseconds
   cudaError_t err;
+  if (!pl.stream && kv_attn_supported(s))
+    return launch_kv_attn(s, tmk, tmv, q, ids, out, lse, partials, partial_bytes, st, stream);
   if (!pl.stream) {
     const dim3 grid((unsigned)pl.ctas);
     if (s.d == 128) {

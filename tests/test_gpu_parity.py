@@ -83,6 +83,10 @@ SMALL_CASES = [
             topk=8, causal=True, seed=107, len_range=(1, 5000)),
     Problem("decode_g1_h16", batch=3, n_q=1, max_kv=3000, H=16, h=16, d=64, d_idx=32, block=16,
             topk=1, causal=True, seed=108),
+    Problem("prefill_kv_varlen", batch=3, n_q=300, max_kv=700, H=12, h=2, d=128, d_idx=64,
+            block=128, topk=3, causal=True, seed=112, len_range=(300, 700)),
+    Problem("prefill_kv_d64_b64", batch=1, n_q=1500, max_kv=1500, H=16, h=1, d=64, d_idx=128,
+            block=64, topk=5, causal=True, force_own=True, seed=113),
     Problem("decode_many_splits", batch=2, n_q=1, max_kv=65536, H=64, h=8, d=128, d_idx=128,
             block=64, topk=600, causal=True, seed=109, len_range=(40000, 65536)),
 ]
