@@ -21,8 +21,11 @@
 // CTA roles (persistent CTAs, each a contiguous share of the chunk's tiles):
 //   warp 0      TMA producer of K and V (a new load only when the block changes);
 //   warp 1      tensor-memory allocation and the single MMA-issuing thread;
-//   warps 2-5   gather the tile's Q rows with 16-byte async copies (swizzled);
-//   warps 6-9   softmax and output epilogue, one thread per tile row.
+//   warps 2-5   gather the tile's Q rows with 16-byte async copies (swizzled): the
+//               tile's query rows are resolved once into a shared table, then
+//               the copies are issued in a tight loop;
+//   warps 6-13  softmax and output epilogue, one thread per tile row; two warp
+//               groups take alternate tiles so one computes while the other waits.
 // Double buffers: Q/P tiles (P overwrites Q once S is computed), K/V stages, and
 // S and O in tensor memory.  Every wait is bounded.
 #include "kernels.h"
@@ -32,7 +35,7 @@ namespace msa {
 namespace {
 
 constexpr int kRows = 128;                  // MMA M: (query, head) rows per tile
-constexpr int kKvThreads = 10 * 32;
+constexpr int kKvThreads = 14 * 32;
 constexpr int kWarpProd = 0, kWarpMma = 1, kWarpGather0 = 2, kWarpSoft0 = 6;
 
 struct KvArgs {
@@ -226,6 +229,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
   const uint32_t b_pfull = b_sfree + 16, b_ofull = b_pfull + 16;
   const uint32_t b_ofree = b_ofull + 16, b_done = b_ofree + 16;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 19);
+  uint64_t* qsrc = bars + 32;  // [2][kRows] source row of each query of a tile
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ntiles = __ldg(a.toffs + a.nj);
@@ -356,27 +360,33 @@ __global__ void __launch_bounds__(kKvThreads, 1)
       const int gt = threadIdx.x - kWarpGather0 * 32;  // 0..127
       int i = 0;
       bool ok = true;
+      constexpr int CPR = D / 8;  // 16-byte chunks per row
       for (int tile = tile0; tile < tile1; ++tile, ++i) {
         w.advance(a, tile);
         const int buf = i & 1;
         if (i >= 2 && ok)
           ok = mbar_wait_bounded(b_qempty + 8 * buf, ((i >> 1) - 1) & 1, a.st, 0x209u, a.wait_ns);
+        const TileInfo ti = tile_info(a, w.j, tile);
+        uint64_t* tab = qsrc + buf * kRows;
+        if (ok && gt < ti.nq) {
+          // the query of this list entry: chunk-relative slot position -> (b, t)
+          const int pos = __ldg(a.entries + ti.first + gt);
+          const int bt = (int)a.bt0 + pos / (a.h * a.topk);
+          const int t = bt % a.n_q;
+          tab[gt] = reinterpret_cast<uint64_t>(a.q + (int64_t)ti.b * a.q_s0 + (int64_t)t * a.q_s1 +
+                                               (int64_t)(ti.g * a.G) * a.q_s2);
+        }
+        asm volatile("bar.sync 2, 128;" ::: "memory");
         if (ok) {
-          const TileInfo ti = tile_info(a, w.j, tile);
           const int nrows = ti.nq * a.G;
-          constexpr int CPR = D / 8;  // 16-byte chunks per row
           const uint32_t dst0 = sqp + buf * QP_BYTES;
           for (int x = gt; x < nrows * CPR; x += 128) {
             const int row = x / CPR, ch = x % CPR;
-            const int qi = row / a.G, hi = row % a.G;
-            const int64_t pos = __ldg(a.entries + ti.first + qi);
-            const int64_t bt = a.bt0 + pos / ((int64_t)a.h * a.topk);
-            const int t = (int)(bt % a.n_q);
-            const uint16_t* src = a.q + (int64_t)ti.b * a.q_s0 + (int64_t)t * a.q_s1 +
-                                  (int64_t)(ti.g * a.G + hi) * a.q_s2 + ch * 8;
+            const int qi = row / a.G, hi = row - qi * a.G;
+            const uint16_t* src =
+                reinterpret_cast<const uint16_t*>(tab[qi]) + (int64_t)hi * a.q_s2 + ch * 8;
             const uint32_t dst = dst0 + (ch >> 3) * (kRows * 128u) + swz128(row, ch & 7);
-            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src)
-                         : "memory");
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src));
           }
         }
         asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
@@ -385,95 +395,70 @@ __global__ void __launch_bounds__(kKvThreads, 1)
       }
     } else {
       // ------------------------------------------- softmax and epilogue warps
+      const int wg = (warp - kWarpSoft0) >> 2;  // warp group: takes tiles with i % 2 == wg
       const int quarter = warp & 3;
       const int row = quarter * 32 + lane;
       const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
       const float ninf = -__int_as_float(0x7f800000);
       const float kLn2 = 0.69314718055994531f;
-      int i = 0;
+      uint8_t* const sm0 = smem;
+      const uint32_t sm0a = smem_u32(smem);
       bool ok = true;
-      // state of the previous tile, written out after the next softmax
-      int64_t prev_pos = -1;
-      float prev_inv_l = 0.f, prev_lse = ninf;
-      int prev_hi = 0;
-      auto epilogue = [&](int pi) {
-        const int pbuf = pi & 1;
-        if (ok) ok = mbar_wait_warp(b_ofull + 8 * pbuf, (pi >> 1) & 1, a.st, 0x20au, a.wait_ns);
-        tc::fence_after_sync();
-        // tcgen05.ld is warp-collective: every lane loads, only live rows store.
-        const bool store = ok && prev_pos >= 0;
-        uint16_t* dst = a.part_o + (store ? (prev_pos * a.G + prev_hi) * (int64_t)D : 0);
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          float v[32];
-          tc::tmem_ld32(lane_base + TM_O + pbuf * D + c * 32, v);
-          tc::tmem_wait_ld();
-          uint32_t pk[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e)
-            pk[e] = pack_bf16(v[2 * e] * prev_inv_l, v[2 * e + 1] * prev_inv_l);
-          if (store) {
-            uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-              d4[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
-          }
-        }
-        if (store) a.part_lse[prev_pos * a.G + prev_hi] = prev_lse;
-        tc::fence_before_sync();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(b_ofree + 8 * pbuf);
-      };
-      int kv_use = -1, kv_prev_j = -1;
+      int i = 0, kv_use = -1, kv_prev_j = -1;
       for (int tile = tile0; tile < tile1; ++tile, ++i) {
         w.advance(a, tile);
         if (w.j != kv_prev_j) {
           kv_prev_j = w.j;
           ++kv_use;
         }
-        const int buf = i & 1;
+        if ((i & 1) != wg) continue;
+        const int buf = wg;
         const TileInfo ti = tile_info(a, w.j, tile);
         const bool live = row < ti.nq * a.G;
-        int64_t pos = -1;
-        int hi = 0, lim = 0;
+        int pos = -1, hi = 0, lim = 0;
         if (live) {
-          pos = __ldg(a.entries + ti.first + row / a.G);
-          hi = row % a.G;
-          const int64_t bt = a.bt0 + pos / ((int64_t)a.h * a.topk);
-          lim = visible_limit(a, ti.b, (int)(bt % a.n_q));
+          const int qi = row / a.G;
+          hi = row - qi * a.G;
+          pos = __ldg(a.entries + ti.first + qi);
+          const int bt = (int)a.bt0 + pos / (a.h * a.topk);
+          lim = visible_limit(a, ti.b, bt % a.n_q);
         }
         if (ok) ok = mbar_wait_warp(b_sfull + 8 * buf, (i >> 1) & 1, a.st, 0x20bu, a.wait_ns);
         tc::fence_after_sync();
-        // Two passes over the scores in tensor memory keep the register use low:
-        // the row maximum first, then probabilities, their sum and the bf16 P row.
+        // Scores from tensor memory, two 32-column loads per wait: the row maximum
+        // first, then probabilities, their sum and the bf16 P row (K-major, swizzled).
         const int vis = lim - ti.beta * BLK;  // keys [0, vis) of the block are visible
         const uint32_t srow = lane_base + TM_S + buf * BLK;
         float mx = ninf;
 #pragma unroll
-        for (int c = 0; c < BLK / 32; ++c) {
-          float v[32];
-          tc::tmem_ld32(srow + c * 32, v);
+        for (int c = 0; c < BLK / 32; c += 2) {
+          float v0[32], v1[32];
+          tc::tmem_ld32(srow + c * 32, v0);
+          tc::tmem_ld32(srow + c * 32 + 32, v1);
           tc::tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) mx = fmaxf(mx, c * 32 + e < vis ? v[e] : ninf);
+          for (int e = 0; e < 32; ++e) {
+            mx = fmaxf(mx, c * 32 + e < vis ? v0[e] : ninf);
+            mx = fmaxf(mx, c * 32 + 32 + e < vis ? v1[e] : ninf);
+          }
         }
         mx *= a.scale_log2;
         const float msafe = live && mx != ninf ? mx : 0.f;
         float l = 0.f;
-        const uint32_t pdst = sqp + buf * QP_BYTES;
-        uint8_t* pbase = smem + (pdst - smem_u32(smem));
+        uint8_t* pbase = sm0 + (sqp + buf * QP_BYTES - sm0a);
 #pragma unroll
-        for (int c = 0; c < BLK / 32; ++c) {
-          float v[32];
-          tc::tmem_ld32(srow + c * 32, v);
+        for (int c = 0; c < BLK / 32; c += 2) {
+          float v[64];
+          tc::tmem_ld32(srow + c * 32, *reinterpret_cast<float(*)[32]>(v));
+          tc::tmem_ld32(srow + c * 32 + 32, *reinterpret_cast<float(*)[32]>(v + 32));
           tc::tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
+          for (int e = 0; e < 64; ++e) {
             v[e] = c * 32 + e < vis ? exp2f(v[e] * a.scale_log2 - msafe) : 0.f;
             l += v[e];
           }
 #pragma unroll
-          for (int q8 = 0; q8 < 4; ++q8) {
+          for (int q8 = 0; q8 < 8; ++q8) {
             const int ch = c * 4 + q8;  // 16-byte chunk of the P row
             const uint4 v4 = make_uint4(pack_bf16(v[8 * q8], v[8 * q8 + 1]),
                                         pack_bf16(v[8 * q8 + 2], v[8 * q8 + 3]),
@@ -493,7 +478,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
           const int r0 = max(0, L - ti.beta * BLK);
           if (r0 < BLK) {
             const int per_h = (BLK - r0) * 8;
-            uint8_t* vb = smem + (skv - smem_u32(smem)) + (kv_use & 1) * KV_BYTES + NH * HALF;
+            uint8_t* vb = sm0 + (skv - sm0a) + (kv_use & 1) * KV_BYTES + NH * HALF;
             for (int x = row; x < per_h * NH; x += 128) {
               const int hh = x / per_h, rem = x % per_h;
               *reinterpret_cast<uint4*>(vb + hh * HALF + (r0 + rem / 8) * 128 + (rem % 8) * 16) =
@@ -505,13 +490,36 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         tc::fence_before_sync();
         __syncwarp();
         if (lane == 0) mbar_arrive(b_pfull + 8 * buf);
-        if (i >= 1) epilogue(i - 1);
-        prev_pos = live ? pos : -1;
-        prev_hi = hi;
-        prev_inv_l = l > 0.f ? 1.f / l : 0.f;
-        prev_lse = (live && mx != ninf && l > 0.f) ? (msafe + log2f(l)) * kLn2 : ninf;
+        // Output of this tile: O / l in bf16 and the log-sum-exp, for live rows.
+        const float inv_l = l > 0.f ? 1.f / l : 0.f;
+        if (ok) ok = mbar_wait_warp(b_ofull + 8 * buf, (i >> 1) & 1, a.st, 0x20au, a.wait_ns);
+        tc::fence_after_sync();
+        const bool store = ok && live;
+        uint16_t* dst = a.part_o + (store ? ((int64_t)pos * a.G + hi) * D : 0);
+#pragma unroll
+        for (int c = 0; c < D / 32; c += 2) {
+          float v[64];
+          tc::tmem_ld32(lane_base + TM_O + buf * D + c * 32, *reinterpret_cast<float(*)[32]>(v));
+          tc::tmem_ld32(lane_base + TM_O + buf * D + c * 32 + 32,
+                        *reinterpret_cast<float(*)[32]>(v + 32));
+          tc::tmem_wait_ld();
+          if (store) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              d4[e] = make_uint4(pack_bf16(v[8 * e] * inv_l, v[8 * e + 1] * inv_l),
+                                 pack_bf16(v[8 * e + 2] * inv_l, v[8 * e + 3] * inv_l),
+                                 pack_bf16(v[8 * e + 4] * inv_l, v[8 * e + 5] * inv_l),
+                                 pack_bf16(v[8 * e + 6] * inv_l, v[8 * e + 7] * inv_l));
+          }
+        }
+        if (store)
+          a.part_lse[(int64_t)pos * a.G + hi] =
+              (mx != ninf && l > 0.f) ? (msafe + log2f(l)) * kLn2 : ninf;
+        tc::fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(b_ofree + 8 * buf);
       }
-      if (i >= 1) epilogue(i - 1);
     }
   }
   tc::fence_before_sync();
@@ -524,7 +532,8 @@ __global__ void __launch_bounds__(kKvThreads, 1)
 
 // -------------------------------------------------------------- combine
 // One warp per (query, head): merge the head's partials over the group's valid
-// slots by log-sum-exp weights; bf16 output and the natural-log LSE.
+// slots by log-sum-exp weights; bf16 output and the natural-log LSE.  Lanes
+// take 32 slots at a time, so the loads of many partials are in flight at once.
 template <int D>
 __global__ void __launch_bounds__(256) kv_combine_kernel(KvArgs a, int BLK) {
   const int lane = threadIdx.x & 31;
@@ -532,51 +541,72 @@ __global__ void __launch_bounds__(256) kv_combine_kernel(KvArgs a, int BLK) {
   const int64_t n = (int64_t)a.nbt * a.H;
   if (wid >= n) return;
   const int hq = (int)(wid % a.H);
-  const int64_t bt_rel = wid / a.H;
-  const int g = hq / a.G, hi = hq % a.G;
-  const int64_t bt = a.bt0 + bt_rel;
-  const int b = (int)(bt / a.n_q), t = (int)(bt % a.n_q);
+  const int bt_rel = (int)(wid / a.H);
+  const int g = hq / a.G, hi = hq - g * a.G;
+  const int bt = (int)a.bt0 + bt_rel;
+  const int b = bt / a.n_q, t = bt % a.n_q;
   const int lim = visible_limit(a, b, t);
-  const int32_t* row_ids = a.ids + (bt * a.h + g) * a.topk;
-  const int64_t p0 = (bt_rel * a.h + g) * a.topk;
+  const int32_t* row_ids = a.ids + ((int64_t)bt * a.h + g) * a.topk;
+  const int64_t p0 = ((int64_t)bt_rel * a.h + g) * a.topk;
   const float ninf = -__int_as_float(0x7f800000);
   constexpr int PER = D / 32;  // dims per lane
   float M = ninf;
-  for (int s = 0; s < a.topk; ++s) {
-    const int beta = __ldg(row_ids + s);
-    if (beta < 0 || beta >= a.nblk || (int64_t)beta * BLK >= lim) continue;
-    M = fmaxf(M, __ldg(a.part_lse + (p0 + s) * a.G + hi));
+  for (int s0 = 0; s0 < a.topk; s0 += 32) {
+    const int s = s0 + lane;
+    float l = ninf;
+    if (s < a.topk) {
+      const int beta = __ldg(row_ids + s);
+      if (beta >= 0 && beta < a.nblk && beta * BLK < lim) l = __ldg(a.part_lse + (p0 + s) * a.G + hi);
+    }
+    M = fmaxf(M, l);
   }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
   float acc[PER];
 #pragma unroll
   for (int e = 0; e < PER; ++e) acc[e] = 0.f;
   float den = 0.f;
   if (M != ninf) {
-    for (int s = 0; s < a.topk; ++s) {
-      const int beta = __ldg(row_ids + s);
-      if (beta < 0 || beta >= a.nblk || (int64_t)beta * BLK >= lim) continue;
-      const int64_t pr = (p0 + s) * a.G + hi;
-      const float wgt = __expf(__ldg(a.part_lse + pr) - M);
+    for (int s0 = 0; s0 < a.topk; s0 += 32) {
+      const int s = s0 + lane;
+      float wgt = 0.f;
+      if (s < a.topk) {
+        const int beta = __ldg(row_ids + s);
+        if (beta >= 0 && beta < a.nblk && beta * BLK < lim)
+          wgt = __expf(__ldg(a.part_lse + (p0 + s) * a.G + hi) - M);
+      }
       den += wgt;
-      const uint16_t* src = a.part_o + pr * D + lane * PER;
-      if constexpr (PER == 4) {
-        const uint2 u = *reinterpret_cast<const uint2*>(src);
-        acc[0] += wgt * __uint_as_float(u.x << 16);
-        acc[1] += wgt * __uint_as_float(u.x & 0xffff0000u);
-        acc[2] += wgt * __uint_as_float(u.y << 16);
-        acc[3] += wgt * __uint_as_float(u.y & 0xffff0000u);
-      } else {
-        const uint32_t u = *reinterpret_cast<const uint32_t*>(src);
-        acc[0] += wgt * __uint_as_float(u << 16);
-        acc[1] += wgt * __uint_as_float(u & 0xffff0000u);
+      const int cnt = min(32, a.topk - s0);
+#pragma unroll 8
+      for (int j = 0; j < cnt; ++j) {
+        const float wj = __shfl_sync(0xffffffffu, wgt, j);
+        if (wj == 0.f) continue;
+        const uint16_t* src = a.part_o + ((p0 + s0 + j) * a.G + hi) * D + lane * PER;
+        if constexpr (PER == 4) {
+          const uint2 u = __ldg(reinterpret_cast<const uint2*>(src));
+          acc[0] += wj * __uint_as_float(u.x << 16);
+          acc[1] += wj * __uint_as_float(u.x & 0xffff0000u);
+          acc[2] += wj * __uint_as_float(u.y << 16);
+          acc[3] += wj * __uint_as_float(u.y & 0xffff0000u);
+        } else {
+          const uint32_t u = __ldg(reinterpret_cast<const uint32_t*>(src));
+          acc[0] += wj * __uint_as_float(u << 16);
+          acc[1] += wj * __uint_as_float(u & 0xffff0000u);
+        }
       }
     }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
   }
   const float inv = den > 0.f ? 1.f / den : 0.f;
   uint16_t* o = a.out + (int64_t)b * a.o_s0 + (int64_t)t * a.o_s1 + (int64_t)hq * a.o_s2 + lane * PER;
-#pragma unroll
-  for (int e = 0; e < PER; ++e) o[e] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[e] * inv));
-  if (lane == 0 && a.lse) a.lse[bt * a.H + hq] = M != ninf ? M + __logf(den) : ninf;
+  if constexpr (PER == 4) {
+    *reinterpret_cast<uint2*>(o) = make_uint2(pack_bf16(acc[0] * inv, acc[1] * inv),
+                                              pack_bf16(acc[2] * inv, acc[3] * inv));
+  } else {
+    *reinterpret_cast<uint32_t*>(o) = pack_bf16(acc[0] * inv, acc[1] * inv);
+  }
+  if (lane == 0 && a.lse) a.lse[(int64_t)bt * a.H + hq] = M != ninf ? M + __logf(den) : ninf;
 }
 
 }  // namespace
@@ -629,7 +659,7 @@ KvPlan plan_kv(const Shape& s) {
 template <int D, int BLK>
 cudaError_t run_kv(const Shape& s, KvArgs& a, const KvPlan& p, const CUtensorMap& tmk,
                    const CUtensorMap& tmv, uint8_t* ws, cudaStream_t stream) {
-  constexpr uint32_t smem = 1024 + 2 * (kRows * (D > BLK ? D : BLK) * 2) + 2 * (4 * D * BLK) + 19 * 8 + 16;
+  constexpr uint32_t smem = 1024 + 2 * (kRows * (D > BLK ? D : BLK) * 2) + 2 * (4 * D * BLK) + 256 + 2 * kRows * 8;
   cudaError_t err = cudaFuncSetAttribute(kv_attn_kernel<D, BLK>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (err != cudaSuccess) return err;
