@@ -465,12 +465,22 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--batch", type=int, default=0,
                     help="override the workload's batch (for small profiling captures)")
+    ap.add_argument("--seq", type=int, default=0,
+                    help="override the sequence length (prefill: queries and context; decode: "
+                         "context) for small profiling captures")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     prob = WORKLOADS[args.workload]
     if args.batch:
         prob = prob.with_(batch=args.batch)
+    if args.seq:
+        if prob.is_decode:
+            lr = prob.len_range
+            prob = prob.with_(max_kv=args.seq,
+                              len_range=None if lr is None else (min(lr[0], args.seq), args.seq))
+        else:
+            prob = prob.with_(n_q=args.seq, max_kv=args.seq)
     world, rank, local = dist_setup(args)
     try:
         if args.impl == "reference":

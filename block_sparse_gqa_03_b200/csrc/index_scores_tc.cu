@@ -299,7 +299,7 @@ cudaError_t launch_index_scores_tc(const Shape& s, const uint16_t* q_idx, const 
   a.scores = scores;
   a.fill_tail = fill_tail ? 1 : 0;
   a.st = st;
-  a.wait_ns = 500000000ull;
+  a.wait_ns = 4000000000ull;
 #define MSA_TC_CASE(DI_, BLK_) \
   if (s.d_idx == DI_ && s.block == BLK_) return run_tc<DI_, BLK_>(s, q_idx, k_idx, a, stream);
   MSA_TC_CASE(128, 16)

@@ -704,7 +704,7 @@ cudaError_t launch_sparse_attn(const Shape& s, const uint16_t* q, const uint16_t
   a.o_s2 = s.o_s[2];
   a.lse = lse;
   a.st = st;
-  a.wait_ns = 500000000ull;  // 0.5 s; a healthy wait takes microseconds
+  a.wait_ns = 4000000000ull;  // 4 s: far above any healthy wait, even under a profiler
   cudaError_t err;
   if (!pl.stream && kv_attn_supported(s))
     return launch_kv_attn(s, tmk, tmv, q, ids, out, lse, partials, partial_bytes, st, stream);

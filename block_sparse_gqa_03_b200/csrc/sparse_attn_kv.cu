@@ -20,10 +20,11 @@
 //
 // CTA roles (persistent CTAs, each a contiguous share of the chunk's tiles):
 //   warp 0      TMA producer of K and V (a new load only when the block changes);
-//   warp 1      tensor-memory allocation and the single MMA-issuing thread;
-//   warps 2-5   gather the tile's Q rows with 16-byte async copies (swizzled): the
-//               tile's query rows are resolved once into a shared table, then
-//               the copies are issued in a tight loop;
+//   warp 1      tensor-memory allocation and the thread issuing the S = Q K^T MMAs;
+//   warp 14     the thread issuing the O = P V MMAs (independent of the first, so
+//               neither kind waits on the other's inputs);
+//   warps 2-5   gather the tile's Q rows with 16-byte async copies (swizzled), one
+//               thread per row;
 //   warps 6-13  softmax and output epilogue, one thread per tile row; two warp
 //               groups take alternate tiles so one computes while the other waits.
 // Double buffers: Q/P tiles (P overwrites Q once S is computed), K/V stages, and
@@ -35,8 +36,8 @@ namespace msa {
 namespace {
 
 constexpr int kRows = 128;                  // MMA M: (query, head) rows per tile
-constexpr int kKvThreads = 14 * 32;
-constexpr int kWarpProd = 0, kWarpMma = 1, kWarpGather0 = 2, kWarpSoft0 = 6;
+constexpr int kKvThreads = 15 * 32;
+constexpr int kWarpProd = 0, kWarpMma = 1, kWarpGather0 = 2, kWarpSoft0 = 6, kWarpPv = 14;
 
 struct KvArgs {
   // problem
@@ -227,9 +228,8 @@ __global__ void __launch_bounds__(kKvThreads, 1)
   const uint32_t b_qfull = b_kvempty + 16, b_qempty = b_qfull + 16;
   const uint32_t b_sfull = b_qempty + 16, b_sfree = b_sfull + 16;
   const uint32_t b_pfull = b_sfree + 16, b_ofull = b_pfull + 16;
-  const uint32_t b_ofree = b_ofull + 16, b_done = b_ofree + 16;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 19);
-  uint64_t* qsrc = bars + 32;  // [2][kRows] source row of each query of a tile
+  const uint32_t b_ofree = b_ofull + 16, b_done = b_ofree + 16, b_done2 = b_done + 8;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 20);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ntiles = __ldg(a.toffs + a.nj);
@@ -250,6 +250,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
       mbar_init(b_ofree + 8 * i, 4);
     }
     mbar_init(b_done, 1);
+    mbar_init(b_done2, 1);
     fence_mbar_init();
   }
   if (warp == kWarpMma) {
@@ -293,71 +294,76 @@ __global__ void __launch_bounds__(kKvThreads, 1)
           mbar_wait_bounded(b_kvempty + 8 * (u & 1), (u >> 1) & 1, a.st, 0x202u, a.wait_ns);
       }
     } else if (warp == kWarpMma) {
-      // ---------------------------------------------------------- MMA issue
+      // ------------------------------------------------------ S = Q K^T issue
       if (lane == 0) {
         const uint32_t id_qk = tc::idesc_bf16(kRows, BLK, false);
-        const uint32_t id_pv = tc::idesc_bf16(kRows, D, true);
-        int use = -1, prev_j = -1;
-        int kv_stage_of[2] = {0, 0};
+        int use = -1, prev_j = -1, i = 0;
         bool ok = true;
-        int i = 0;
-        for (int tile = tile0; tile <= tile1 && ok; ++tile, ++i) {
-          // QK of tile i (if any), then PV of tile i - 1.
-          if (tile < tile1) {
-            w.advance(a, tile);
-            if (w.j != prev_j) {
-              prev_j = w.j;
-              ++use;
-              ok = mbar_wait_bounded(b_kvfull + 8 * (use & 1), (use >> 1) & 1, a.st, 0x203u,
-                                     a.wait_ns);
-            }
-            const int buf = i & 1;
-            kv_stage_of[buf] = use;
-            if (ok) ok = mbar_wait_bounded(b_qfull + 8 * buf, (i >> 1) & 1, a.st, 0x204u, a.wait_ns);
-            if (ok && i >= 2)
-              ok = mbar_wait_bounded(b_sfree + 8 * buf, ((i >> 1) - 1) & 1, a.st, 0x205u, a.wait_ns);
-            if (!ok) break;
-            tc::fence_after_sync();
-            const uint32_t kd = skv + (use & 1) * KV_BYTES;
-#pragma unroll
-            for (int ks = 0; ks < D / 16; ++ks) {
-              const uint32_t koff = (ks >> 2) * (kRows * 128u) + (ks & 3) * 32;
-              const uint32_t kboff = (ks >> 2) * HALF + (ks & 3) * 32;
-              tc::mma_bf16(tmem + TM_S + buf * BLK, tc::desc_k_sw128(sqp + buf * QP_BYTES + koff),
-                           tc::desc_k_sw128(kd + kboff), id_qk, ks > 0 ? 1u : 0u);
-            }
-            tc::commit(b_sfull + 8 * buf);
+        for (int tile = tile0; tile < tile1 && ok; ++tile, ++i) {
+          w.advance(a, tile);
+          if (w.j != prev_j) {
+            prev_j = w.j;
+            ++use;
+            ok = mbar_wait_bounded(b_kvfull + 8 * (use & 1), (use >> 1) & 1, a.st, 0x203u,
+                                   a.wait_ns);
           }
-          if (i >= 1) {
-            const int pi = i - 1, pbuf = pi & 1;
-            ok = mbar_wait_bounded(b_pfull + 8 * pbuf, (pi >> 1) & 1, a.st, 0x206u, a.wait_ns);
-            if (ok && pi >= 2)
-              ok = mbar_wait_bounded(b_ofree + 8 * pbuf, ((pi >> 1) - 1) & 1, a.st, 0x207u,
-                                     a.wait_ns);
-            if (!ok) break;
-            tc::fence_after_sync();
-            const int pu = kv_stage_of[pbuf];
-            const uint32_t vd = skv + (pu & 1) * KV_BYTES + NH * HALF;
+          const int buf = i & 1;
+          if (ok) ok = mbar_wait_bounded(b_qfull + 8 * buf, (i >> 1) & 1, a.st, 0x204u, a.wait_ns);
+          if (ok && i >= 2)
+            ok = mbar_wait_bounded(b_sfree + 8 * buf, ((i >> 1) - 1) & 1, a.st, 0x205u, a.wait_ns);
+          if (!ok) break;
+          tc::fence_after_sync();
+          const uint32_t kd = skv + (use & 1) * KV_BYTES;
 #pragma unroll
-            for (int ks = 0; ks < BLK / 16; ++ks) {
-              const uint32_t poff = (ks >> 2) * (kRows * 128u) + (ks & 3) * 32;
-              tc::mma_bf16(tmem + TM_O + pbuf * D, tc::desc_k_sw128(sqp + pbuf * QP_BYTES + poff),
-                           tc::desc_mn_sw128(vd + ks * 16 * 128, HALF), id_pv, ks > 0 ? 1u : 0u);
-            }
-            tc::commit(b_ofull + 8 * pbuf);
-            tc::commit(b_qempty + 8 * pbuf);  // the Q/P buffer may be refilled
-            // Release the K/V stage after the last tile that reads it.
-            bool last_use = true;
-            if (tile < tile1) last_use = kv_stage_of[(i) & 1] != pu;
-            if (last_use) tc::commit(b_kvempty + 8 * (pu & 1));
+          for (int ks = 0; ks < D / 16; ++ks) {
+            const uint32_t koff = (ks >> 2) * (kRows * 128u) + (ks & 3) * 32;
+            const uint32_t kboff = (ks >> 2) * HALF + (ks & 3) * 32;
+            tc::mma_bf16(tmem + TM_S + buf * BLK, tc::desc_k_sw128(sqp + buf * QP_BYTES + koff),
+                         tc::desc_k_sw128(kd + kboff), id_qk, ks > 0 ? 1u : 0u);
           }
+          tc::commit(b_sfull + 8 * buf);
         }
         tc::commit(b_done);
         mbar_wait_bounded(b_done, 0, a.st, 0x208u, a.wait_ns);
       }
+    } else if (warp == kWarpPv) {
+      // ------------------------------------------------------- O = P V issue
+      if (lane == 0) {
+        const uint32_t id_pv = tc::idesc_bf16(kRows, D, true);
+        int use = -1, prev_j = -1, i = 0;
+        bool ok = true;
+        for (int tile = tile0; tile < tile1 && ok; ++tile, ++i) {
+          w.advance(a, tile);
+          if (w.j != prev_j) {
+            prev_j = w.j;
+            ++use;
+          }
+          const int buf = i & 1;
+          ok = mbar_wait_bounded(b_pfull + 8 * buf, (i >> 1) & 1, a.st, 0x206u, a.wait_ns);
+          if (ok && i >= 2)
+            ok = mbar_wait_bounded(b_ofree + 8 * buf, ((i >> 1) - 1) & 1, a.st, 0x207u, a.wait_ns);
+          if (!ok) break;
+          tc::fence_after_sync();
+          const uint32_t vd = skv + (use & 1) * KV_BYTES + NH * HALF;
+#pragma unroll
+          for (int ks = 0; ks < BLK / 16; ++ks) {
+            const uint32_t poff = (ks >> 2) * (kRows * 128u) + (ks & 3) * 32;
+            tc::mma_bf16(tmem + TM_O + buf * D, tc::desc_k_sw128(sqp + buf * QP_BYTES + poff),
+                         tc::desc_mn_sw128(vd + ks * 16 * 128, HALF), id_pv, ks > 0 ? 1u : 0u);
+          }
+          tc::commit(b_ofull + 8 * buf);
+          tc::commit(b_qempty + 8 * buf);  // the Q/P buffer may be refilled
+          // Release the K/V stage after the last tile that reads it (its S MMAs
+          // finished before the softmax that fed this P).
+          const bool last_use = tile + 1 >= tile1 || __ldg(a.toffs + w.j + 1) <= tile + 1;
+          if (last_use) tc::commit(b_kvempty + 8 * (use & 1));
+        }
+        tc::commit(b_done2);
+        mbar_wait_bounded(b_done2, 0, a.st, 0x20cu, a.wait_ns);
+      }
     } else if (warp < kWarpSoft0) {
       // ----------------------------------------------------- Q gather warps
-      const int gt = threadIdx.x - kWarpGather0 * 32;  // 0..127
+      const int row = threadIdx.x - kWarpGather0 * 32;  // 0..127: one tile row each
       int i = 0;
       bool ok = true;
       constexpr int CPR = D / 8;  // 16-byte chunks per row
@@ -367,26 +373,17 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         if (i >= 2 && ok)
           ok = mbar_wait_bounded(b_qempty + 8 * buf, ((i >> 1) - 1) & 1, a.st, 0x209u, a.wait_ns);
         const TileInfo ti = tile_info(a, w.j, tile);
-        uint64_t* tab = qsrc + buf * kRows;
-        if (ok && gt < ti.nq) {
-          // the query of this list entry: chunk-relative slot position -> (b, t)
-          const int pos = __ldg(a.entries + ti.first + gt);
+        if (ok && row < ti.nq * a.G) {
+          const int qi = row / a.G, hi = row - qi * a.G;
+          const int pos = __ldg(a.entries + ti.first + qi);  // chunk-relative slot position
           const int bt = (int)a.bt0 + pos / (a.h * a.topk);
-          const int t = bt % a.n_q;
-          tab[gt] = reinterpret_cast<uint64_t>(a.q + (int64_t)ti.b * a.q_s0 + (int64_t)t * a.q_s1 +
-                                               (int64_t)(ti.g * a.G) * a.q_s2);
-        }
-        asm volatile("bar.sync 2, 128;" ::: "memory");
-        if (ok) {
-          const int nrows = ti.nq * a.G;
-          const uint32_t dst0 = sqp + buf * QP_BYTES;
-          for (int x = gt; x < nrows * CPR; x += 128) {
-            const int row = x / CPR, ch = x % CPR;
-            const int qi = row / a.G, hi = row - qi * a.G;
-            const uint16_t* src =
-                reinterpret_cast<const uint16_t*>(tab[qi]) + (int64_t)hi * a.q_s2 + ch * 8;
-            const uint32_t dst = dst0 + (ch >> 3) * (kRows * 128u) + swz128(row, ch & 7);
-            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src));
+          const uint16_t* src = a.q + (int64_t)ti.b * a.q_s0 + (int64_t)(bt % a.n_q) * a.q_s1 +
+                                (int64_t)(ti.g * a.G + hi) * a.q_s2;
+          const uint32_t dst0 = sqp + buf * QP_BYTES + row * 128u;
+#pragma unroll
+          for (int ch = 0; ch < CPR; ++ch) {
+            const uint32_t dst = dst0 + (ch >> 3) * (kRows * 128u) + (((ch & 7) ^ (row & 7)) << 4);
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src + ch * 8));
           }
         }
         asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
@@ -429,6 +426,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         // first, then probabilities, their sum and the bf16 P row (K-major, swizzled).
         const int vis = lim - ti.beta * BLK;  // keys [0, vis) of the block are visible
         const uint32_t srow = lane_base + TM_S + buf * BLK;
+        const bool full = vis >= BLK;  // every key of the block is visible to this row
         float mx = ninf;
 #pragma unroll
         for (int c = 0; c < BLK / 32; c += 2) {
@@ -436,11 +434,20 @@ __global__ void __launch_bounds__(kKvThreads, 1)
           tc::tmem_ld32(srow + c * 32, v0);
           tc::tmem_ld32(srow + c * 32 + 32, v1);
           tc::tmem_wait_ld();
+          if (!full) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            mx = fmaxf(mx, c * 32 + e < vis ? v0[e] : ninf);
-            mx = fmaxf(mx, c * 32 + 32 + e < vis ? v1[e] : ninf);
+            for (int e = 0; e < 32; ++e) {
+              v0[e] = c * 32 + e < vis ? v0[e] : ninf;
+              v1[e] = c * 32 + 32 + e < vis ? v1[e] : ninf;
+            }
           }
+          float m4[4] = {ninf, ninf, ninf, ninf};
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            m4[(e >> 1) & 1] = fmax3(m4[(e >> 1) & 1], v0[e], v0[e + 1]);
+            m4[2 + ((e >> 1) & 1)] = fmax3(m4[2 + ((e >> 1) & 1)], v1[e], v1[e + 1]);
+          }
+          mx = fmax3(mx, fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
         }
         mx *= a.scale_log2;
         const float msafe = live && mx != ninf ? mx : 0.f;
@@ -452,11 +459,16 @@ __global__ void __launch_bounds__(kKvThreads, 1)
           tc::tmem_ld32(srow + c * 32, *reinterpret_cast<float(*)[32]>(v));
           tc::tmem_ld32(srow + c * 32 + 32, *reinterpret_cast<float(*)[32]>(v + 32));
           tc::tmem_wait_ld();
+          float l4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-          for (int e = 0; e < 64; ++e) {
-            v[e] = c * 32 + e < vis ? exp2f(v[e] * a.scale_log2 - msafe) : 0.f;
-            l += v[e];
+          for (int e = 0; e < 64; ++e) v[e] = exp2_approx(fmaf(v[e], a.scale_log2, -msafe));
+          if (!full) {
+#pragma unroll
+            for (int e = 0; e < 64; ++e) v[e] = c * 32 + e < vis ? v[e] : 0.f;
           }
+#pragma unroll
+          for (int e = 0; e < 64; ++e) l4[e & 3] += v[e];
+          l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
 #pragma unroll
           for (int q8 = 0; q8 < 8; ++q8) {
             const int ch = c * 4 + q8;  // 16-byte chunk of the P row
@@ -577,21 +589,25 @@ __global__ void __launch_bounds__(256) kv_combine_kernel(KvArgs a, int BLK) {
       }
       den += wgt;
       const int cnt = min(32, a.topk - s0);
-#pragma unroll 8
+      // Loads are issued for every slot of the pass (the buffer is allocated for all
+      // of them); a slot without a partial contributes through a select, never a
+      // multiply, so whatever its memory holds cannot leak into the sum.
+#pragma unroll 4
       for (int j = 0; j < cnt; ++j) {
         const float wj = __shfl_sync(0xffffffffu, wgt, j);
-        if (wj == 0.f) continue;
         const uint16_t* src = a.part_o + ((p0 + s0 + j) * a.G + hi) * D + lane * PER;
         if constexpr (PER == 4) {
           const uint2 u = __ldg(reinterpret_cast<const uint2*>(src));
-          acc[0] += wj * __uint_as_float(u.x << 16);
-          acc[1] += wj * __uint_as_float(u.x & 0xffff0000u);
-          acc[2] += wj * __uint_as_float(u.y << 16);
-          acc[3] += wj * __uint_as_float(u.y & 0xffff0000u);
+          const bool use = wj != 0.f;
+          acc[0] += use ? wj * __uint_as_float(u.x << 16) : 0.f;
+          acc[1] += use ? wj * __uint_as_float(u.x & 0xffff0000u) : 0.f;
+          acc[2] += use ? wj * __uint_as_float(u.y << 16) : 0.f;
+          acc[3] += use ? wj * __uint_as_float(u.y & 0xffff0000u) : 0.f;
         } else {
           const uint32_t u = __ldg(reinterpret_cast<const uint32_t*>(src));
-          acc[0] += wj * __uint_as_float(u << 16);
-          acc[1] += wj * __uint_as_float(u & 0xffff0000u);
+          const bool use = wj != 0.f;
+          acc[0] += use ? wj * __uint_as_float(u << 16) : 0.f;
+          acc[1] += use ? wj * __uint_as_float(u & 0xffff0000u) : 0.f;
         }
       }
     }
@@ -659,7 +675,7 @@ KvPlan plan_kv(const Shape& s) {
 template <int D, int BLK>
 cudaError_t run_kv(const Shape& s, KvArgs& a, const KvPlan& p, const CUtensorMap& tmk,
                    const CUtensorMap& tmv, uint8_t* ws, cudaStream_t stream) {
-  constexpr uint32_t smem = 1024 + 2 * (kRows * (D > BLK ? D : BLK) * 2) + 2 * (4 * D * BLK) + 256 + 2 * kRows * 8;
+  constexpr uint32_t smem = 1024 + 2 * (kRows * (D > BLK ? D : BLK) * 2) + 2 * (4 * D * BLK) + 256;
   cudaError_t err = cudaFuncSetAttribute(kv_attn_kernel<D, BLK>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (err != cudaSuccess) return err;
@@ -730,7 +746,7 @@ cudaError_t launch_kv_attn(const Shape& s, const CUtensorMap& tmk, const CUtenso
   a.o_s2 = s.o_s[2];
   a.lse = lse;
   a.st = st;
-  a.wait_ns = 500000000ull;
+  a.wait_ns = 4000000000ull;
   if (s.d == 128 && s.block == 128) return run_kv<128, 128>(s, a, p, tmk, tmv, w, stream);
   if (s.d == 128 && s.block == 64) return run_kv<128, 64>(s, a, p, tmk, tmv, w, stream);
   if (s.d == 64 && s.block == 128) return run_kv<64, 128>(s, a, p, tmk, tmv, w, stream);
