@@ -21,14 +21,15 @@
 // CTA roles (persistent CTAs, each a contiguous share of the chunk's tiles):
 //   warp 0      TMA producer of K and V (a new load only when the block changes);
 //   warp 1      tensor-memory allocation and the thread issuing the S = Q K^T MMAs;
-//   warp 14     the thread issuing the O = P V MMAs (independent of the first, so
-//               neither kind waits on the other's inputs);
 //   warps 2-5   gather the tile's Q rows with 16-byte async copies (swizzled), one
 //               thread per row;
-//   warps 6-13  softmax and output epilogue, one thread per tile row; two warp
-//               groups take alternate tiles so one computes while the other waits.
-// Double buffers: Q/P tiles (P overwrites Q once S is computed), K/V stages, and
-// S and O in tensor memory.  Every wait is bounded.
+//   warps 6-17  three softmax warp groups taking tiles in turn, one thread per tile
+//               row: softmax from tensor memory, the P tile into shared memory, then
+//               (one elected thread) the O = P V MMA, then the output epilogue.
+// Buffers: 3-4 Q/P tiles (P overwrites its Q once S is computed), 2 K/V stages
+// (each released by every warp group once its products are done), and 4 tile
+// buffers in tensor memory where O = P V overwrites the S it was computed from.
+// Every wait is bounded.
 #include "kernels.h"
 #include "sm100.cuh"
 
@@ -36,8 +37,9 @@ namespace msa {
 namespace {
 
 constexpr int kRows = 128;                  // MMA M: (query, head) rows per tile
-constexpr int kKvThreads = 15 * 32;
-constexpr int kWarpProd = 0, kWarpMma = 1, kWarpGather0 = 2, kWarpSoft0 = 6, kWarpPv = 14;
+constexpr int kNw = 3;                     // softmax warp groups
+constexpr int kKvThreads = (6 + 4 * kNw) * 32;
+constexpr int kWarpProd = 0, kWarpMma = 1, kWarpGather0 = 2, kWarpSoft0 = 6;
 
 struct KvArgs {
   // problem
@@ -206,30 +208,46 @@ __device__ __forceinline__ TileInfo tile_info(const KvArgs& a, int j, int tile) 
 }
 
 // --------------------------------------------------------- attention tiles
+// Shared-memory plan of the attention kernel for one (D, BLK).
+template <int D, int BLK>
+struct KvSmem {
+  static constexpr uint32_t QP = kRows * (D > BLK ? D : BLK) * 2;  // a Q tile or a P tile
+  static constexpr uint32_t HALF = BLK * 128u;                     // one 64-dim atom of K or V
+  static constexpr uint32_t KV = 2 * (D / 64) * HALF;              // K and V of one block
+  static constexpr int NQ = (4 * QP + 2 * KV + 2048 <= 227u * 1024u) ? 4 : 3;
+  static constexpr uint32_t BYTES = 1024 + NQ * QP + 2 * KV + 512;
+};
+
 template <int D, int BLK>
 __global__ void __launch_bounds__(kKvThreads, 1)
     kv_attn_kernel(const __grid_constant__ CUtensorMap tmk,
                    const __grid_constant__ CUtensorMap tmv, KvArgs a) {
-  constexpr int NH = D / 64;                  // 64-dim atoms of a head row
-  constexpr uint32_t QP_BYTES = kRows * (D > BLK ? D : BLK) * 2;  // a Q tile or a P tile
-  constexpr uint32_t HALF = BLK * 128u;       // one 64-dim atom of a K or V block
-  constexpr uint32_t KV_BYTES = 2 * NH * HALF;
-  constexpr uint32_t TM_S = 0, TM_O = 2 * BLK;  // tensor-memory columns: S[2], O[2]
-  constexpr uint32_t TMEM_COLS = 2 * BLK + 2 * D <= 256 ? 256 : 512;
-  static_assert(QP_BYTES >= kRows * BLK * 2, "P tile must fit the Q buffer");
+  using SM = KvSmem<D, BLK>;
+  constexpr int NH = D / 64;
+  constexpr int NQ = SM::NQ;                  // Q/P tile buffers
+  constexpr int NB = 4;                       // tensor-memory tile buffers
+  constexpr uint32_t TB = D > BLK ? D : BLK;  // columns per buffer: S, then O in place
+  constexpr uint32_t QP_BYTES = SM::QP, HALF = SM::HALF, KV_BYTES = SM::KV;
+  constexpr uint32_t TMEM_COLS = NB * TB <= 256 ? 256 : 512;
+  static_assert(NB * TB <= 512, "tensor memory");
   if (status_failed(a.st)) return;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  const uint32_t sqp = smem_u32(smem);            // 2 x QP_BYTES
-  const uint32_t skv = sqp + 2 * QP_BYTES;        // 2 x KV_BYTES
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 2 * QP_BYTES + 2 * KV_BYTES);
-  const uint32_t b_kvfull = smem_u32(bars), b_kvempty = b_kvfull + 16;
-  const uint32_t b_qfull = b_kvempty + 16, b_qempty = b_qfull + 16;
-  const uint32_t b_sfull = b_qempty + 16, b_sfree = b_sfull + 16;
-  const uint32_t b_pfull = b_sfree + 16, b_ofull = b_pfull + 16;
-  const uint32_t b_ofree = b_ofull + 16, b_done = b_ofree + 16, b_done2 = b_done + 8;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 20);
+  const uint32_t sm0a = smem_u32(smem);
+  const uint32_t sqp = sm0a;                     // NQ x QP_BYTES
+  const uint32_t skv = sqp + NQ * QP_BYTES;      // 2 x KV_BYTES
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + NQ * QP_BYTES + 2 * KV_BYTES);
+  // barrier blocks (8 bytes each)
+  const uint32_t b_kvfull = smem_u32(bars);                 // [2]
+  const uint32_t b_kvempty = b_kvfull + 16;                 // [2][kNw]
+  const uint32_t b_qfull = b_kvempty + 16 * kNw;            // [NQ]
+  const uint32_t b_qempty = b_qfull + 8 * NQ;               // [NQ]
+  const uint32_t b_sfull = b_qempty + 8 * NQ;               // [NB]
+  const uint32_t b_ofull = b_sfull + 8 * NB;                // [NB]
+  const uint32_t b_ofree = b_ofull + 8 * NB;                // [NB]
+  const uint32_t b_done = b_ofree + 8 * NB;                 // [1 + kNw]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + NQ * QP_BYTES + 2 * KV_BYTES + 480);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ntiles = __ldg(a.toffs + a.nj);
@@ -238,19 +256,20 @@ __global__ void __launch_bounds__(kKvThreads, 1)
   const int tile1 = min(ntiles, tile0 + per);
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(b_kvfull + 8 * i, 1);
-      mbar_init(b_kvempty + 8 * i, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(b_kvfull + 8 * s, 1);
+      for (int w = 0; w < kNw; ++w) mbar_init(b_kvempty + 8 * (s * kNw + w), 1);
+    }
+    for (int i = 0; i < NQ; ++i) {
       mbar_init(b_qfull + 8 * i, 128);
       mbar_init(b_qempty + 8 * i, 1);
+    }
+    for (int i = 0; i < NB; ++i) {
       mbar_init(b_sfull + 8 * i, 1);
-      mbar_init(b_sfree + 8 * i, 4);
-      mbar_init(b_pfull + 8 * i, 4);
       mbar_init(b_ofull + 8 * i, 1);
       mbar_init(b_ofree + 8 * i, 4);
     }
-    mbar_init(b_done, 1);
-    mbar_init(b_done2, 1);
+    for (int i = 0; i <= kNw; ++i) mbar_init(b_done + 8 * i, 1);
     fence_mbar_init();
   }
   if (warp == kWarpMma) {
@@ -271,15 +290,18 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         prefetch_tensormap(&tmk);
         prefetch_tensormap(&tmv);
         int use = -1, prev_j = -1, issued = 0;
-        for (int tile = tile0; tile < tile1; ++tile) {
+        bool ok = true;
+        for (int tile = tile0; tile < tile1 && ok; ++tile) {
           w.advance(a, tile);
           if (w.j == prev_j) continue;
           prev_j = w.j;
           ++use;
           const int s = use & 1;
-          if (use >= 2 &&
-              !mbar_wait_bounded(b_kvempty + 8 * s, ((use >> 1) - 1) & 1, a.st, 0x201u, a.wait_ns))
-            break;
+          if (use >= 2)
+            for (int g = 0; g < kNw && ok; ++g)
+              ok = mbar_wait_bounded(b_kvempty + 8 * (s * kNw + g), ((use >> 1) - 1) & 1, a.st,
+                                     0x201u, a.wait_ns);
+          if (!ok) break;
           const TileInfo ti = tile_info(a, w.j, tile);
           mbar_arrive_expect_tx(b_kvfull + 8 * s, KV_BYTES);
           const uint32_t kd = skv + s * KV_BYTES, vd = kd + NH * HALF;
@@ -290,8 +312,12 @@ __global__ void __launch_bounds__(kKvThreads, 1)
           }
           issued = use + 1;
         }
+        // drain: the stages of the last two blocks are released once every
+        // warp group's O = P V products that read them have completed
         for (int u = max(0, issued - 2); u < issued; ++u)
-          mbar_wait_bounded(b_kvempty + 8 * (u & 1), (u >> 1) & 1, a.st, 0x202u, a.wait_ns);
+          for (int g = 0; g < kNw; ++g)
+            mbar_wait_bounded(b_kvempty + 8 * ((u & 1) * kNw + g), (u >> 1) & 1, a.st, 0x202u,
+                              a.wait_ns);
       }
     } else if (warp == kWarpMma) {
       // ------------------------------------------------------ S = Q K^T issue
@@ -307,10 +333,10 @@ __global__ void __launch_bounds__(kKvThreads, 1)
             ok = mbar_wait_bounded(b_kvfull + 8 * (use & 1), (use >> 1) & 1, a.st, 0x203u,
                                    a.wait_ns);
           }
-          const int buf = i & 1;
-          if (ok) ok = mbar_wait_bounded(b_qfull + 8 * buf, (i >> 1) & 1, a.st, 0x204u, a.wait_ns);
-          if (ok && i >= 2)
-            ok = mbar_wait_bounded(b_sfree + 8 * buf, ((i >> 1) - 1) & 1, a.st, 0x205u, a.wait_ns);
+          const int qb = i % NQ, tb = i % NB;
+          if (ok) ok = mbar_wait_bounded(b_qfull + 8 * qb, (i / NQ) & 1, a.st, 0x204u, a.wait_ns);
+          if (ok && i >= NB)
+            ok = mbar_wait_bounded(b_ofree + 8 * tb, ((i / NB) - 1) & 1, a.st, 0x205u, a.wait_ns);
           if (!ok) break;
           tc::fence_after_sync();
           const uint32_t kd = skv + (use & 1) * KV_BYTES;
@@ -318,48 +344,13 @@ __global__ void __launch_bounds__(kKvThreads, 1)
           for (int ks = 0; ks < D / 16; ++ks) {
             const uint32_t koff = (ks >> 2) * (kRows * 128u) + (ks & 3) * 32;
             const uint32_t kboff = (ks >> 2) * HALF + (ks & 3) * 32;
-            tc::mma_bf16(tmem + TM_S + buf * BLK, tc::desc_k_sw128(sqp + buf * QP_BYTES + koff),
+            tc::mma_bf16(tmem + tb * TB, tc::desc_k_sw128(sqp + qb * QP_BYTES + koff),
                          tc::desc_k_sw128(kd + kboff), id_qk, ks > 0 ? 1u : 0u);
           }
-          tc::commit(b_sfull + 8 * buf);
+          tc::commit(b_sfull + 8 * tb);
         }
         tc::commit(b_done);
         mbar_wait_bounded(b_done, 0, a.st, 0x208u, a.wait_ns);
-      }
-    } else if (warp == kWarpPv) {
-      // ------------------------------------------------------- O = P V issue
-      if (lane == 0) {
-        const uint32_t id_pv = tc::idesc_bf16(kRows, D, true);
-        int use = -1, prev_j = -1, i = 0;
-        bool ok = true;
-        for (int tile = tile0; tile < tile1 && ok; ++tile, ++i) {
-          w.advance(a, tile);
-          if (w.j != prev_j) {
-            prev_j = w.j;
-            ++use;
-          }
-          const int buf = i & 1;
-          ok = mbar_wait_bounded(b_pfull + 8 * buf, (i >> 1) & 1, a.st, 0x206u, a.wait_ns);
-          if (ok && i >= 2)
-            ok = mbar_wait_bounded(b_ofree + 8 * buf, ((i >> 1) - 1) & 1, a.st, 0x207u, a.wait_ns);
-          if (!ok) break;
-          tc::fence_after_sync();
-          const uint32_t vd = skv + (use & 1) * KV_BYTES + NH * HALF;
-#pragma unroll
-          for (int ks = 0; ks < BLK / 16; ++ks) {
-            const uint32_t poff = (ks >> 2) * (kRows * 128u) + (ks & 3) * 32;
-            tc::mma_bf16(tmem + TM_O + buf * D, tc::desc_k_sw128(sqp + buf * QP_BYTES + poff),
-                         tc::desc_mn_sw128(vd + ks * 16 * 128, HALF), id_pv, ks > 0 ? 1u : 0u);
-          }
-          tc::commit(b_ofull + 8 * buf);
-          tc::commit(b_qempty + 8 * buf);  // the Q/P buffer may be refilled
-          // Release the K/V stage after the last tile that reads it (its S MMAs
-          // finished before the softmax that fed this P).
-          const bool last_use = tile + 1 >= tile1 || __ldg(a.toffs + w.j + 1) <= tile + 1;
-          if (last_use) tc::commit(b_kvempty + 8 * (use & 1));
-        }
-        tc::commit(b_done2);
-        mbar_wait_bounded(b_done2, 0, a.st, 0x20cu, a.wait_ns);
       }
     } else if (warp < kWarpSoft0) {
       // ----------------------------------------------------- Q gather warps
@@ -369,9 +360,9 @@ __global__ void __launch_bounds__(kKvThreads, 1)
       constexpr int CPR = D / 8;  // 16-byte chunks per row
       for (int tile = tile0; tile < tile1; ++tile, ++i) {
         w.advance(a, tile);
-        const int buf = i & 1;
-        if (i >= 2 && ok)
-          ok = mbar_wait_bounded(b_qempty + 8 * buf, ((i >> 1) - 1) & 1, a.st, 0x209u, a.wait_ns);
+        const int qb = i % NQ;
+        if (i >= NQ && ok)
+          ok = mbar_wait_bounded(b_qempty + 8 * qb, ((i / NQ) - 1) & 1, a.st, 0x209u, a.wait_ns);
         const TileInfo ti = tile_info(a, w.j, tile);
         if (ok && row < ti.nq * a.G) {
           const int qi = row / a.G, hi = row - qi * a.G;
@@ -379,7 +370,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
           const int bt = (int)a.bt0 + pos / (a.h * a.topk);
           const uint16_t* src = a.q + (int64_t)ti.b * a.q_s0 + (int64_t)(bt % a.n_q) * a.q_s1 +
                                 (int64_t)(ti.g * a.G + hi) * a.q_s2;
-          const uint32_t dst0 = sqp + buf * QP_BYTES + row * 128u;
+          const uint32_t dst0 = sqp + qb * QP_BYTES + row * 128u;
 #pragma unroll
           for (int ch = 0; ch < CPR; ++ch) {
             const uint32_t dst = dst0 + (ch >> 3) * (kRows * 128u) + (((ch & 7) ^ (row & 7)) << 4);
@@ -388,28 +379,37 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         }
         asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
         fence_proxy_async_smem();
-        mbar_arrive(b_qfull + 8 * buf);
+        mbar_arrive(b_qfull + 8 * qb);
       }
     } else {
-      // ------------------------------------------- softmax and epilogue warps
-      const int wg = (warp - kWarpSoft0) >> 2;  // warp group: takes tiles with i % 2 == wg
+      // ------------------------- softmax, O = P V issue and epilogue (warp groups)
+      const int wg = (warp - kWarpSoft0) >> 2;  // takes tiles with i % kNw == wg
       const int quarter = warp & 3;
       const int row = quarter * 32 + lane;
+      const bool leader = ((warp - kWarpSoft0) & 3) == 0 && lane == 0;
       const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
       const float ninf = -__int_as_float(0x7f800000);
       const float kLn2 = 0.69314718055994531f;
-      uint8_t* const sm0 = smem;
-      const uint32_t sm0a = smem_u32(smem);
+      const uint32_t id_pv = tc::idesc_bf16(kRows, D, true);
       bool ok = true;
-      int i = 0, kv_use = -1, kv_prev_j = -1;
+      int i = 0, use = -1, prev_j = -1;
       for (int tile = tile0; tile < tile1; ++tile, ++i) {
         w.advance(a, tile);
-        if (w.j != kv_prev_j) {
-          kv_prev_j = w.j;
-          ++kv_use;
+        if (w.j != prev_j) {
+          // Leaving block `use`: this group's O = P V products that read it have
+          // all been issued; release its K/V stage once they complete.  The release
+          // waits until the producer has loaded that block, so that a group owning
+          // no tile of several short blocks never runs two phases ahead of the
+          // producer on the stage's barrier.
+          if (use >= 0 && leader) {
+            mbar_wait_bounded(b_kvfull + 8 * (use & 1), (use >> 1) & 1, a.st, 0x20du, a.wait_ns);
+            tc::commit(b_kvempty + 8 * ((use & 1) * kNw + wg));
+          }
+          prev_j = w.j;
+          ++use;
         }
-        if ((i & 1) != wg) continue;
-        const int buf = wg;
+        if (i % kNw != wg) continue;
+        const int qb = i % NQ, tb = i % NB;
         const TileInfo ti = tile_info(a, w.j, tile);
         const bool live = row < ti.nq * a.G;
         int pos = -1, hi = 0, lim = 0;
@@ -420,57 +420,52 @@ __global__ void __launch_bounds__(kKvThreads, 1)
           const int bt = (int)a.bt0 + pos / (a.h * a.topk);
           lim = visible_limit(a, ti.b, bt % a.n_q);
         }
-        if (ok) ok = mbar_wait_warp(b_sfull + 8 * buf, (i >> 1) & 1, a.st, 0x20bu, a.wait_ns);
+        if (ok) ok = mbar_wait_warp(b_sfull + 8 * tb, (i / NB) & 1, a.st, 0x20bu, a.wait_ns);
         tc::fence_after_sync();
-        // Scores from tensor memory, two 32-column loads per wait: the row maximum
-        // first, then probabilities, their sum and the bf16 P row (K-major, swizzled).
+        // Scores from tensor memory in 32-column pieces: the row maximum first,
+        // then probabilities, their sum and the bf16 P row (K-major, swizzled).
         const int vis = lim - ti.beta * BLK;  // keys [0, vis) of the block are visible
-        const uint32_t srow = lane_base + TM_S + buf * BLK;
-        const bool full = vis >= BLK;  // every key of the block is visible to this row
+        const bool full = vis >= BLK;
+        const uint32_t srow = lane_base + tb * TB;
         float mx = ninf;
 #pragma unroll
-        for (int c = 0; c < BLK / 32; c += 2) {
-          float v0[32], v1[32];
-          tc::tmem_ld32(srow + c * 32, v0);
-          tc::tmem_ld32(srow + c * 32 + 32, v1);
+        for (int c = 0; c < BLK / 32; ++c) {
+          float v[32];
+          tc::tmem_ld32(srow + c * 32, v);
           tc::tmem_wait_ld();
           if (!full) {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              v0[e] = c * 32 + e < vis ? v0[e] : ninf;
-              v1[e] = c * 32 + 32 + e < vis ? v1[e] : ninf;
-            }
+            for (int e = 0; e < 32; ++e) v[e] = c * 32 + e < vis ? v[e] : ninf;
           }
-          float m4[4] = {ninf, ninf, ninf, ninf};
+          float m2[2] = {ninf, ninf};
 #pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            m4[(e >> 1) & 1] = fmax3(m4[(e >> 1) & 1], v0[e], v0[e + 1]);
-            m4[2 + ((e >> 1) & 1)] = fmax3(m4[2 + ((e >> 1) & 1)], v1[e], v1[e + 1]);
+          for (int e = 0; e < 32; e += 4) {
+            m2[0] = fmax3(m2[0], v[e], v[e + 1]);
+            m2[1] = fmax3(m2[1], v[e + 2], v[e + 3]);
           }
-          mx = fmax3(mx, fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+          mx = fmax3(mx, m2[0], m2[1]);
         }
         mx *= a.scale_log2;
         const float msafe = live && mx != ninf ? mx : 0.f;
         float l = 0.f;
-        uint8_t* pbase = sm0 + (sqp + buf * QP_BYTES - sm0a);
+        uint8_t* pbase = smem + qb * QP_BYTES;
 #pragma unroll
-        for (int c = 0; c < BLK / 32; c += 2) {
-          float v[64];
-          tc::tmem_ld32(srow + c * 32, *reinterpret_cast<float(*)[32]>(v));
-          tc::tmem_ld32(srow + c * 32 + 32, *reinterpret_cast<float(*)[32]>(v + 32));
+        for (int c = 0; c < BLK / 32; ++c) {
+          float v[32];
+          tc::tmem_ld32(srow + c * 32, v);
           tc::tmem_wait_ld();
-          float l4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-          for (int e = 0; e < 64; ++e) v[e] = exp2_approx(fmaf(v[e], a.scale_log2, -msafe));
+          for (int e = 0; e < 32; ++e) v[e] = exp2_approx(fmaf(v[e], a.scale_log2, -msafe));
           if (!full) {
 #pragma unroll
-            for (int e = 0; e < 64; ++e) v[e] = c * 32 + e < vis ? v[e] : 0.f;
+            for (int e = 0; e < 32; ++e) v[e] = c * 32 + e < vis ? v[e] : 0.f;
           }
+          float l2[2] = {0.f, 0.f};
 #pragma unroll
-          for (int e = 0; e < 64; ++e) l4[e & 3] += v[e];
-          l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+          for (int e = 0; e < 32; ++e) l2[e & 1] += v[e];
+          l += l2[0] + l2[1];
 #pragma unroll
-          for (int q8 = 0; q8 < 8; ++q8) {
+          for (int q8 = 0; q8 < 4; ++q8) {
             const int ch = c * 4 + q8;  // 16-byte chunk of the P row
             const uint4 v4 = make_uint4(pack_bf16(v[8 * q8], v[8 * q8 + 1]),
                                         pack_bf16(v[8 * q8 + 2], v[8 * q8 + 3]),
@@ -480,9 +475,6 @@ __global__ void __launch_bounds__(kKvThreads, 1)
                 v4;
           }
         }
-        tc::fence_before_sync();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(b_sfree + 8 * buf);  // S may be overwritten
         // V rows at or past the sequence end may hold anything; zero them so that a
         // zero probability never meets a non-finite value (idempotent per stage).
         {
@@ -490,7 +482,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
           const int r0 = max(0, L - ti.beta * BLK);
           if (r0 < BLK) {
             const int per_h = (BLK - r0) * 8;
-            uint8_t* vb = sm0 + (skv - sm0a) + (kv_use & 1) * KV_BYTES + NH * HALF;
+            uint8_t* vb = smem + (skv - sm0a) + (use & 1) * KV_BYTES + NH * HALF;
             for (int x = row; x < per_h * NH; x += 128) {
               const int hh = x / per_h, rem = x % per_h;
               *reinterpret_cast<uint4*>(vb + hh * HALF + (r0 + rem / 8) * 128 + (rem % 8) * 16) =
@@ -498,27 +490,37 @@ __global__ void __launch_bounds__(kKvThreads, 1)
             }
           }
         }
+        // The P tile is complete once every warp of the group has written its rows.
         fence_proxy_async_smem();
         tc::fence_before_sync();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(b_pfull + 8 * buf);
+        asm volatile("bar.sync %0, 128;" ::"r"(3 + wg) : "memory");
+        if (leader && ok) {
+          tc::fence_after_sync();
+          const uint32_t vd = skv + (use & 1) * KV_BYTES + NH * HALF;
+#pragma unroll
+          for (int ks = 0; ks < BLK / 16; ++ks) {
+            const uint32_t poff = (ks >> 2) * (kRows * 128u) + (ks & 3) * 32;
+            tc::mma_bf16(tmem + tb * TB, tc::desc_k_sw128(sqp + qb * QP_BYTES + poff),
+                         tc::desc_mn_sw128(vd + ks * 16 * 128, HALF), id_pv, ks > 0 ? 1u : 0u);
+          }
+          tc::commit(b_ofull + 8 * tb);
+          tc::commit(b_qempty + 8 * qb);  // the Q/P buffer may be refilled
+        }
         // Output of this tile: O / l in bf16 and the log-sum-exp, for live rows.
         const float inv_l = l > 0.f ? 1.f / l : 0.f;
-        if (ok) ok = mbar_wait_warp(b_ofull + 8 * buf, (i >> 1) & 1, a.st, 0x20au, a.wait_ns);
+        if (ok) ok = mbar_wait_warp(b_ofull + 8 * tb, (i / NB) & 1, a.st, 0x20au, a.wait_ns);
         tc::fence_after_sync();
         const bool store = ok && live;
         uint16_t* dst = a.part_o + (store ? ((int64_t)pos * a.G + hi) * D : 0);
 #pragma unroll
-        for (int c = 0; c < D / 32; c += 2) {
-          float v[64];
-          tc::tmem_ld32(lane_base + TM_O + buf * D + c * 32, *reinterpret_cast<float(*)[32]>(v));
-          tc::tmem_ld32(lane_base + TM_O + buf * D + c * 32 + 32,
-                        *reinterpret_cast<float(*)[32]>(v + 32));
+        for (int c = 0; c < D / 32; ++c) {
+          float v[32];
+          tc::tmem_ld32(lane_base + tb * TB + c * 32, v);
           tc::tmem_wait_ld();
           if (store) {
             uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
 #pragma unroll
-            for (int e = 0; e < 8; ++e)
+            for (int e = 0; e < 4; ++e)
               d4[e] = make_uint4(pack_bf16(v[8 * e] * inv_l, v[8 * e + 1] * inv_l),
                                  pack_bf16(v[8 * e + 2] * inv_l, v[8 * e + 3] * inv_l),
                                  pack_bf16(v[8 * e + 4] * inv_l, v[8 * e + 5] * inv_l),
@@ -530,7 +532,16 @@ __global__ void __launch_bounds__(kKvThreads, 1)
               (mx != ninf && l > 0.f) ? (msafe + log2f(l)) * kLn2 : ninf;
         tc::fence_before_sync();
         __syncwarp();
-        if (lane == 0) mbar_arrive(b_ofree + 8 * buf);
+        if (lane == 0) mbar_arrive(b_ofree + 8 * tb);
+      }
+      if (leader) {
+        // release the last block, and wait for this group's products to complete
+        if (use >= 0) {
+          mbar_wait_bounded(b_kvfull + 8 * (use & 1), (use >> 1) & 1, a.st, 0x20du, a.wait_ns);
+          tc::commit(b_kvempty + 8 * ((use & 1) * kNw + wg));
+        }
+        tc::commit(b_done + 8 * (1 + wg));
+        mbar_wait_bounded(b_done + 8 * (1 + wg), 0, a.st, 0x20cu, a.wait_ns);
       }
     }
   }
@@ -588,26 +599,35 @@ __global__ void __launch_bounds__(256) kv_combine_kernel(KvArgs a, int BLK) {
           wgt = __expf(__ldg(a.part_lse + (p0 + s) * a.G + hi) - M);
       }
       den += wgt;
-      const int cnt = min(32, a.topk - s0);
       // Loads are issued for every slot of the pass (the buffer is allocated for all
       // of them); a slot without a partial contributes through a select, never a
-      // multiply, so whatever its memory holds cannot leak into the sum.
-#pragma unroll 4
-      for (int j = 0; j < cnt; ++j) {
-        const float wj = __shfl_sync(0xffffffffu, wgt, j);
-        const uint16_t* src = a.part_o + ((p0 + s0 + j) * a.G + hi) * D + lane * PER;
-        if constexpr (PER == 4) {
-          const uint2 u = __ldg(reinterpret_cast<const uint2*>(src));
-          const bool use = wj != 0.f;
-          acc[0] += use ? wj * __uint_as_float(u.x << 16) : 0.f;
-          acc[1] += use ? wj * __uint_as_float(u.x & 0xffff0000u) : 0.f;
-          acc[2] += use ? wj * __uint_as_float(u.y << 16) : 0.f;
-          acc[3] += use ? wj * __uint_as_float(u.y & 0xffff0000u) : 0.f;
-        } else {
-          const uint32_t u = __ldg(reinterpret_cast<const uint32_t*>(src));
-          const bool use = wj != 0.f;
-          acc[0] += use ? wj * __uint_as_float(u << 16) : 0.f;
-          acc[1] += use ? wj * __uint_as_float(u & 0xffff0000u) : 0.f;
+      // multiply, so whatever its memory holds cannot leak into the sum.  Eight
+      // slots per round keep several loads in flight per lane.
+      const int cnt = min(32, a.topk - s0);
+      for (int j0 = 0; j0 < cnt; j0 += 8) {
+        uint2 u[8];
+        float wj[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int jj = min(j0 + j, cnt - 1);
+          wj[j] = __shfl_sync(0xffffffffu, wgt, jj);
+          if (j0 + j >= cnt) wj[j] = 0.f;
+          const uint16_t* src = a.part_o + ((p0 + s0 + jj) * a.G + hi) * D + lane * PER;
+          if constexpr (PER == 4) {
+            u[j] = __ldg(reinterpret_cast<const uint2*>(src));
+          } else {
+            u[j] = make_uint2(__ldg(reinterpret_cast<const uint32_t*>(src)), 0u);
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const bool use = wj[j] != 0.f;
+          acc[0] += use ? wj[j] * __uint_as_float(u[j].x << 16) : 0.f;
+          acc[1] += use ? wj[j] * __uint_as_float(u[j].x & 0xffff0000u) : 0.f;
+          if constexpr (PER == 4) {
+            acc[2] += use ? wj[j] * __uint_as_float(u[j].y << 16) : 0.f;
+            acc[3] += use ? wj[j] * __uint_as_float(u[j].y & 0xffff0000u) : 0.f;
+          }
         }
       }
     }
@@ -675,7 +695,7 @@ KvPlan plan_kv(const Shape& s) {
 template <int D, int BLK>
 cudaError_t run_kv(const Shape& s, KvArgs& a, const KvPlan& p, const CUtensorMap& tmk,
                    const CUtensorMap& tmv, uint8_t* ws, cudaStream_t stream) {
-  constexpr uint32_t smem = 1024 + 2 * (kRows * (D > BLK ? D : BLK) * 2) + 2 * (4 * D * BLK) + 256;
+  constexpr uint32_t smem = KvSmem<D, BLK>::BYTES;
   cudaError_t err = cudaFuncSetAttribute(kv_attn_kernel<D, BLK>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (err != cudaSuccess) return err;
