@@ -204,6 +204,29 @@ __device__ __forceinline__ float exp2_approx(float x) {
   return r;
 }
 
+// 2^x for x <= 0 on the FMA and integer pipes, leaving the special-function unit
+// free: x = n + f with n = round(x) and f in [-1/2, 1/2]; 2^f from a cubic fitted
+// to it on that interval by iterated weighted least squares on the relative
+// error (largest relative error 7.5e-5 evaluated in float), and 2^n added to the
+// exponent field.  Inputs below -125 are clamped there (2^-125 instead of a
+// smaller positive number).  Adding 1.5 * 2^23 rounds x to an integer held in
+// the low mantissa bits, which the shift by 23 moves into the exponent field.
+__device__ __forceinline__ float exp2_poly(float x) {
+  x = fmaxf(x, -125.f);
+  const float t = __fadd_rn(x, 12582912.f);
+  const float f = __fsub_rn(x, __fsub_rn(t, 12582912.f));
+  const float p = fmaf(fmaf(fmaf(0.0551716685f, f, 0.2426111400f), f, 0.6932609677f), f,
+                       0.9999280572f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+// Two floats to bf16x2 (lo in the low half) on the integer pipe: half a bf16 unit
+// in the last place is added to the magnitude and the high halves are kept, i.e.
+// rounding to nearest with ties away from zero.  Finite inputs only.
+__device__ __forceinline__ uint32_t pack_bf16_int(float lo, float hi) {
+  return __byte_perm(__float_as_uint(lo) + 0x8000u, __float_as_uint(hi) + 0x8000u, 0x7632);
+}
+
 __device__ __forceinline__ float warp_max_xor(float v, int mask) {
   return fmaxf(v, __shfl_xor_sync(0xffffffffu, v, mask));
 }

@@ -48,7 +48,8 @@ cudaError_t launch_sparse_attn(const Shape& s, const uint16_t* q, const uint16_t
 bool kv_attn_supported(const Shape& s);
 size_t kv_workspace_bytes(const Shape& s);
 int kv_launches(const Shape& s);
-cudaError_t launch_kv_attn(const Shape& s, const CUtensorMap& tmk, const CUtensorMap& tmv,
+cudaError_t launch_kv_attn(const Shape& s, const CUtensorMap& tmq, const CUtensorMap& tmk,
+                           const CUtensorMap& tmv,
                            const uint16_t* q, const int32_t* ids, uint16_t* out, float* lse,
                            void* ws, size_t ws_bytes, DeviceStatus* st, cudaStream_t stream);
 

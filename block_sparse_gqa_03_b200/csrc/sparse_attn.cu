@@ -587,6 +587,22 @@ bool make_kv_map(CUtensorMap* map, const uint16_t* base, const Shape& s, const i
          CUDA_SUCCESS;
 }
 
+// Q as a 4-D tensor [batch][token][head][dim]; one box is 64 dims x the G heads
+// of a group x 1 token, i.e. G rows of 128 bytes (128-byte swizzle).
+bool make_q_group_map(CUtensorMap* map, const uint16_t* base, const Shape& s) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[4] = {(cuuint64_t)s.d, (cuuint64_t)s.H, (cuuint64_t)s.n_q, (cuuint64_t)s.batch};
+  cuuint64_t strides[3] = {(cuuint64_t)s.q_s[2] * 2, (cuuint64_t)s.q_s[1] * 2,
+                           (cuuint64_t)s.q_s[0] * 2};
+  cuuint32_t box[4] = {64, (cuuint32_t)s.G, 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<uint16_t*>(base), dims,
+             strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
 constexpr int kStreamNC = 4;       // consumer warps of the streaming kernel
 constexpr int kMaxList = 4096;     // entries a streaming CTA compacts up front
 constexpr uint32_t kSmemCap = 227u * 1024u;
@@ -706,8 +722,11 @@ cudaError_t launch_sparse_attn(const Shape& s, const uint16_t* q, const uint16_t
   a.st = st;
   a.wait_ns = 4000000000ull;  // 4 s: far above any healthy wait, even under a profiler
   cudaError_t err;
-  if (!pl.stream && kv_attn_supported(s))
-    return launch_kv_attn(s, tmk, tmv, q, ids, out, lse, partials, partial_bytes, st, stream);
+  if (!pl.stream && kv_attn_supported(s)) {
+    CUtensorMap tmq;
+    if (!make_q_group_map(&tmq, q, s)) return cudaErrorInvalidValue;
+    return launch_kv_attn(s, tmq, tmk, tmv, q, ids, out, lse, partials, partial_bytes, st, stream);
+  }
   if (!pl.stream) {
     const dim3 grid((unsigned)pl.ctas);
     if (s.d == 128) {

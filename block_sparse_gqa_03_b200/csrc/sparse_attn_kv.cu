@@ -11,35 +11,43 @@
 // by counting, scanning and scattering), and a CTA loads the block's K and V once
 // and streams tiles of up to 128 (query, head) rows through it:
 //   S = Q_tile K^T      tcgen05 MMA, M = 128 rows, N = block, K = d   (TMEM)
-//   P = softmax(S)      registers, one thread per row, masked to visible keys
-//   O = P V             tcgen05 MMA, M = 128, N = d, K = block       (TMEM)
+//   P = softmax(S)      registers, one thread per row, masked to visible keys,
+//                       written back to tensor memory over S as bf16
+//   O = P V             tcgen05 MMA with A = P from tensor memory, N = d (TMEM)
 // Each (query, head, block) gives a normalised bf16 partial output and its
 // log-sum-exp; a combine kernel merges a query's partials by log-sum-exp weights.
 // Queries are processed in chunks so that the partials of one chunk fit a bounded
 // workspace.
 //
-// CTA roles (persistent CTAs, each a contiguous share of the chunk's tiles):
-//   warp 0      TMA producer of K and V (a new load only when the block changes);
-//   warp 1      tensor-memory allocation and the thread issuing the S = Q K^T MMAs;
-//   warps 2-5   gather the tile's Q rows with 16-byte async copies (swizzled), one
-//               thread per row;
-//   warps 6-17  three softmax warp groups taking tiles in turn, one thread per tile
-//               row: softmax from tensor memory, the P tile into shared memory, then
-//               (one elected thread) the O = P V MMA, then the output epilogue.
-// Buffers: 3-4 Q/P tiles (P overwrites its Q once S is computed), 2 K/V stages
-// (each released by every warp group once its products are done), and 4 tile
-// buffers in tensor memory where O = P V overwrites the S it was computed from.
-// Every wait is bounded.
+// CTA roles (persistent CTAs, each a contiguous share of the chunk's tiles), four
+// warpgroups with registers moved from the first and last to the softmax ones:
+//   warp 0        TMA producer of K and V (a new load only when the block changes;
+//                 V rows past the sequence end are zeroed after the load lands);
+//   warp 1        tensor-memory allocation and the thread issuing all MMAs: S of
+//                 tile i, then O of tile i - 1, so the next scores are computed
+//                 while a softmax runs;
+//   warps 2-3     gather the tile's Q rows with TMA, one load per (query, 64-dim
+//                 atom) bringing the query's G heads into the swizzled layout;
+//   warps 4-11    two softmax warpgroups taking tiles in turn, one thread per tile
+//                 row, each owning one S/P buffer in tensor memory;
+//   warps 12-15   output warpgroup: O / l from tensor memory to the partials.
+// Buffers: 2-4 Q tiles (released when S is computed), 2 K/V stages, and in tensor
+// memory two S/P buffers and two O buffers.  Every wait is bounded.
 #include "kernels.h"
 #include "sm100.cuh"
 
 namespace msa {
 namespace {
 
-constexpr int kRows = 128;                  // MMA M: (query, head) rows per tile
-constexpr int kNw = 3;                     // softmax warp groups
-constexpr int kKvThreads = (6 + 4 * kNw) * 32;
-constexpr int kWarpProd = 0, kWarpMma = 1, kWarpGather0 = 2, kWarpSoft0 = 6;
+constexpr int kRows = 128;  // MMA M: (query, head) rows per tile
+constexpr int kKvThreads = 512;
+constexpr int kWarpProd = 0, kWarpMma = 1, kWarpGather = 2;
+// Registers per thread after reallocation.  The four warpgroups' shares add up to
+// what the kernel is launched with (128 per thread; the host refuses to launch a
+// build that was given another count, since the softmax warpgroups would then
+// wait for registers that are never released).
+constexpr int kRegsLaunch = 128, kRegsLoad = 48, kRegsSoft = 184, kRegsOut = 96;
+static_assert(kRegsLoad + 2 * kRegsSoft + kRegsOut == 4 * kRegsLaunch, "register split");
 
 struct KvArgs {
   // problem
@@ -56,12 +64,14 @@ struct KvArgs {
   int* counts;             // [batch * h * nblk]
   int* offs;               // [batch * h * nblk + 1] entry offsets
   int* toffs;              // [batch * h * nblk + 1] tile offsets
-  int* entries;            // chunk-relative slot positions, grouped by (b, g, block)
+  int* entries;            // query index t of each entry, grouped by (b, g, block)
+  int* slot_row;           // [slot] partial row of a valid slot's query (head 0) in its tile
   int qpt;                 // queries per tile
   int nj;                  // batch * h * nblk
-  // partials (chunk-relative position p = (bt_rel * h + g) * topk + slot)
-  uint16_t* part_o;        // [p][G][d] bf16
-  float* part_lse;         // [p][G]
+  // partials: 128 rows per tile, row = tile * 128 + query-in-tile * G + head, so
+  // that a tile's output is one contiguous block
+  uint16_t* part_o;        // [row][d] bf16
+  float* part_lse;         // [row]
   uint16_t* out;
   int64_t o_s0, o_s1, o_s2;
   float* lse;
@@ -69,21 +79,24 @@ struct KvArgs {
   uint64_t wait_ns;
 };
 
-__device__ __forceinline__ int visible_limit(const KvArgs& a, int b, int t) {
-  const int L = kv_length(a.seq_lens, b, a.max_kv, a.st);
+__device__ __forceinline__ int visible_from_length(const KvArgs& a, int L, int t) {
   const int p = L - a.n_q + t;
   return max(0, a.causal ? min(L, p + 1) : L);
 }
 
+__device__ __forceinline__ int visible_limit(const KvArgs& a, int b, int t) {
+  return visible_from_length(a, kv_length(a.seq_lens, b, a.max_kv, a.st), t);
+}
+
 // Valid slot of the chunk: a block id that exists and holds a visible token.
-__device__ __forceinline__ bool slot_block(const KvArgs& a, int64_t pos, int& b, int& g,
+__device__ __forceinline__ bool slot_block(const KvArgs& a, int64_t pos, int& b, int& g, int& t,
                                            int& beta, int BLK) {
   const int64_t bt_rel = pos / ((int64_t)a.h * a.topk);
   const int rem = (int)(pos % ((int64_t)a.h * a.topk));
   g = rem / a.topk;
   const int64_t bt = a.bt0 + bt_rel;
   b = (int)(bt / a.n_q);
-  const int t = (int)(bt % a.n_q);
+  t = (int)(bt % a.n_q);
   beta = a.ids[(bt * a.h + g) * a.topk + rem % a.topk];
   if (beta < 0) return false;
   if (beta >= a.nblk) {
@@ -98,8 +111,8 @@ __global__ void kv_count_kernel(KvArgs a, int BLK) {
   const int64_t n = (int64_t)a.nbt * a.h * a.topk;
   for (int64_t pos = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; pos < n;
        pos += (int64_t)gridDim.x * blockDim.x) {
-    int b, g, beta;
-    if (slot_block(a, pos, b, g, beta, BLK))
+    int b, g, t, beta;
+    if (slot_block(a, pos, b, g, t, beta, BLK))
       atomicAdd(&a.counts[((int64_t)b * a.h + g) * a.nblk + beta], 1);
   }
 }
@@ -162,20 +175,29 @@ __global__ void kv_scatter_kernel(KvArgs a, int BLK) {
   const int64_t n = (int64_t)a.nbt * a.h * a.topk;
   for (int64_t pos = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; pos < n;
        pos += (int64_t)gridDim.x * blockDim.x) {
-    int b, g, beta;
-    if (slot_block(a, pos, b, g, beta, BLK)) {
+    int b, g, t, beta;
+    if (slot_block(a, pos, b, g, t, beta, BLK)) {
       const int64_t j = ((int64_t)b * a.h + g) * a.nblk + beta;
       const int k = atomicAdd(&a.counts[j], 1);
-      a.entries[a.offs[j] + k] = (int)pos;
+      a.entries[a.offs[j] + k] = t;
+      a.slot_row[pos] = (a.toffs[j] + k / a.qpt) * kRows + (k % a.qpt) * a.G;
     }
   }
 }
 
 // ------------------------------------------------------------ tile walker
-// Tiles are numbered through the (b, g, block) lists in order; a walker moves
-// forward through them, amortising the lookup of the list a tile belongs to.
-struct TileWalker {
-  int j;
+// Tiles are numbered through the (b, g, block) lists in order.  A walker moves
+// forward through them and steps the list's (b, g, block) along, so that only
+// the initial seek divides.
+struct Walker {
+  int j, b, g, beta;  // current list
+  int t0, t1;         // its tiles [t0, t1)
+  int e0, cnt;        // its entries [e0, e0 + cnt)
+
+  __device__ __forceinline__ void load_list(const KvArgs& a) {
+    e0 = __ldg(a.offs + j);
+    cnt = __ldg(a.offs + j + 1) - e0;
+  }
   __device__ __forceinline__ void seek(const KvArgs& a, int tile) {
     int lo = 0, hi = a.nj;  // toffs[lo] <= tile < toffs[hi]
     while (hi - lo > 1) {
@@ -183,93 +205,114 @@ struct TileWalker {
       if (__ldg(a.toffs + mid) <= tile) lo = mid; else hi = mid;
     }
     j = lo;
+    beta = j % a.nblk;
+    const int bg = j / a.nblk;
+    g = bg % a.h;
+    b = bg / a.h;
+    t0 = __ldg(a.toffs + j);
+    t1 = __ldg(a.toffs + j + 1);
+    load_list(a);
   }
-  __device__ __forceinline__ void advance(const KvArgs& a, int tile) {
-    while (__ldg(a.toffs + j + 1) <= tile) ++j;
+  // Moves to the list holding `tile` (visited in increasing order); true when
+  // the list changed.
+  __device__ __forceinline__ bool advance(const KvArgs& a, int tile) {
+    if (tile < t1) return false;
+    do {
+      ++j;
+      if (++beta == a.nblk) {
+        beta = 0;
+        if (++g == a.h) {
+          g = 0;
+          ++b;
+        }
+      }
+      t0 = t1;
+      t1 = __ldg(a.toffs + j + 1);
+    } while (tile >= t1);
+    load_list(a);
+    return true;
+  }
+  __device__ __forceinline__ int first(const KvArgs& a, int tile) const {
+    return e0 + (tile - t0) * a.qpt;
+  }
+  __device__ __forceinline__ int count(const KvArgs& a, int tile) const {
+    return min(a.qpt, cnt - (tile - t0) * a.qpt);
   }
 };
-
-struct TileInfo {
-  int j, b, g, beta, first, nq;  // entries [first, first + nq)
-};
-
-__device__ __forceinline__ TileInfo tile_info(const KvArgs& a, int j, int tile) {
-  TileInfo ti;
-  ti.j = j;
-  ti.beta = j % a.nblk;
-  const int bg = j / a.nblk;
-  ti.g = bg % a.h;
-  ti.b = bg / a.h;
-  const int u = tile - __ldg(a.toffs + j);
-  const int cnt = __ldg(a.offs + j + 1) - __ldg(a.offs + j);
-  ti.first = __ldg(a.offs + j) + u * a.qpt;
-  ti.nq = min(a.qpt, cnt - u * a.qpt);
-  return ti;
-}
 
 // --------------------------------------------------------- attention tiles
 // Shared-memory plan of the attention kernel for one (D, BLK).
 template <int D, int BLK>
 struct KvSmem {
-  static constexpr uint32_t QP = kRows * (D > BLK ? D : BLK) * 2;  // a Q tile or a P tile
-  static constexpr uint32_t HALF = BLK * 128u;                     // one 64-dim atom of K or V
-  static constexpr uint32_t KV = 2 * (D / 64) * HALF;              // K and V of one block
-  static constexpr int NQ = (4 * QP + 2 * KV + 2048 <= 227u * 1024u) ? 4 : 3;
-  static constexpr uint32_t BYTES = 1024 + NQ * QP + 2 * KV + 512;
+  static constexpr uint32_t Q = kRows * D * 2;         // one Q tile
+  static constexpr uint32_t HALF = BLK * 128u;         // one 64-dim atom of K or V
+  static constexpr uint32_t KV = 2 * (D / 64) * HALF;  // K and V of one block
+  // row statistics [4][128] float2, row table [128] int, barriers, TMEM address
+  static constexpr uint32_t MISC = 5120;
+  static constexpr uint32_t LIMIT = 227u * 1024u;
+  static constexpr int NQ = 1024 + 4 * Q + 2 * KV + MISC <= LIMIT   ? 4
+                            : 1024 + 3 * Q + 2 * KV + MISC <= LIMIT ? 3
+                                                                    : 2;
+  static constexpr uint32_t BYTES = 1024 + NQ * Q + 2 * KV + MISC;
+  static_assert(BYTES <= LIMIT, "shared memory");
 };
 
 template <int D, int BLK>
 __global__ void __launch_bounds__(kKvThreads, 1)
-    kv_attn_kernel(const __grid_constant__ CUtensorMap tmk,
+    kv_attn_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                    const __grid_constant__ CUtensorMap tmv, KvArgs a) {
   using SM = KvSmem<D, BLK>;
   constexpr int NH = D / 64;
-  constexpr int NQ = SM::NQ;                  // Q/P tile buffers
-  constexpr int NB = 4;                       // tensor-memory tile buffers
-  constexpr uint32_t TB = D > BLK ? D : BLK;  // columns per buffer: S, then O in place
-  constexpr uint32_t QP_BYTES = SM::QP, HALF = SM::HALF, KV_BYTES = SM::KV;
-  constexpr uint32_t TMEM_COLS = NB * TB <= 256 ? 256 : 512;
-  static_assert(NB * TB <= 512, "tensor memory");
+  constexpr int NQ = SM::NQ;
+  constexpr uint32_t QB = SM::Q, HALF = SM::HALF, KV_BYTES = SM::KV;
+  constexpr uint32_t TMEM_COLS = 2 * (BLK + D) <= 256 ? 256 : 512;
+  constexpr uint32_t O_COL = 2 * BLK;  // two S/P buffers, then two O buffers
+  static_assert(2 * (BLK + D) <= 512, "tensor memory");
   if (status_failed(a.st)) return;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  const uint32_t sm0a = smem_u32(smem);
-  const uint32_t sqp = sm0a;                     // NQ x QP_BYTES
-  const uint32_t skv = sqp + NQ * QP_BYTES;      // 2 x KV_BYTES
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + NQ * QP_BYTES + 2 * KV_BYTES);
-  // barrier blocks (8 bytes each)
-  const uint32_t b_kvfull = smem_u32(bars);                 // [2]
-  const uint32_t b_kvempty = b_kvfull + 16;                 // [2][kNw]
-  const uint32_t b_qfull = b_kvempty + 16 * kNw;            // [NQ]
-  const uint32_t b_qempty = b_qfull + 8 * NQ;               // [NQ]
-  const uint32_t b_sfull = b_qempty + 8 * NQ;               // [NB]
-  const uint32_t b_ofull = b_sfull + 8 * NB;                // [NB]
-  const uint32_t b_ofree = b_ofull + 8 * NB;                // [NB]
-  const uint32_t b_done = b_ofree + 8 * NB;                 // [1 + kNw]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + NQ * QP_BYTES + 2 * KV_BYTES + 480);
+  const uint32_t sq = smem_u32(smem);         // NQ Q tiles
+  const uint32_t skv = sq + NQ * QB;          // 2 K/V stages
+  uint8_t* misc = smem + NQ * QB + 2 * KV_BYTES;
+  float2* rstat = reinterpret_cast<float2*>(misc);      // [4][128]: 1 / l, log-sum-exp
+  int* rowtab = reinterpret_cast<int*>(misc + 4096);    // [128]: query | head << 16
+  const uint32_t b_kvfull = smem_u32(misc + 4608);      // [2] K/V usable
+  const uint32_t b_kvland = b_kvfull + 16;              // [2] K/V landed (before fix-up)
+  const uint32_t b_kvempty = b_kvland + 16;             // [2]
+  const uint32_t b_qfull = b_kvempty + 16;              // [NQ]
+  const uint32_t b_qempty = b_qfull + 8 * NQ;           // [NQ]
+  const uint32_t b_sfull = b_qempty + 8 * NQ;           // [2]
+  const uint32_t b_pfull = b_sfull + 16;                // [2]
+  const uint32_t b_ofull = b_pfull + 16;                // [2]
+  const uint32_t b_ofree = b_ofull + 16;                // [2]
+  const uint32_t b_lfull = b_ofree + 16;                // [4]
+  const uint32_t b_done = b_lfull + 32;                 // [1]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + 4864);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ntiles = __ldg(a.toffs + a.nj);
   const int per = (ntiles + gridDim.x - 1) / gridDim.x;
   const int tile0 = blockIdx.x * per;
-  const int tile1 = min(ntiles, tile0 + per);
+  const int n = max(0, min(ntiles, tile0 + per) - tile0);
 
+  if (threadIdx.x < kRows) rowtab[threadIdx.x] = (threadIdx.x / a.G) | ((threadIdx.x % a.G) << 16);
   if (threadIdx.x == 0) {
     for (int s = 0; s < 2; ++s) {
       mbar_init(b_kvfull + 8 * s, 1);
-      for (int w = 0; w < kNw; ++w) mbar_init(b_kvempty + 8 * (s * kNw + w), 1);
+      mbar_init(b_kvland + 8 * s, 1);
+      mbar_init(b_kvempty + 8 * s, 1);
+      mbar_init(b_sfull + 8 * s, 1);
+      mbar_init(b_pfull + 8 * s, 4);
+      mbar_init(b_ofull + 8 * s, 1);
+      mbar_init(b_ofree + 8 * s, 4);
     }
     for (int i = 0; i < NQ; ++i) {
-      mbar_init(b_qfull + 8 * i, 128);
+      mbar_init(b_qfull + 8 * i, 2);
       mbar_init(b_qempty + 8 * i, 1);
     }
-    for (int i = 0; i < NB; ++i) {
-      mbar_init(b_sfull + 8 * i, 1);
-      mbar_init(b_ofull + 8 * i, 1);
-      mbar_init(b_ofree + 8 * i, 4);
-    }
-    for (int i = 0; i <= kNw; ++i) mbar_init(b_done + 8 * i, 1);
+    for (int i = 0; i < 4; ++i) mbar_init(b_lfull + 8 * i, 4);
+    mbar_init(b_done, 1);
     fence_mbar_init();
   }
   if (warp == kWarpMma) {
@@ -280,274 +323,300 @@ __global__ void __launch_bounds__(kKvThreads, 1)
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
-
-  if (tile0 < tile1) {
-    TileWalker w;
-    w.seek(a, tile0);
-    if (warp == kWarpProd) {
-      // ------------------------------------------------------ K/V producer
+  // Each role sets its register limit first thing in its own branch, so that the
+  // code under each limit is exactly that branch.
+  const int wg = warp >> 2;
+  Walker w;
+  if (warp == kWarpProd) {
+    // ---------------------------------------------------------- K/V producer
+    tc::regs_dec<kRegsLoad>();
+    if (n > 0) {
+      w.seek(a, tile0);
       if (lane == 0) {
         prefetch_tensormap(&tmk);
         prefetch_tensormap(&tmv);
-        int use = -1, prev_j = -1, issued = 0;
-        bool ok = true;
-        for (int tile = tile0; tile < tile1 && ok; ++tile) {
-          w.advance(a, tile);
-          if (w.j == prev_j) continue;
-          prev_j = w.j;
-          ++use;
-          const int s = use & 1;
-          if (use >= 2)
-            for (int g = 0; g < kNw && ok; ++g)
-              ok = mbar_wait_bounded(b_kvempty + 8 * (s * kNw + g), ((use >> 1) - 1) & 1, a.st,
-                                     0x201u, a.wait_ns);
-          if (!ok) break;
-          const TileInfo ti = tile_info(a, w.j, tile);
-          mbar_arrive_expect_tx(b_kvfull + 8 * s, KV_BYTES);
-          const uint32_t kd = skv + s * KV_BYTES, vd = kd + NH * HALF;
+      }
+      int use = -1;
+      uint32_t land_par = 0;  // bit s: parity of the next wait on kv_land[s]
+      bool ok = true;
+      for (int idx = 0; idx < n && ok; ++idx) {
+        const int tile = tile0 + idx;
+        if (!w.advance(a, tile) && idx > 0) continue;
+        ++use;
+        const int s = use & 1;
+        if (use >= 2)
+          ok = mbar_wait_warp(b_kvempty + 8 * s, ((use >> 1) - 1) & 1, a.st, 0x201u, a.wait_ns);
+        if (!ok) break;
+        // V rows [r0, BLK) lie past the sequence end and may hold anything: they
+        // are zeroed once the block has landed, so that a zero probability never
+        // meets a non-finite value.
+        const int L = kv_length(a.seq_lens, w.b, a.max_kv, a.st);
+        const int r0 = max(0, L - w.beta * BLK);
+        const bool fix = r0 < BLK;
+        const uint32_t bar = (fix ? b_kvland : b_kvfull) + 8 * s;
+        const uint32_t kd = skv + s * KV_BYTES, vd = kd + NH * HALF;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(bar, KV_BYTES);
 #pragma unroll
           for (int hh = 0; hh < NH; ++hh) {
-            tma_load_4d(kd + hh * HALF, &tmk, b_kvfull + 8 * s, hh * 64, ti.g, ti.beta * BLK, ti.b);
-            tma_load_4d(vd + hh * HALF, &tmv, b_kvfull + 8 * s, hh * 64, ti.g, ti.beta * BLK, ti.b);
-          }
-          issued = use + 1;
-        }
-        // drain: the stages of the last two blocks are released once every
-        // warp group's O = P V products that read them have completed
-        for (int u = max(0, issued - 2); u < issued; ++u)
-          for (int g = 0; g < kNw; ++g)
-            mbar_wait_bounded(b_kvempty + 8 * ((u & 1) * kNw + g), (u >> 1) & 1, a.st, 0x202u,
-                              a.wait_ns);
-      }
-    } else if (warp == kWarpMma) {
-      // ------------------------------------------------------ S = Q K^T issue
-      if (lane == 0) {
-        const uint32_t id_qk = tc::idesc_bf16(kRows, BLK, false);
-        int use = -1, prev_j = -1, i = 0;
-        bool ok = true;
-        for (int tile = tile0; tile < tile1 && ok; ++tile, ++i) {
-          w.advance(a, tile);
-          if (w.j != prev_j) {
-            prev_j = w.j;
-            ++use;
-            ok = mbar_wait_bounded(b_kvfull + 8 * (use & 1), (use >> 1) & 1, a.st, 0x203u,
-                                   a.wait_ns);
-          }
-          const int qb = i % NQ, tb = i % NB;
-          if (ok) ok = mbar_wait_bounded(b_qfull + 8 * qb, (i / NQ) & 1, a.st, 0x204u, a.wait_ns);
-          if (ok && i >= NB)
-            ok = mbar_wait_bounded(b_ofree + 8 * tb, ((i / NB) - 1) & 1, a.st, 0x205u, a.wait_ns);
-          if (!ok) break;
-          tc::fence_after_sync();
-          const uint32_t kd = skv + (use & 1) * KV_BYTES;
-#pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks) {
-            const uint32_t koff = (ks >> 2) * (kRows * 128u) + (ks & 3) * 32;
-            const uint32_t kboff = (ks >> 2) * HALF + (ks & 3) * 32;
-            tc::mma_bf16(tmem + tb * TB, tc::desc_k_sw128(sqp + qb * QP_BYTES + koff),
-                         tc::desc_k_sw128(kd + kboff), id_qk, ks > 0 ? 1u : 0u);
-          }
-          tc::commit(b_sfull + 8 * tb);
-        }
-        tc::commit(b_done);
-        mbar_wait_bounded(b_done, 0, a.st, 0x208u, a.wait_ns);
-      }
-    } else if (warp < kWarpSoft0) {
-      // ----------------------------------------------------- Q gather warps
-      const int row = threadIdx.x - kWarpGather0 * 32;  // 0..127: one tile row each
-      int i = 0;
-      bool ok = true;
-      constexpr int CPR = D / 8;  // 16-byte chunks per row
-      for (int tile = tile0; tile < tile1; ++tile, ++i) {
-        w.advance(a, tile);
-        const int qb = i % NQ;
-        if (i >= NQ && ok)
-          ok = mbar_wait_bounded(b_qempty + 8 * qb, ((i / NQ) - 1) & 1, a.st, 0x209u, a.wait_ns);
-        const TileInfo ti = tile_info(a, w.j, tile);
-        if (ok && row < ti.nq * a.G) {
-          const int qi = row / a.G, hi = row - qi * a.G;
-          const int pos = __ldg(a.entries + ti.first + qi);  // chunk-relative slot position
-          const int bt = (int)a.bt0 + pos / (a.h * a.topk);
-          const uint16_t* src = a.q + (int64_t)ti.b * a.q_s0 + (int64_t)(bt % a.n_q) * a.q_s1 +
-                                (int64_t)(ti.g * a.G + hi) * a.q_s2;
-          const uint32_t dst0 = sqp + qb * QP_BYTES + row * 128u;
-#pragma unroll
-          for (int ch = 0; ch < CPR; ++ch) {
-            const uint32_t dst = dst0 + (ch >> 3) * (kRows * 128u) + (((ch & 7) ^ (row & 7)) << 4);
-            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src + ch * 8));
+            tma_load_4d(kd + hh * HALF, &tmk, bar, hh * 64, w.g, w.beta * BLK, w.b);
+            tma_load_4d(vd + hh * HALF, &tmv, bar, hh * 64, w.g, w.beta * BLK, w.b);
           }
         }
-        asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
-        fence_proxy_async_smem();
-        mbar_arrive(b_qfull + 8 * qb);
-      }
-    } else {
-      // ------------------------- softmax, O = P V issue and epilogue (warp groups)
-      const int wg = (warp - kWarpSoft0) >> 2;  // takes tiles with i % kNw == wg
-      const int quarter = warp & 3;
-      const int row = quarter * 32 + lane;
-      const bool leader = ((warp - kWarpSoft0) & 3) == 0 && lane == 0;
-      const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
-      const float ninf = -__int_as_float(0x7f800000);
-      const float kLn2 = 0.69314718055994531f;
-      const uint32_t id_pv = tc::idesc_bf16(kRows, D, true);
-      bool ok = true;
-      int i = 0, use = -1, prev_j = -1;
-      for (int tile = tile0; tile < tile1; ++tile, ++i) {
-        w.advance(a, tile);
-        if (w.j != prev_j) {
-          // Leaving block `use`: this group's O = P V products that read it have
-          // all been issued; release its K/V stage once they complete.  The release
-          // waits until the producer has loaded that block, so that a group owning
-          // no tile of several short blocks never runs two phases ahead of the
-          // producer on the stage's barrier.
-          if (use >= 0 && leader) {
-            mbar_wait_bounded(b_kvfull + 8 * (use & 1), (use >> 1) & 1, a.st, 0x20du, a.wait_ns);
-            tc::commit(b_kvempty + 8 * ((use & 1) * kNw + wg));
-          }
-          prev_j = w.j;
-          ++use;
-        }
-        if (i % kNw != wg) continue;
-        const int qb = i % NQ, tb = i % NB;
-        const TileInfo ti = tile_info(a, w.j, tile);
-        const bool live = row < ti.nq * a.G;
-        int pos = -1, hi = 0, lim = 0;
-        if (live) {
-          const int qi = row / a.G;
-          hi = row - qi * a.G;
-          pos = __ldg(a.entries + ti.first + qi);
-          const int bt = (int)a.bt0 + pos / (a.h * a.topk);
-          lim = visible_limit(a, ti.b, bt % a.n_q);
-        }
-        if (ok) ok = mbar_wait_warp(b_sfull + 8 * tb, (i / NB) & 1, a.st, 0x20bu, a.wait_ns);
-        tc::fence_after_sync();
-        // Scores from tensor memory in 32-column pieces: the row maximum first,
-        // then probabilities, their sum and the bf16 P row (K-major, swizzled).
-        const int vis = lim - ti.beta * BLK;  // keys [0, vis) of the block are visible
-        const bool full = vis >= BLK;
-        const uint32_t srow = lane_base + tb * TB;
-        float mx = ninf;
-#pragma unroll
-        for (int c = 0; c < BLK / 32; ++c) {
-          float v[32];
-          tc::tmem_ld32(srow + c * 32, v);
-          tc::tmem_wait_ld();
-          if (!full) {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] = c * 32 + e < vis ? v[e] : ninf;
-          }
-          float m2[2] = {ninf, ninf};
-#pragma unroll
-          for (int e = 0; e < 32; e += 4) {
-            m2[0] = fmax3(m2[0], v[e], v[e + 1]);
-            m2[1] = fmax3(m2[1], v[e + 2], v[e + 3]);
-          }
-          mx = fmax3(mx, m2[0], m2[1]);
-        }
-        mx *= a.scale_log2;
-        const float msafe = live && mx != ninf ? mx : 0.f;
-        float l = 0.f;
-        uint8_t* pbase = smem + qb * QP_BYTES;
-#pragma unroll
-        for (int c = 0; c < BLK / 32; ++c) {
-          float v[32];
-          tc::tmem_ld32(srow + c * 32, v);
-          tc::tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) v[e] = exp2_approx(fmaf(v[e], a.scale_log2, -msafe));
-          if (!full) {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] = c * 32 + e < vis ? v[e] : 0.f;
-          }
-          float l2[2] = {0.f, 0.f};
-#pragma unroll
-          for (int e = 0; e < 32; ++e) l2[e & 1] += v[e];
-          l += l2[0] + l2[1];
-#pragma unroll
-          for (int q8 = 0; q8 < 4; ++q8) {
-            const int ch = c * 4 + q8;  // 16-byte chunk of the P row
-            const uint4 v4 = make_uint4(pack_bf16(v[8 * q8], v[8 * q8 + 1]),
-                                        pack_bf16(v[8 * q8 + 2], v[8 * q8 + 3]),
-                                        pack_bf16(v[8 * q8 + 4], v[8 * q8 + 5]),
-                                        pack_bf16(v[8 * q8 + 6], v[8 * q8 + 7]));
-            *reinterpret_cast<uint4*>(pbase + (ch >> 3) * (kRows * 128u) + swz128(row, ch & 7)) =
-                v4;
-          }
-        }
-        // V rows at or past the sequence end may hold anything; zero them so that a
-        // zero probability never meets a non-finite value (idempotent per stage).
-        {
-          const int L = kv_length(a.seq_lens, ti.b, a.max_kv, a.st);
-          const int r0 = max(0, L - ti.beta * BLK);
-          if (r0 < BLK) {
-            const int per_h = (BLK - r0) * 8;
-            uint8_t* vb = smem + (skv - sm0a) + (use & 1) * KV_BYTES + NH * HALF;
-            for (int x = row; x < per_h * NH; x += 128) {
-              const int hh = x / per_h, rem = x % per_h;
+        if (fix) {
+          ok = mbar_wait_warp(b_kvland + 8 * s, (land_par >> s) & 1u, a.st, 0x202u, a.wait_ns);
+          land_par ^= 1u << s;
+          if (ok) {
+            const int per_h = (BLK - r0) * 8;  // 16-byte pieces per 64-dim atom
+            uint8_t* vb = smem + (vd - sq);
+            for (int x = lane; x < per_h * NH; x += 32) {
+              const int hh = x / per_h, rem = x - hh * per_h;
               *reinterpret_cast<uint4*>(vb + hh * HALF + (r0 + rem / 8) * 128 + (rem % 8) * 16) =
                   make_uint4(0, 0, 0, 0);
             }
+            fence_proxy_async_smem();
           }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(b_kvfull + 8 * s);
         }
-        // The P tile is complete once every warp of the group has written its rows.
-        fence_proxy_async_smem();
-        tc::fence_before_sync();
-        asm volatile("bar.sync %0, 128;" ::"r"(3 + wg) : "memory");
-        if (leader && ok) {
-          tc::fence_after_sync();
-          const uint32_t vd = skv + (use & 1) * KV_BYTES + NH * HALF;
+      }
+      // drain: the last two stages are released once their products complete
+      for (int u = max(0, use - 1); u <= use; ++u)
+        mbar_wait_warp(b_kvempty + 8 * (u & 1), (u >> 1) & 1, a.st, 0x203u, a.wait_ns);
+    }
+  } else if (warp == kWarpMma) {
+    // ----------------------------------------------- MMA issue (one thread)
+    tc::regs_dec<kRegsLoad>();
+    if (n > 0) {
+      w.seek(a, tile0);
+      if (lane == 0) {
+        const uint32_t id_qk = tc::idesc_bf16(kRows, BLK, false);
+        const uint32_t id_pv = tc::idesc_bf16(kRows, D, true);
+        int use = -1, stage_prev = 0;
+        bool ok = true;
+        for (int idx = 0; idx <= n && ok; ++idx) {
+          bool block_ends = true;  // the previous tile was the last of its block
+          if (idx < n) {
+            // S = Q K^T of tile idx into S/P buffer idx & 1
+            const int tile = tile0 + idx;
+            block_ends = w.advance(a, tile) || idx == 0;
+            if (block_ends) {
+              ++use;
+              ok = mbar_wait_bounded(b_kvfull + 8 * (use & 1), (use >> 1) & 1, a.st, 0x204u,
+                                     a.wait_ns);
+            }
+            const int qb = idx % NQ, s = idx & 1;
+            if (ok) ok = mbar_wait_bounded(b_qfull + 8 * qb, (idx / NQ) & 1, a.st, 0x205u, a.wait_ns);
+            // the buffer's previous P has been consumed by its O = P V
+            if (ok && idx >= 2)
+              ok = mbar_wait_bounded(b_ofull + 8 * s, ((idx - 2) >> 1) & 1, a.st, 0x206u, a.wait_ns);
+            if (!ok) break;
+            tc::fence_after_sync();
+            const uint32_t kd = skv + (use & 1) * KV_BYTES, qd = sq + qb * QB;
 #pragma unroll
-          for (int ks = 0; ks < BLK / 16; ++ks) {
-            const uint32_t poff = (ks >> 2) * (kRows * 128u) + (ks & 3) * 32;
-            tc::mma_bf16(tmem + tb * TB, tc::desc_k_sw128(sqp + qb * QP_BYTES + poff),
-                         tc::desc_mn_sw128(vd + ks * 16 * 128, HALF), id_pv, ks > 0 ? 1u : 0u);
+            for (int ks = 0; ks < D / 16; ++ks) {
+              const uint32_t qoff = (ks >> 2) * (kRows * 128u) + (ks & 3) * 32;
+              const uint32_t koff = (ks >> 2) * HALF + (ks & 3) * 32;
+              tc::mma_bf16(tmem + s * BLK, tc::desc_k_sw128(qd + qoff), tc::desc_k_sw128(kd + koff),
+                           id_qk, ks > 0 ? 1u : 0u);
+            }
+            tc::commit(b_sfull + 8 * s);
+            tc::commit(b_qempty + 8 * qb);  // the Q tile may be refilled
           }
-          tc::commit(b_ofull + 8 * tb);
-          tc::commit(b_qempty + 8 * qb);  // the Q/P buffer may be refilled
+          if (idx >= 1) {
+            // O = P V of tile idx - 1 into O buffer (idx - 1) & 1
+            const int k = idx - 1, s = k & 1;
+            ok = mbar_wait_bounded(b_pfull + 8 * s, (k >> 1) & 1, a.st, 0x207u, a.wait_ns);
+            if (ok && k >= 2)
+              ok = mbar_wait_bounded(b_ofree + 8 * s, ((k >> 1) - 1) & 1, a.st, 0x208u, a.wait_ns);
+            if (!ok) break;
+            tc::fence_after_sync();
+            const uint32_t vd = skv + stage_prev * KV_BYTES + NH * HALF;
+#pragma unroll
+            for (int ks = 0; ks < BLK / 16; ++ks)
+              tc::mma_bf16_ts(tmem + O_COL + s * D, tmem + s * BLK + ks * 8,
+                              tc::desc_mn_sw128(vd + ks * 16 * 128, HALF), id_pv, ks > 0 ? 1u : 0u);
+            tc::commit(b_ofull + 8 * s);
+            if (block_ends) tc::commit(b_kvempty + 8 * stage_prev);  // K/V stage released
+          }
+          stage_prev = use & 1;
         }
-        // Output of this tile: O / l in bf16 and the log-sum-exp, for live rows.
-        const float inv_l = l > 0.f ? 1.f / l : 0.f;
-        if (ok) ok = mbar_wait_warp(b_ofull + 8 * tb, (i / NB) & 1, a.st, 0x20au, a.wait_ns);
+        tc::commit(b_done);
+        mbar_wait_bounded(b_done, 0, a.st, 0x209u, a.wait_ns);
+      }
+    }
+  } else if (warp == kWarpGather || warp == kWarpGather + 1) {
+    // -------------------------------------------------------------- Q gather
+    // One TMA load per (query, 64-dim atom) brings the query's G heads, i.e. G
+    // consecutive tile rows, into the swizzled operand layout.  Two warps share
+    // the loads (one atom each, or alternate queries when d = 64); the query
+    // positions of the next tile are read while the current one is issued.
+    tc::regs_dec<kRegsLoad>();
+    if (n > 0) {
+      w.seek(a, tile0);
+      const int gw = warp - kWarpGather;
+      if (lane == 0) prefetch_tensormap(&tmq);
+      const uint32_t rows_bytes = (uint32_t)a.G * 128u;
+      // query positions of a tile's (at most 128) queries: query 32 k + lane in tq[k]
+      auto load_t = [&](int first, int nq, int (&tq)[4]) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          tq[k] = 32 * k + lane < nq ? __ldg(a.entries + first + 32 * k + lane) : 0;
+      };
+      int first = w.first(a, tile0), nq = w.count(a, tile0), b = w.b, g = w.g;
+      int tq[4];
+      load_t(first, nq, tq);
+      const int hh = NH == 2 ? gw : 0;
+      bool ok = true;
+      for (int idx = 0; idx < n; ++idx) {
+        const int qb = idx % NQ;
+        if (idx >= NQ && ok)
+          ok = mbar_wait_warp(b_qempty + 8 * qb, ((idx / NQ) - 1) & 1, a.st, 0x20au, a.wait_ns);
+        const int mine = !ok ? 0 : NH == 2 ? nq : (nq + 1 - gw) / 2;  // loads of this warp
+        const uint32_t bar = b_qfull + 8 * qb, qd = sq + qb * QB + hh * (kRows * 128u);
+        if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)mine * rows_bytes);
+        __syncwarp();
+        if (ok) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int qi = 32 * k + lane;
+            if (qi < nq && (NH == 2 || (qi & 1) == gw))
+              tma_load_4d(qd + qi * rows_bytes, &tmq, bar, hh * 64, g * a.G, tq[k], b);
+          }
+        }
+        if (idx + 1 < n) {
+          const int tile = tile0 + idx + 1;
+          w.advance(a, tile);
+          first = w.first(a, tile);
+          nq = w.count(a, tile);
+          b = w.b;
+          g = w.g;
+          load_t(first, nq, tq);
+        }
+      }
+    }
+  } else if (wg < 3) {
+    // ------------------------------------------------------ softmax warpgroups
+    tc::regs_inc<kRegsSoft>();
+    if (n > 0) {
+      w.seek(a, tile0);
+      const int sw = wg - 1;  // tiles idx with idx % 2 == sw; S/P buffer sw
+      const int quarter = warp & 3, row = quarter * 32 + lane;
+      const uint32_t sp = tmem + ((uint32_t)(quarter * 32) << 16) + sw * BLK;
+      const int qi = rowtab[row] & 0xffff;
+      const float ninf = -__int_as_float(0x7f800000);
+      const float kLn2 = 0.69314718055994531f;
+      int Lb = -1, L = 0;
+      bool ok = true;
+      for (int idx = sw; idx < n; idx += 2) {
+        const int tile = tile0 + idx;
+        w.advance(a, tile);
+        int vis = BLK;  // keys [0, vis) of the block are visible to this row
+        if (qi < w.count(a, tile)) {
+          const int t = __ldg(a.entries + w.first(a, tile) + qi);
+          if (w.b != Lb) {
+            Lb = w.b;
+            L = kv_length(a.seq_lens, w.b, a.max_kv, a.st);
+          }
+          vis = visible_from_length(a, L, t) - w.beta * BLK;
+        }
+        if (ok) ok = mbar_wait_warp(b_sfull + 8 * sw, (idx >> 1) & 1, a.st, 0x20bu, a.wait_ns);
+        tc::fence_after_sync();
+        float v[BLK];
+#pragma unroll
+        for (int c = 0; c < BLK / 32; ++c) tc::tmem_ld32_at(sp + c * 32, v + c * 32);
+        tc::tmem_wait_ld();
+        if (vis < BLK) {
+#pragma unroll
+          for (int e = 0; e < BLK; ++e) v[e] = e < vis ? v[e] : ninf;
+        }
+        float m4[4] = {ninf, ninf, ninf, ninf};
+#pragma unroll
+        for (int e = 0; e < BLK; e += 8) {
+          m4[0] = fmax3(m4[0], v[e], v[e + 1]);
+          m4[1] = fmax3(m4[1], v[e + 2], v[e + 3]);
+          m4[2] = fmax3(m4[2], v[e + 4], v[e + 5]);
+          m4[3] = fmax3(m4[3], v[e + 6], v[e + 7]);
+        }
+        const float ms = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3])) * a.scale_log2;
+        const float msafe = ms != ninf ? ms : 0.f;
+        // probabilities (masked keys hold -inf and give exactly 0), their sum and
+        // the bf16 P row written over the first half of the row's S columns
+        float l4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int c = 0; c < BLK / 32; ++c) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float p0 = exp2_approx(fmaf(v[c * 32 + 2 * e], a.scale_log2, -msafe));
+            const float p1 = exp2_approx(fmaf(v[c * 32 + 2 * e + 1], a.scale_log2, -msafe));
+            l4[e & 3] += p0 + p1;
+            pk[e] = pack_bf16(p0, p1);
+          }
+          tc::tmem_st16(sp + c * 16, pk);
+        }
+        tc::tmem_wait_st();
+        const float l = (l4[0] + l4[1]) + (l4[2] + l4[3]);
+        rstat[(idx & 3) * kRows + row] =
+            make_float2(l > 0.f ? 1.f / l : 0.f, (ms != ninf && l > 0.f) ? (msafe + log2f(l)) * kLn2 : ninf);
+        tc::fence_before_sync();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(b_pfull + 8 * sw);
+          mbar_arrive(b_lfull + 8 * (idx & 3));
+        }
+      }
+    }
+  } else {
+    // -------------------------------------------------------- output warpgroup
+    tc::regs_dec<kRegsOut>();
+    if (n > 0) {
+      w.seek(a, tile0);
+      const int quarter = warp & 3, row = quarter * 32 + lane;
+      const int qi = rowtab[row] & 0xffff;
+      const uint32_t obase = tmem + ((uint32_t)(quarter * 32) << 16) + O_COL;
+      bool ok = true;
+      for (int idx = 0; idx < n; ++idx) {
+        const int tile = tile0 + idx;
+        w.advance(a, tile);
+        const bool live = qi < w.count(a, tile);
+        if (ok) ok = mbar_wait_warp(b_lfull + 8 * (idx & 3), (idx >> 2) & 1, a.st, 0x20cu, a.wait_ns);
+        const float2 rs = rstat[(idx & 3) * kRows + row];
+        if (ok) ok = mbar_wait_warp(b_ofull + 8 * (idx & 1), (idx >> 1) & 1, a.st, 0x20du, a.wait_ns);
         tc::fence_after_sync();
         const bool store = ok && live;
-        uint16_t* dst = a.part_o + (store ? ((int64_t)pos * a.G + hi) * D : 0);
+        const int64_t prow = (int64_t)tile * kRows + row;  // this thread's partial row
+        uint16_t* dst = a.part_o + (store ? prow * D : 0);
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          float v[32];
-          tc::tmem_ld32(lane_base + tb * TB + c * 32, v);
+        for (int c = 0; c < D / 32; c += 2) {
+          float v[64];
+          tc::tmem_ld32_at(obase + (idx & 1) * D + c * 32, v);
+          tc::tmem_ld32_at(obase + (idx & 1) * D + c * 32 + 32, v + 32);
           tc::tmem_wait_ld();
+          if (c + 2 >= D / 32) {
+            // the O buffer has been read: the next O = P V may overwrite it
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(b_ofree + 8 * (idx & 1));
+          }
           if (store) {
             uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-              d4[e] = make_uint4(pack_bf16(v[8 * e] * inv_l, v[8 * e + 1] * inv_l),
-                                 pack_bf16(v[8 * e + 2] * inv_l, v[8 * e + 3] * inv_l),
-                                 pack_bf16(v[8 * e + 4] * inv_l, v[8 * e + 5] * inv_l),
-                                 pack_bf16(v[8 * e + 6] * inv_l, v[8 * e + 7] * inv_l));
+            for (int e = 0; e < 8; ++e)
+              d4[e] = make_uint4(pack_bf16(v[8 * e] * rs.x, v[8 * e + 1] * rs.x),
+                                 pack_bf16(v[8 * e + 2] * rs.x, v[8 * e + 3] * rs.x),
+                                 pack_bf16(v[8 * e + 4] * rs.x, v[8 * e + 5] * rs.x),
+                                 pack_bf16(v[8 * e + 6] * rs.x, v[8 * e + 7] * rs.x));
           }
         }
-        if (store)
-          a.part_lse[(int64_t)pos * a.G + hi] =
-              (mx != ninf && l > 0.f) ? (msafe + log2f(l)) * kLn2 : ninf;
-        tc::fence_before_sync();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(b_ofree + 8 * tb);
-      }
-      if (leader) {
-        // release the last block, and wait for this group's products to complete
-        if (use >= 0) {
-          mbar_wait_bounded(b_kvfull + 8 * (use & 1), (use >> 1) & 1, a.st, 0x20du, a.wait_ns);
-          tc::commit(b_kvempty + 8 * ((use & 1) * kNw + wg));
-        }
-        tc::commit(b_done + 8 * (1 + wg));
-        mbar_wait_bounded(b_done + 8 * (1 + wg), 0, a.st, 0x20cu, a.wait_ns);
+        if (store) a.part_lse[prow] = rs.y;
       }
     }
   }
   tc::fence_before_sync();
   __syncthreads();
   if (warp == kWarpMma) {
+    __syncwarp();
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, TMEM_COLS);
   }
@@ -579,7 +648,8 @@ __global__ void __launch_bounds__(256) kv_combine_kernel(KvArgs a, int BLK) {
     float l = ninf;
     if (s < a.topk) {
       const int beta = __ldg(row_ids + s);
-      if (beta >= 0 && beta < a.nblk && beta * BLK < lim) l = __ldg(a.part_lse + (p0 + s) * a.G + hi);
+      if (beta >= 0 && beta < a.nblk && beta * BLK < lim)
+        l = __ldg(a.part_lse + __ldg(a.slot_row + p0 + s) + hi);
     }
     M = fmaxf(M, l);
   }
@@ -593,16 +663,19 @@ __global__ void __launch_bounds__(256) kv_combine_kernel(KvArgs a, int BLK) {
     for (int s0 = 0; s0 < a.topk; s0 += 32) {
       const int s = s0 + lane;
       float wgt = 0.f;
+      int prow = 0;  // partial row of this lane's slot (row 0 stands in for none)
       if (s < a.topk) {
         const int beta = __ldg(row_ids + s);
-        if (beta >= 0 && beta < a.nblk && beta * BLK < lim)
-          wgt = __expf(__ldg(a.part_lse + (p0 + s) * a.G + hi) - M);
+        if (beta >= 0 && beta < a.nblk && beta * BLK < lim) {
+          prow = __ldg(a.slot_row + p0 + s) + hi;
+          wgt = __expf(__ldg(a.part_lse + prow) - M);
+        }
       }
       den += wgt;
-      // Loads are issued for every slot of the pass (the buffer is allocated for all
-      // of them); a slot without a partial contributes through a select, never a
-      // multiply, so whatever its memory holds cannot leak into the sum.  Eight
-      // slots per round keep several loads in flight per lane.
+      // Loads are issued for every slot of the pass (a slot without a partial reads
+      // row 0, which exists); such a slot contributes through a select, never a
+      // multiply, so whatever that row holds cannot leak into the sum.  Eight slots
+      // per round keep several loads in flight per lane.
       const int cnt = min(32, a.topk - s0);
       for (int j0 = 0; j0 < cnt; j0 += 8) {
         uint2 u[8];
@@ -612,7 +685,8 @@ __global__ void __launch_bounds__(256) kv_combine_kernel(KvArgs a, int BLK) {
           const int jj = min(j0 + j, cnt - 1);
           wj[j] = __shfl_sync(0xffffffffu, wgt, jj);
           if (j0 + j >= cnt) wj[j] = 0.f;
-          const uint16_t* src = a.part_o + ((p0 + s0 + jj) * a.G + hi) * D + lane * PER;
+          const int rj = __shfl_sync(0xffffffffu, prow, jj);
+          const uint16_t* src = a.part_o + (int64_t)rj * D + lane * PER;
           if constexpr (PER == 4) {
             u[j] = __ldg(reinterpret_cast<const uint2*>(src));
           } else {
@@ -656,8 +730,8 @@ constexpr size_t kKvPartialBudget = size_t(6) << 30;  // partial bytes per query
 struct KvPlan {
   int64_t rows, chunk_rows;
   int nchunks, qpt;
-  int64_t nj;
-  size_t counts_off, offs_off, toffs_off, entries_off, lse_off, o_off, total;
+  int64_t nj, max_tiles;
+  size_t counts_off, offs_off, toffs_off, entries_off, slot_row_off, lse_off, o_off, total;
 };
 
 size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -667,14 +741,19 @@ KvPlan plan_kv(const Shape& s) {
   p.rows = (int64_t)s.batch * s.n_q;
   p.nj = (int64_t)s.batch * s.h * s.nblk;
   p.qpt = kRows / s.G;
-  const size_t per_row = (size_t)s.h * s.topk * (4 + (size_t)s.G * 4 + (size_t)s.G * s.d * 2);
-  int64_t cr = (int64_t)(kKvPartialBudget / per_row);
+  // A chunk's tiles number at most ceil(slots / qpt) + nj (one partly filled
+  // tile per list); each holds 128 partial rows of d bf16 and one float.
+  const size_t row_bytes = (size_t)s.d * 2 + 4;
+  const size_t fixed = (size_t)(p.nj + 1) * kRows * row_bytes;
+  const size_t per_bt = (size_t)s.h * s.topk * (8 + kRows * row_bytes / p.qpt + 1);
+  int64_t cr = fixed < kKvPartialBudget ? (int64_t)((kKvPartialBudget - fixed) / per_bt) : 1;
   cr = cr < 1 ? 1 : cr;
   const int64_t max_slots = (int64_t)1 << 30;  // chunk-relative positions are int32
   if (cr * s.h * s.topk > max_slots) cr = max_slots / ((int64_t)s.h * s.topk);
   p.chunk_rows = cr < p.rows ? cr : p.rows;
   p.nchunks = (int)((p.rows + p.chunk_rows - 1) / p.chunk_rows);
   const size_t slots = (size_t)p.chunk_rows * s.h * s.topk;
+  p.max_tiles = (int64_t)((slots + p.qpt - 1) / p.qpt) + p.nj;
   size_t off = 0;
   p.counts_off = off;
   off = up256(off + p.nj * 4);
@@ -684,20 +763,29 @@ KvPlan plan_kv(const Shape& s) {
   off = up256(off + (p.nj + 1) * 4);
   p.entries_off = off;
   off = up256(off + slots * 4);
+  p.slot_row_off = off;
+  off = up256(off + slots * 4);
   p.lse_off = off;
-  off = up256(off + slots * s.G * 4);
+  off = up256(off + (size_t)p.max_tiles * kRows * 4);
   p.o_off = off;
-  off = up256(off + slots * s.G * s.d * 2);
+  off = up256(off + (size_t)p.max_tiles * kRows * s.d * 2);
   p.total = off;
   return p;
 }
 
 template <int D, int BLK>
-cudaError_t run_kv(const Shape& s, KvArgs& a, const KvPlan& p, const CUtensorMap& tmk,
-                   const CUtensorMap& tmv, uint8_t* ws, cudaStream_t stream) {
+cudaError_t run_kv(const Shape& s, KvArgs& a, const KvPlan& p, const CUtensorMap& tmq,
+                   const CUtensorMap& tmk, const CUtensorMap& tmv, uint8_t* ws,
+                   cudaStream_t stream) {
   constexpr uint32_t smem = KvSmem<D, BLK>::BYTES;
-  cudaError_t err = cudaFuncSetAttribute(kv_attn_kernel<D, BLK>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  // The register reallocation inside the kernel is sized for a launch with
+  // kRegsLaunch registers per thread; any other build would wait forever.
+  cudaFuncAttributes fa;
+  cudaError_t err = cudaFuncGetAttributes(&fa, kv_attn_kernel<D, BLK>);
+  if (err != cudaSuccess) return err;
+  if (fa.numRegs != kRegsLaunch) return cudaErrorInvalidKernelImage;
+  err = cudaFuncSetAttribute(kv_attn_kernel<D, BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem);
   if (err != cudaSuccess) return err;
   const int sms = num_sms();
   for (int c = 0; c < p.nchunks; ++c) {
@@ -710,7 +798,7 @@ cudaError_t run_kv(const Shape& s, KvArgs& a, const KvPlan& p, const CUtensorMap
     kv_count_kernel<<<grid, 256, 0, stream>>>(a, BLK);
     kv_scan_kernel<<<1, 1024, 0, stream>>>(a);
     kv_scatter_kernel<<<grid, 256, 0, stream>>>(a, BLK);
-    kv_attn_kernel<D, BLK><<<sms, kKvThreads, smem, stream>>>(tmk, tmv, a);
+    kv_attn_kernel<D, BLK><<<sms, kKvThreads, smem, stream>>>(tmq, tmk, tmv, a);
     const int64_t warps = (int64_t)a.nbt * s.H;
     kv_combine_kernel<D><<<(unsigned)((warps + 7) / 8), 256, 0, stream>>>(a, BLK);
     err = cudaGetLastError();
@@ -722,15 +810,17 @@ cudaError_t run_kv(const Shape& s, KvArgs& a, const KvPlan& p, const CUtensorMap
 }  // namespace
 
 bool kv_attn_supported(const Shape& s) {
+  // partial rows are addressed with int32
   return s.n_q > 1 && (s.d == 64 || s.d == 128) && (s.block == 64 || s.block == 128) &&
-         (int64_t)s.batch * s.h * s.nblk < ((int64_t)1 << 30);
+         plan_kv(s).max_tiles * kRows < ((int64_t)1 << 31);
 }
 
 size_t kv_workspace_bytes(const Shape& s) { return plan_kv(s).total; }
 
 int kv_launches(const Shape& s) { return 5 * plan_kv(s).nchunks; }
 
-cudaError_t launch_kv_attn(const Shape& s, const CUtensorMap& tmk, const CUtensorMap& tmv,
+cudaError_t launch_kv_attn(const Shape& s, const CUtensorMap& tmq, const CUtensorMap& tmk,
+                           const CUtensorMap& tmv,
                            const uint16_t* q, const int32_t* ids, uint16_t* out, float* lse,
                            void* ws, size_t ws_bytes, DeviceStatus* st, cudaStream_t stream) {
   const KvPlan p = plan_kv(s);
@@ -756,6 +846,7 @@ cudaError_t launch_kv_attn(const Shape& s, const CUtensorMap& tmk, const CUtenso
   a.offs = reinterpret_cast<int*>(w + p.offs_off);
   a.toffs = reinterpret_cast<int*>(w + p.toffs_off);
   a.entries = reinterpret_cast<int*>(w + p.entries_off);
+  a.slot_row = reinterpret_cast<int*>(w + p.slot_row_off);
   a.qpt = p.qpt;
   a.nj = (int)p.nj;
   a.part_lse = reinterpret_cast<float*>(w + p.lse_off);
@@ -767,10 +858,10 @@ cudaError_t launch_kv_attn(const Shape& s, const CUtensorMap& tmk, const CUtenso
   a.lse = lse;
   a.st = st;
   a.wait_ns = 4000000000ull;
-  if (s.d == 128 && s.block == 128) return run_kv<128, 128>(s, a, p, tmk, tmv, w, stream);
-  if (s.d == 128 && s.block == 64) return run_kv<128, 64>(s, a, p, tmk, tmv, w, stream);
-  if (s.d == 64 && s.block == 128) return run_kv<64, 128>(s, a, p, tmk, tmv, w, stream);
-  if (s.d == 64 && s.block == 64) return run_kv<64, 64>(s, a, p, tmk, tmv, w, stream);
+  if (s.d == 128 && s.block == 128) return run_kv<128, 128>(s, a, p, tmq, tmk, tmv, w, stream);
+  if (s.d == 128 && s.block == 64) return run_kv<128, 64>(s, a, p, tmq, tmk, tmv, w, stream);
+  if (s.d == 64 && s.block == 128) return run_kv<64, 128>(s, a, p, tmq, tmk, tmv, w, stream);
+  if (s.d == 64 && s.block == 64) return run_kv<64, 64>(s, a, p, tmq, tmk, tmv, w, stream);
   return cudaErrorInvalidValue;
 }
 
