@@ -46,6 +46,9 @@ cudaError_t launch_sparse_attn(const Shape& s, const uint16_t* q, const uint16_t
 // inverted index, tiles of gathered (query, head) rows per selected block,
 // partials merged by a combine kernel; processed in query chunks.
 bool kv_attn_supported(const Shape& s);
+// Rows of d bf16 as a 2-D tensor map with 64 x 32 boxes (128-byte swizzle), for
+// TMA stores of partial outputs.
+bool make_rows_map(CUtensorMap* map, uint16_t* base, int64_t rows, int d);
 size_t kv_workspace_bytes(const Shape& s);
 int kv_launches(const Shape& s);
 cudaError_t launch_kv_attn(const Shape& s, const CUtensorMap& tmq, const CUtensorMap& tmk,

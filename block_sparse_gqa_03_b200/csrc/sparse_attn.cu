@@ -664,6 +664,18 @@ AttnPlan plan_attn(const Shape& s) {
 
 }  // namespace
 
+bool make_rows_map(CUtensorMap* map, uint16_t* base, int64_t rows, int d) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+  cuuint32_t box[2] = {64, 32};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 size_t attn_partial_bytes(const Shape& s) {
   const AttnPlan pl = plan_attn(s);
   if (!pl.stream) return kv_attn_supported(s) ? kv_workspace_bytes(s) : 0;

@@ -12,8 +12,9 @@
 // and streams tiles of up to 128 (query, head) rows through it:
 //   S = Q_tile K^T      tcgen05 MMA, M = 128 rows, N = block, K = d   (TMEM)
 //   P = softmax(S)      registers, one thread per row, masked to visible keys,
-//                       written back to tensor memory over S as bf16
-//   O = P V             tcgen05 MMA with A = P from tensor memory, N = d (TMEM)
+//                       written to tensor memory as bf16
+//   O = P V             tcgen05 MMA with A = P from tensor memory, N = d, into
+//                       the columns that held S (TMEM)
 // Each (query, head, block) gives a normalised bf16 partial output and its
 // log-sum-exp; a combine kernel merges a query's partials by log-sum-exp weights.
 // Queries are processed in chunks so that the partials of one chunk fit a bounded
@@ -24,15 +25,16 @@
 //   warp 0        TMA producer of K and V (a new load only when the block changes;
 //                 V rows past the sequence end are zeroed after the load lands);
 //   warp 1        tensor-memory allocation and the thread issuing all MMAs: S of
-//                 tile i, then O of tile i - 1, so the next scores are computed
-//                 while a softmax runs;
+//                 tile i, then O of tile i - 2, so that a softmax warpgroup finds
+//                 its next scores computed;
 //   warps 2-3     gather the tile's Q rows with TMA, one load per (query, 64-dim
 //                 atom) bringing the query's G heads into the swizzled layout;
 //   warps 4-11    two softmax warpgroups taking tiles in turn, one thread per tile
-//                 row, each owning one S/P buffer in tensor memory;
+//                 row, each owning one P region in tensor memory;
 //   warps 12-15   output warpgroup: O / l from tensor memory to the partials.
 // Buffers: 2-4 Q tiles (released when S is computed), 2 K/V stages, and in tensor
-// memory two S/P buffers and two O buffers.  Every wait is bounded.
+// memory 3-4 slots, each holding a tile's S and then its O, plus the two P
+// regions.  Every wait is bounded.
 #include "kernels.h"
 #include "sm100.cuh"
 
@@ -46,7 +48,7 @@ constexpr int kWarpProd = 0, kWarpMma = 1, kWarpGather = 2;
 // what the kernel is launched with (128 per thread; the host refuses to launch a
 // build that was given another count, since the softmax warpgroups would then
 // wait for registers that are never released).
-constexpr int kRegsLaunch = 128, kRegsLoad = 48, kRegsSoft = 184, kRegsOut = 96;
+constexpr int kRegsLaunch = 128, kRegsLoad = 40, kRegsSoft = 184, kRegsOut = 104;
 static_assert(kRegsLoad + 2 * kRegsSoft + kRegsOut == 4 * kRegsLaunch, "register split");
 
 struct KvArgs {
@@ -64,14 +66,17 @@ struct KvArgs {
   int* counts;             // [batch * h * nblk]
   int* offs;               // [batch * h * nblk + 1] entry offsets
   int* toffs;              // [batch * h * nblk + 1] tile offsets
-  int* entries;            // query index t of each entry, grouped by (b, g, block)
+  int2* entries;           // {chunk-relative slot position, query index t} of each
+                           // entry, grouped by (b, g, block)
   int* slot_row;           // [slot] partial row of a valid slot's query (head 0) in its tile
   int qpt;                 // queries per tile
   int nj;                  // batch * h * nblk
-  // partials: 128 rows per tile, row = tile * 128 + query-in-tile * G + head, so
-  // that a tile's output is one contiguous block
+  // partial outputs: 128 rows per tile, row = tile * 128 + query-in-tile * G +
+  // head, so that a tile's output is one contiguous block; their log-sum-exps by
+  // chunk-relative slot position p = (bt_rel * h + g) * topk + slot, so that a
+  // query's are contiguous
   uint16_t* part_o;        // [row][d] bf16
-  float* part_lse;         // [row]
+  float* part_lse;         // [p][G]
   uint16_t* out;
   int64_t o_s0, o_s1, o_s2;
   float* lse;
@@ -179,7 +184,7 @@ __global__ void kv_scatter_kernel(KvArgs a, int BLK) {
     if (slot_block(a, pos, b, g, t, beta, BLK)) {
       const int64_t j = ((int64_t)b * a.h + g) * a.nblk + beta;
       const int k = atomicAdd(&a.counts[j], 1);
-      a.entries[a.offs[j] + k] = t;
+      a.entries[a.offs[j] + k] = make_int2((int)pos, t);
       a.slot_row[pos] = (a.toffs[j] + k / a.qpt) * kRows + (k % a.qpt) * a.G;
     }
   }
@@ -248,26 +253,33 @@ struct KvSmem {
   static constexpr uint32_t HALF = BLK * 128u;         // one 64-dim atom of K or V
   static constexpr uint32_t KV = 2 * (D / 64) * HALF;  // K and V of one block
   // row statistics [4][128] float2, row table [128] int, barriers, TMEM address
+  // (barriers from 4608, the TMEM address at 4992)
   static constexpr uint32_t MISC = 5120;
+  static constexpr uint32_t STAGE = 4 * 32 * 128;  // output staging, one tile per warp
   static constexpr uint32_t LIMIT = 227u * 1024u;
-  static constexpr int NQ = 1024 + 4 * Q + 2 * KV + MISC <= LIMIT   ? 4
-                            : 1024 + 3 * Q + 2 * KV + MISC <= LIMIT ? 3
-                                                                    : 2;
-  static constexpr uint32_t BYTES = 1024 + NQ * Q + 2 * KV + MISC;
+  static constexpr uint32_t FIXED = 1024 + 2 * KV + MISC + STAGE;
+  static constexpr int NQ = FIXED + 4 * Q <= LIMIT ? 4 : FIXED + 3 * Q <= LIMIT ? 3 : 2;
+  static constexpr uint32_t BYTES = FIXED + NQ * Q;
   static_assert(BYTES <= LIMIT, "shared memory");
 };
 
 template <int D, int BLK>
 __global__ void __launch_bounds__(kKvThreads, 1)
     kv_attn_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
-                   const __grid_constant__ CUtensorMap tmv, KvArgs a) {
+                   const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmo,
+                   KvArgs a) {
   using SM = KvSmem<D, BLK>;
   constexpr int NH = D / 64;
   constexpr int NQ = SM::NQ;
   constexpr uint32_t QB = SM::Q, HALF = SM::HALF, KV_BYTES = SM::KV;
-  constexpr uint32_t TMEM_COLS = 2 * (BLK + D) <= 256 ? 256 : 512;
-  constexpr uint32_t O_COL = 2 * BLK;  // two S/P buffers, then two O buffers
-  static_assert(2 * (BLK + D) <= 512, "tensor memory");
+  // Tensor memory: NS slots of W columns, each holding a tile's S and then its
+  // O (O = P V overwrites the S it was computed from), and two P regions of
+  // BLK / 2 columns (bf16 pairs), one per softmax warpgroup.
+  constexpr uint32_t W = BLK > D ? BLK : D;
+  constexpr int NS = (512 - BLK) / W < 4 ? (512 - BLK) / W : 4;
+  constexpr uint32_t PB = NS * W;
+  constexpr uint32_t TMEM_COLS = PB + BLK <= 256 ? 256 : 512;
+  static_assert(NS >= 3 && PB + BLK <= 512, "tensor memory");
   if (status_failed(a.st)) return;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -282,13 +294,15 @@ __global__ void __launch_bounds__(kKvThreads, 1)
   const uint32_t b_kvempty = b_kvland + 16;             // [2]
   const uint32_t b_qfull = b_kvempty + 16;              // [NQ]
   const uint32_t b_qempty = b_qfull + 8 * NQ;           // [NQ]
-  const uint32_t b_sfull = b_qempty + 8 * NQ;           // [2]
-  const uint32_t b_pfull = b_sfull + 16;                // [2]
-  const uint32_t b_ofull = b_pfull + 16;                // [2]
-  const uint32_t b_ofree = b_ofull + 16;                // [2]
-  const uint32_t b_lfull = b_ofree + 16;                // [4]
+  const uint32_t b_sfull = b_qempty + 8 * NQ;           // [4] S of a slot computed
+  const uint32_t b_ofull = b_sfull + 32;                // [4] O of a slot computed
+  const uint32_t b_sfree = b_ofull + 32;                // [4] O of a slot read out
+  const uint32_t b_pfull = b_sfree + 32;                // [2] P written
+  const uint32_t b_pfree = b_pfull + 16;                // [2] P consumed
+  const uint32_t b_lfull = b_pfree + 16;                // [4] row statistics written
   const uint32_t b_done = b_lfull + 32;                 // [1]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + 4864);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + 4992);
+  uint8_t* staging = misc + SM::MISC;                   // [4 warps][32 rows][128 bytes]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ntiles = __ldg(a.toffs + a.nj);
@@ -302,10 +316,13 @@ __global__ void __launch_bounds__(kKvThreads, 1)
       mbar_init(b_kvfull + 8 * s, 1);
       mbar_init(b_kvland + 8 * s, 1);
       mbar_init(b_kvempty + 8 * s, 1);
-      mbar_init(b_sfull + 8 * s, 1);
       mbar_init(b_pfull + 8 * s, 4);
-      mbar_init(b_ofull + 8 * s, 1);
-      mbar_init(b_ofree + 8 * s, 4);
+      mbar_init(b_pfree + 8 * s, 1);
+    }
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(b_sfull + 8 * i, 1);
+      mbar_init(b_ofull + 8 * i, 1);
+      mbar_init(b_sfree + 8 * i, 4);
     }
     for (int i = 0; i < NQ; ++i) {
       mbar_init(b_qfull + 8 * i, 2);
@@ -390,26 +407,53 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     if (n > 0) {
       w.seek(a, tile0);
       if (lane == 0) {
+        // S of tile i is issued two tiles ahead of O = P V of tile i - 2, so that a
+        // softmax warpgroup finds its next S ready.  For each tile, two bits of
+        // `hist` record its K/V stage and whether it is the last tile of its block.
         const uint32_t id_qk = tc::idesc_bf16(kRows, BLK, false);
         const uint32_t id_pv = tc::idesc_bf16(kRows, D, true);
-        int use = -1, stage_prev = 0;
+        int use = -1;
+        uint32_t hist = 0;
         bool ok = true;
-        for (int idx = 0; idx <= n && ok; ++idx) {
-          bool block_ends = true;  // the previous tile was the last of its block
+        auto issue_pv = [&](int k) {
+          const int p = k & 1, sk = k % NS;
+          ok = mbar_wait_bounded(b_pfull + 8 * p, (k >> 1) & 1, a.st, 0x207u, a.wait_ns);
+          if (!ok) return;
+          tc::fence_after_sync();
+          const uint32_t h = hist >> (2 * (k & 7));
+          const uint32_t vd = skv + (h & 1u) * KV_BYTES + NH * HALF;
+#pragma unroll
+          for (int ks = 0; ks < BLK / 16; ++ks)
+            tc::mma_bf16_ts(tmem + sk * W, tmem + PB + p * (BLK / 2) + ks * 8,
+                            tc::desc_mn_sw128(vd + ks * 16 * 128, HALF), id_pv, ks > 0 ? 1u : 0u);
+          tc::commit(b_ofull + 8 * sk);
+          tc::commit(b_pfree + 8 * p);
+          if (h & 2u) tc::commit(b_kvempty + 8 * (h & 1u));  // K/V stage released
+        };
+        for (int idx = 0; idx < n + 2 && ok; ++idx) {
+          bool pv_done = idx < 2;  // O = P V of tile idx - 2 issued
           if (idx < n) {
-            // S = Q K^T of tile idx into S/P buffer idx & 1
-            const int tile = tile0 + idx;
-            block_ends = w.advance(a, tile) || idx == 0;
-            if (block_ends) {
+            const int tile = tile0 + idx, sk = idx % NS, qb = idx % NQ;
+            const bool nb = w.advance(a, tile) || idx == 0;
+            if (nb) {
               ++use;
+              if (idx > 0) hist |= 2u << (2 * ((idx - 1) & 7));  // previous tile ends a block
+              // The new block's stage is released by the products of the block
+              // before the previous one; the last of those may be tile idx - 2.
+              if (!pv_done) {
+                issue_pv(idx - 2);
+                pv_done = true;
+                if (!ok) break;
+              }
               ok = mbar_wait_bounded(b_kvfull + 8 * (use & 1), (use >> 1) & 1, a.st, 0x204u,
                                      a.wait_ns);
             }
-            const int qb = idx % NQ, s = idx & 1;
+            hist = (hist & ~(3u << (2 * (idx & 7)))) | ((uint32_t)(use & 1) << (2 * (idx & 7)));
             if (ok) ok = mbar_wait_bounded(b_qfull + 8 * qb, (idx / NQ) & 1, a.st, 0x205u, a.wait_ns);
-            // the buffer's previous P has been consumed by its O = P V
-            if (ok && idx >= 2)
-              ok = mbar_wait_bounded(b_ofull + 8 * s, ((idx - 2) >> 1) & 1, a.st, 0x206u, a.wait_ns);
+            // the slot's previous O has been read out
+            if (ok && idx >= NS)
+              ok = mbar_wait_bounded(b_sfree + 8 * sk, ((idx / NS) - 1) & 1, a.st, 0x206u,
+                                     a.wait_ns);
             if (!ok) break;
             tc::fence_after_sync();
             const uint32_t kd = skv + (use & 1) * KV_BYTES, qd = sq + qb * QB;
@@ -417,29 +461,15 @@ __global__ void __launch_bounds__(kKvThreads, 1)
             for (int ks = 0; ks < D / 16; ++ks) {
               const uint32_t qoff = (ks >> 2) * (kRows * 128u) + (ks & 3) * 32;
               const uint32_t koff = (ks >> 2) * HALF + (ks & 3) * 32;
-              tc::mma_bf16(tmem + s * BLK, tc::desc_k_sw128(qd + qoff), tc::desc_k_sw128(kd + koff),
+              tc::mma_bf16(tmem + sk * W, tc::desc_k_sw128(qd + qoff), tc::desc_k_sw128(kd + koff),
                            id_qk, ks > 0 ? 1u : 0u);
             }
-            tc::commit(b_sfull + 8 * s);
+            tc::commit(b_sfull + 8 * sk);
             tc::commit(b_qempty + 8 * qb);  // the Q tile may be refilled
+          } else if (idx == n) {
+            hist |= 2u << (2 * ((n - 1) & 7));  // the last tile ends its block
           }
-          if (idx >= 1) {
-            // O = P V of tile idx - 1 into O buffer (idx - 1) & 1
-            const int k = idx - 1, s = k & 1;
-            ok = mbar_wait_bounded(b_pfull + 8 * s, (k >> 1) & 1, a.st, 0x207u, a.wait_ns);
-            if (ok && k >= 2)
-              ok = mbar_wait_bounded(b_ofree + 8 * s, ((k >> 1) - 1) & 1, a.st, 0x208u, a.wait_ns);
-            if (!ok) break;
-            tc::fence_after_sync();
-            const uint32_t vd = skv + stage_prev * KV_BYTES + NH * HALF;
-#pragma unroll
-            for (int ks = 0; ks < BLK / 16; ++ks)
-              tc::mma_bf16_ts(tmem + O_COL + s * D, tmem + s * BLK + ks * 8,
-                              tc::desc_mn_sw128(vd + ks * 16 * 128, HALF), id_pv, ks > 0 ? 1u : 0u);
-            tc::commit(b_ofull + 8 * s);
-            if (block_ends) tc::commit(b_kvempty + 8 * stage_prev);  // K/V stage released
-          }
-          stage_prev = use & 1;
+          if (!pv_done) issue_pv(idx - 2);
         }
         tc::commit(b_done);
         mbar_wait_bounded(b_done, 0, a.st, 0x209u, a.wait_ns);
@@ -461,7 +491,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
       auto load_t = [&](int first, int nq, int (&tq)[4]) {
 #pragma unroll
         for (int k = 0; k < 4; ++k)
-          tq[k] = 32 * k + lane < nq ? __ldg(a.entries + first + 32 * k + lane) : 0;
+          tq[k] = 32 * k + lane < nq ? __ldg(&a.entries[first + 32 * k + lane].y) : 0;
       };
       int first = w.first(a, tile0), nq = w.count(a, tile0), b = w.b, g = w.g;
       int tq[4];
@@ -500,9 +530,10 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     tc::regs_inc<kRegsSoft>();
     if (n > 0) {
       w.seek(a, tile0);
-      const int sw = wg - 1;  // tiles idx with idx % 2 == sw; S/P buffer sw
+      const int sw = wg - 1;  // tiles idx with idx % 2 == sw; P region sw
       const int quarter = warp & 3, row = quarter * 32 + lane;
-      const uint32_t sp = tmem + ((uint32_t)(quarter * 32) << 16) + sw * BLK;
+      const uint32_t lanes = tmem + ((uint32_t)(quarter * 32) << 16);
+      const uint32_t pr = lanes + PB + sw * (BLK / 2);
       const int qi = rowtab[row] & 0xffff;
       const float ninf = -__int_as_float(0x7f800000);
       const float kLn2 = 0.69314718055994531f;
@@ -513,18 +544,19 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         w.advance(a, tile);
         int vis = BLK;  // keys [0, vis) of the block are visible to this row
         if (qi < w.count(a, tile)) {
-          const int t = __ldg(a.entries + w.first(a, tile) + qi);
+          const int t = __ldg(&a.entries[w.first(a, tile) + qi].y);
           if (w.b != Lb) {
             Lb = w.b;
             L = kv_length(a.seq_lens, w.b, a.max_kv, a.st);
           }
           vis = visible_from_length(a, L, t) - w.beta * BLK;
         }
-        if (ok) ok = mbar_wait_warp(b_sfull + 8 * sw, (idx >> 1) & 1, a.st, 0x20bu, a.wait_ns);
+        const int sk = idx % NS;
+        if (ok) ok = mbar_wait_warp(b_sfull + 8 * sk, (idx / NS) & 1, a.st, 0x20bu, a.wait_ns);
         tc::fence_after_sync();
         float v[BLK];
 #pragma unroll
-        for (int c = 0; c < BLK / 32; ++c) tc::tmem_ld32_at(sp + c * 32, v + c * 32);
+        for (int c = 0; c < BLK / 32; ++c) tc::tmem_ld32_at(lanes + sk * W + c * 32, v + c * 32);
         tc::tmem_wait_ld();
         if (vis < BLK) {
 #pragma unroll
@@ -541,7 +573,11 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         const float ms = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3])) * a.scale_log2;
         const float msafe = ms != ninf ? ms : 0.f;
         // probabilities (masked keys hold -inf and give exactly 0), their sum and
-        // the bf16 P row written over the first half of the row's S columns
+        // the bf16 P row, written to this warpgroup's P region once the O = P V of
+        // its previous tile has consumed it
+        if (ok && idx >= 2)
+          ok = mbar_wait_warp(b_pfree + 8 * sw, ((idx >> 1) - 1) & 1, a.st, 0x20eu, a.wait_ns);
+        tc::fence_after_sync();
         float l4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int c = 0; c < BLK / 32; ++c) {
@@ -553,7 +589,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
             l4[e & 3] += p0 + p1;
             pk[e] = pack_bf16(p0, p1);
           }
-          tc::tmem_st16(sp + c * 16, pk);
+          tc::tmem_st16(pr + c * 16, pk);
         }
         tc::tmem_wait_st();
         const float l = (l4[0] + l4[1]) + (l4[2] + l4[3]);
@@ -569,48 +605,65 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     }
   } else {
     // -------------------------------------------------------- output warpgroup
+    // Each warp writes its 32 rows of a 64-dim half into a 128-byte-swizzled
+    // staging tile (four shared-memory wavefronts per instruction) and one TMA
+    // store moves the tile to the partials; a tile's padding rows receive
+    // whatever the unused tensor-memory lanes hold and are never read.
     tc::regs_dec<kRegsOut>();
     if (n > 0) {
       w.seek(a, tile0);
       const int quarter = warp & 3, row = quarter * 32 + lane;
-      const int qi = rowtab[row] & 0xffff;
-      const uint32_t obase = tmem + ((uint32_t)(quarter * 32) << 16) + O_COL;
+      const int info = rowtab[row];
+      const int qi = info & 0xffff, hi = info >> 16;
+      const uint32_t lanes = tmem + ((uint32_t)(quarter * 32) << 16);
+      const uint32_t stg = smem_u32(staging) + quarter * 4096u;
+      if (lane == 0) prefetch_tensormap(&tmo);
       bool ok = true;
       for (int idx = 0; idx < n; ++idx) {
         const int tile = tile0 + idx;
         w.advance(a, tile);
         const bool live = qi < w.count(a, tile);
+        const int pos = live ? __ldg(&a.entries[w.first(a, tile) + qi].x) : 0;
         if (ok) ok = mbar_wait_warp(b_lfull + 8 * (idx & 3), (idx >> 2) & 1, a.st, 0x20cu, a.wait_ns);
         const float2 rs = rstat[(idx & 3) * kRows + row];
-        if (ok) ok = mbar_wait_warp(b_ofull + 8 * (idx & 1), (idx >> 1) & 1, a.st, 0x20du, a.wait_ns);
+        const int sk = idx % NS;
+        if (ok) ok = mbar_wait_warp(b_ofull + 8 * sk, (idx / NS) & 1, a.st, 0x20du, a.wait_ns);
         tc::fence_after_sync();
-        const bool store = ok && live;
-        const int64_t prow = (int64_t)tile * kRows + row;  // this thread's partial row
-        uint16_t* dst = a.part_o + (store ? prow * D : 0);
 #pragma unroll
         for (int c = 0; c < D / 32; c += 2) {
           float v[64];
-          tc::tmem_ld32_at(obase + (idx & 1) * D + c * 32, v);
-          tc::tmem_ld32_at(obase + (idx & 1) * D + c * 32 + 32, v + 32);
+          tc::tmem_ld32_at(lanes + sk * W + c * 32, v);
+          tc::tmem_ld32_at(lanes + sk * W + c * 32 + 32, v + 32);
           tc::tmem_wait_ld();
           if (c + 2 >= D / 32) {
-            // the O buffer has been read: the next O = P V may overwrite it
+            // the slot has been read out: the next S may overwrite it
             tc::fence_before_sync();
             __syncwarp();
-            if (lane == 0) mbar_arrive(b_ofree + 8 * (idx & 1));
+            if (lane == 0) mbar_arrive(b_sfree + 8 * sk);
           }
-          if (store) {
-            uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+          // the previous store has finished reading the staging tile
+          if (lane == 0) bulk_wait_read0();
+          __syncwarp();
 #pragma unroll
-            for (int e = 0; e < 8; ++e)
-              d4[e] = make_uint4(pack_bf16(v[8 * e] * rs.x, v[8 * e + 1] * rs.x),
-                                 pack_bf16(v[8 * e + 2] * rs.x, v[8 * e + 3] * rs.x),
-                                 pack_bf16(v[8 * e + 4] * rs.x, v[8 * e + 5] * rs.x),
-                                 pack_bf16(v[8 * e + 6] * rs.x, v[8 * e + 7] * rs.x));
+          for (int e = 0; e < 8; ++e) {
+            const uint32_t u0 = pack_bf16(v[8 * e] * rs.x, v[8 * e + 1] * rs.x);
+            const uint32_t u1 = pack_bf16(v[8 * e + 2] * rs.x, v[8 * e + 3] * rs.x);
+            const uint32_t u2 = pack_bf16(v[8 * e + 4] * rs.x, v[8 * e + 5] * rs.x);
+            const uint32_t u3 = pack_bf16(v[8 * e + 6] * rs.x, v[8 * e + 7] * rs.x);
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(stg + swz128(lane, e)),
+                         "r"(u0), "r"(u1), "r"(u2), "r"(u3)
+                         : "memory");
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0 && ok) {
+            tma_store_2d(&tmo, stg, (c / 2) * 64, tile * kRows + quarter * 32);
+            bulk_commit();
           }
         }
-        if (store) a.part_lse[prow] = rs.y;
+        if (ok && live) a.part_lse[(int64_t)pos * a.G + hi] = rs.y;
       }
+      if (lane == 0) bulk_wait0();
     }
   }
   tc::fence_before_sync();
@@ -648,8 +701,7 @@ __global__ void __launch_bounds__(256) kv_combine_kernel(KvArgs a, int BLK) {
     float l = ninf;
     if (s < a.topk) {
       const int beta = __ldg(row_ids + s);
-      if (beta >= 0 && beta < a.nblk && beta * BLK < lim)
-        l = __ldg(a.part_lse + __ldg(a.slot_row + p0 + s) + hi);
+      if (beta >= 0 && beta < a.nblk && beta * BLK < lim) l = __ldg(a.part_lse + (p0 + s) * a.G + hi);
     }
     M = fmaxf(M, l);
   }
@@ -668,20 +720,20 @@ __global__ void __launch_bounds__(256) kv_combine_kernel(KvArgs a, int BLK) {
         const int beta = __ldg(row_ids + s);
         if (beta >= 0 && beta < a.nblk && beta * BLK < lim) {
           prow = __ldg(a.slot_row + p0 + s) + hi;
-          wgt = __expf(__ldg(a.part_lse + prow) - M);
+          wgt = __expf(__ldg(a.part_lse + (p0 + s) * a.G + hi) - M);
         }
       }
       den += wgt;
       // Loads are issued for every slot of the pass (a slot without a partial reads
       // row 0, which exists); such a slot contributes through a select, never a
-      // multiply, so whatever that row holds cannot leak into the sum.  Eight slots
+      // multiply, so whatever that row holds cannot leak into the sum.  Sixteen slots
       // per round keep several loads in flight per lane.
       const int cnt = min(32, a.topk - s0);
-      for (int j0 = 0; j0 < cnt; j0 += 8) {
-        uint2 u[8];
-        float wj[8];
+      for (int j0 = 0; j0 < cnt; j0 += 16) {
+        uint2 u[16];
+        float wj[16];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
+        for (int j = 0; j < 16; ++j) {
           const int jj = min(j0 + j, cnt - 1);
           wj[j] = __shfl_sync(0xffffffffu, wgt, jj);
           if (j0 + j >= cnt) wj[j] = 0.f;
@@ -694,7 +746,7 @@ __global__ void __launch_bounds__(256) kv_combine_kernel(KvArgs a, int BLK) {
           }
         }
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
+        for (int j = 0; j < 16; ++j) {
           const bool use = wj[j] != 0.f;
           acc[0] += use ? wj[j] * __uint_as_float(u[j].x << 16) : 0.f;
           acc[1] += use ? wj[j] * __uint_as_float(u[j].x & 0xffff0000u) : 0.f;
@@ -742,10 +794,12 @@ KvPlan plan_kv(const Shape& s) {
   p.nj = (int64_t)s.batch * s.h * s.nblk;
   p.qpt = kRows / s.G;
   // A chunk's tiles number at most ceil(slots / qpt) + nj (one partly filled
-  // tile per list); each holds 128 partial rows of d bf16 and one float.
-  const size_t row_bytes = (size_t)s.d * 2 + 4;
+  // tile per list); each holds 128 partial rows of d bf16.  Per slot: its entry,
+  // its partial row and G log-sum-exps.
+  const size_t row_bytes = (size_t)s.d * 2;
   const size_t fixed = (size_t)(p.nj + 1) * kRows * row_bytes;
-  const size_t per_bt = (size_t)s.h * s.topk * (8 + kRows * row_bytes / p.qpt + 1);
+  const size_t per_bt =
+      (size_t)s.h * s.topk * (12 + (size_t)s.G * 4 + kRows * row_bytes / p.qpt + 1);
   int64_t cr = fixed < kKvPartialBudget ? (int64_t)((kKvPartialBudget - fixed) / per_bt) : 1;
   cr = cr < 1 ? 1 : cr;
   const int64_t max_slots = (int64_t)1 << 30;  // chunk-relative positions are int32
@@ -762,11 +816,11 @@ KvPlan plan_kv(const Shape& s) {
   p.toffs_off = off;
   off = up256(off + (p.nj + 1) * 4);
   p.entries_off = off;
-  off = up256(off + slots * 4);
+  off = up256(off + slots * 8);
   p.slot_row_off = off;
   off = up256(off + slots * 4);
   p.lse_off = off;
-  off = up256(off + (size_t)p.max_tiles * kRows * 4);
+  off = up256(off + slots * s.G * 4);
   p.o_off = off;
   off = up256(off + (size_t)p.max_tiles * kRows * s.d * 2);
   p.total = off;
@@ -775,8 +829,8 @@ KvPlan plan_kv(const Shape& s) {
 
 template <int D, int BLK>
 cudaError_t run_kv(const Shape& s, KvArgs& a, const KvPlan& p, const CUtensorMap& tmq,
-                   const CUtensorMap& tmk, const CUtensorMap& tmv, uint8_t* ws,
-                   cudaStream_t stream) {
+                   const CUtensorMap& tmk, const CUtensorMap& tmv, const CUtensorMap& tmo,
+                   uint8_t* ws, cudaStream_t stream) {
   constexpr uint32_t smem = KvSmem<D, BLK>::BYTES;
   // The register reallocation inside the kernel is sized for a launch with
   // kRegsLaunch registers per thread; any other build would wait forever.
@@ -798,7 +852,7 @@ cudaError_t run_kv(const Shape& s, KvArgs& a, const KvPlan& p, const CUtensorMap
     kv_count_kernel<<<grid, 256, 0, stream>>>(a, BLK);
     kv_scan_kernel<<<1, 1024, 0, stream>>>(a);
     kv_scatter_kernel<<<grid, 256, 0, stream>>>(a, BLK);
-    kv_attn_kernel<D, BLK><<<sms, kKvThreads, smem, stream>>>(tmq, tmk, tmv, a);
+    kv_attn_kernel<D, BLK><<<sms, kKvThreads, smem, stream>>>(tmq, tmk, tmv, tmo, a);
     const int64_t warps = (int64_t)a.nbt * s.H;
     kv_combine_kernel<D><<<(unsigned)((warps + 7) / 8), 256, 0, stream>>>(a, BLK);
     err = cudaGetLastError();
@@ -845,7 +899,7 @@ cudaError_t launch_kv_attn(const Shape& s, const CUtensorMap& tmq, const CUtenso
   a.counts = reinterpret_cast<int*>(w + p.counts_off);
   a.offs = reinterpret_cast<int*>(w + p.offs_off);
   a.toffs = reinterpret_cast<int*>(w + p.toffs_off);
-  a.entries = reinterpret_cast<int*>(w + p.entries_off);
+  a.entries = reinterpret_cast<int2*>(w + p.entries_off);
   a.slot_row = reinterpret_cast<int*>(w + p.slot_row_off);
   a.qpt = p.qpt;
   a.nj = (int)p.nj;
@@ -858,10 +912,12 @@ cudaError_t launch_kv_attn(const Shape& s, const CUtensorMap& tmq, const CUtenso
   a.lse = lse;
   a.st = st;
   a.wait_ns = 4000000000ull;
-  if (s.d == 128 && s.block == 128) return run_kv<128, 128>(s, a, p, tmq, tmk, tmv, w, stream);
-  if (s.d == 128 && s.block == 64) return run_kv<128, 64>(s, a, p, tmq, tmk, tmv, w, stream);
-  if (s.d == 64 && s.block == 128) return run_kv<64, 128>(s, a, p, tmq, tmk, tmv, w, stream);
-  if (s.d == 64 && s.block == 64) return run_kv<64, 64>(s, a, p, tmq, tmk, tmv, w, stream);
+  CUtensorMap tmo;
+  if (!make_rows_map(&tmo, a.part_o, p.max_tiles * kRows, s.d)) return cudaErrorInvalidValue;
+  if (s.d == 128 && s.block == 128) return run_kv<128, 128>(s, a, p, tmq, tmk, tmv, tmo, w, stream);
+  if (s.d == 128 && s.block == 64) return run_kv<128, 64>(s, a, p, tmq, tmk, tmv, tmo, w, stream);
+  if (s.d == 64 && s.block == 128) return run_kv<64, 128>(s, a, p, tmq, tmk, tmv, tmo, w, stream);
+  if (s.d == 64 && s.block == 64) return run_kv<64, 64>(s, a, p, tmq, tmk, tmv, tmo, w, stream);
   return cudaErrorInvalidValue;
 }
 
