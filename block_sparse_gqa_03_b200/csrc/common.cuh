@@ -97,6 +97,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of the phase with the given parity.
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Waits until the phase with the given parity has completed, for at most
 // `limit_ns` nanoseconds.  On expiry it records kErrTimeout and returns false;
 // it never traps and never spins without bound.
@@ -208,16 +221,18 @@ __device__ __forceinline__ float exp2_approx(float x) {
 // free: x = n + f with n = round(x) and f in [-1/2, 1/2]; 2^f from a cubic fitted
 // to it on that interval by iterated weighted least squares on the relative
 // error (largest relative error 7.5e-5 evaluated in float), and 2^n added to the
-// exponent field.  Inputs below -125 are clamped there (2^-125 instead of a
-// smaller positive number).  Adding 1.5 * 2^23 rounds x to an integer held in
-// the low mantissa bits, which the shift by 23 moves into the exponent field.
+// exponent field.  Adding 1.5 * 2^23 rounds x to an integer held in the low
+// mantissa bits, which the shift by 23 moves into the exponent field.  Inputs
+// below -125 (-inf included) give exactly 0; they are clamped first so that the
+// exponent arithmetic stays in range.
 __device__ __forceinline__ float exp2_poly(float x) {
-  x = fmaxf(x, -125.f);
-  const float t = __fadd_rn(x, 12582912.f);
-  const float f = __fsub_rn(x, __fsub_rn(t, 12582912.f));
+  const float xc = fmaxf(x, -125.f);
+  const float t = __fadd_rn(xc, 12582912.f);
+  const float f = __fsub_rn(xc, __fsub_rn(t, 12582912.f));
   const float p = fmaf(fmaf(fmaf(0.0551716685f, f, 0.2426111400f), f, 0.6932609677f), f,
                        0.9999280572f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+  const float r = __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+  return x > -125.f ? r : 0.f;
 }
 
 // Two floats to bf16x2 (lo in the low half) on the integer pipe: half a bf16 unit

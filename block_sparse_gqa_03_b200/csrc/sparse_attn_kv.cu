@@ -407,69 +407,80 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     if (n > 0) {
       w.seek(a, tile0);
       if (lane == 0) {
-        // S of tile i is issued two tiles ahead of O = P V of tile i - 2, so that a
-        // softmax warpgroup finds its next S ready.  For each tile, two bits of
-        // `hist` record its K/V stage and whether it is the last tile of its block.
+        // Two in-order streams, S = Q K^T by tile and O = P V by tile, issued as
+        // their inputs become ready, O = P V first: a blocking wait on one stream
+        // would hold back the other (an S waits for its slot to be read out, which
+        // waits for an O).  Two bits of `hist` per tile (ring of 8; O never lags S
+        // by more than NS tiles) hold its K/V stage and whether it is the last
+        // tile of its block.  No progress for wait_ns records a timeout.
         const uint32_t id_qk = tc::idesc_bf16(kRows, BLK, false);
         const uint32_t id_pv = tc::idesc_bf16(kRows, D, true);
-        int use = -1;
-        uint32_t hist = 0;
-        bool ok = true;
-        auto issue_pv = [&](int k) {
-          const int p = k & 1, sk = k % NS;
-          ok = mbar_wait_bounded(b_pfull + 8 * p, (k >> 1) & 1, a.st, 0x207u, a.wait_ns);
-          if (!ok) return;
-          tc::fence_after_sync();
-          const uint32_t h = hist >> (2 * (k & 7));
-          const uint32_t vd = skv + (h & 1u) * KV_BYTES + NH * HALF;
-#pragma unroll
-          for (int ks = 0; ks < BLK / 16; ++ks)
-            tc::mma_bf16_ts(tmem + sk * W, tmem + PB + p * (BLK / 2) + ks * 8,
-                            tc::desc_mn_sw128(vd + ks * 16 * 128, HALF), id_pv, ks > 0 ? 1u : 0u);
-          tc::commit(b_ofull + 8 * sk);
-          tc::commit(b_pfree + 8 * p);
-          if (h & 2u) tc::commit(b_kvempty + 8 * (h & 1u));  // K/V stage released
-        };
-        for (int idx = 0; idx < n + 2 && ok; ++idx) {
-          bool pv_done = idx < 2;  // O = P V of tile idx - 2 issued
-          if (idx < n) {
-            const int tile = tile0 + idx, sk = idx % NS, qb = idx % NQ;
-            const bool nb = w.advance(a, tile) || idx == 0;
-            if (nb) {
-              ++use;
-              if (idx > 0) hist |= 2u << (2 * ((idx - 1) & 7));  // previous tile ends a block
-              // The new block's stage is released by the products of the block
-              // before the previous one; the last of those may be tile idx - 2.
-              if (!pv_done) {
-                issue_pv(idx - 2);
-                pv_done = true;
-                if (!ok) break;
-              }
-              ok = mbar_wait_bounded(b_kvfull + 8 * (use & 1), (use >> 1) & 1, a.st, 0x204u,
-                                     a.wait_ns);
-            }
-            hist = (hist & ~(3u << (2 * (idx & 7)))) | ((uint32_t)(use & 1) << (2 * (idx & 7)));
-            if (ok) ok = mbar_wait_bounded(b_qfull + 8 * qb, (idx / NQ) & 1, a.st, 0x205u, a.wait_ns);
-            // the slot's previous O has been read out
-            if (ok && idx >= NS)
-              ok = mbar_wait_bounded(b_sfree + 8 * sk, ((idx / NS) - 1) & 1, a.st, 0x206u,
-                                     a.wait_ns);
-            if (!ok) break;
+        // Shared-memory descriptors of the first Q tile, the first K stage and the
+        // first V stage; an operand elsewhere is the base plus its byte offset / 16
+        // (the start-address field never carries: shared addresses are < 2^18).
+        const uint64_t dq0 = tc::desc_k_sw128(sq);
+        const uint64_t dk0 = tc::desc_k_sw128(skv);
+        const uint64_t dv0 = tc::desc_mn_sw128(skv + NH * HALF, HALF);
+        int use = -1, nq = 0, np = 0;
+        uint32_t hist = 0, spins = 0;
+        uint64_t stall = 0;
+        bool looked = false, new_block = false;  // tile nq's list, once looked up
+        while (np < n) {
+          bool progress = false;
+          if (np < nq && mbar_test(b_pfull + 8 * (np & 1), (np >> 1) & 1)) {
+            const int p = np & 1, sk = np % NS;
+            const uint32_t h = hist >> (2 * (np & 7));
+            const uint64_t dv = dv0 + (h & 1u) * (KV_BYTES >> 4);
+            const uint32_t pa = tmem + PB + p * (BLK / 2), oa = tmem + sk * W;
             tc::fence_after_sync();
-            const uint32_t kd = skv + (use & 1) * KV_BYTES, qd = sq + qb * QB;
 #pragma unroll
-            for (int ks = 0; ks < D / 16; ++ks) {
-              const uint32_t qoff = (ks >> 2) * (kRows * 128u) + (ks & 3) * 32;
-              const uint32_t koff = (ks >> 2) * HALF + (ks & 3) * 32;
-              tc::mma_bf16(tmem + sk * W, tc::desc_k_sw128(qd + qoff), tc::desc_k_sw128(kd + koff),
-                           id_qk, ks > 0 ? 1u : 0u);
+            for (int ks = 0; ks < BLK / 16; ++ks)
+              tc::mma_bf16_ts(oa, pa + ks * 8, dv + ks * (16 * 128 / 16), id_pv, ks > 0 ? 1u : 0u);
+            tc::commit(b_ofull + 8 * sk);
+            tc::commit(b_pfree + 8 * p);
+            if (h & 2u) tc::commit(b_kvempty + 8 * (h & 1u));  // K/V stage released
+            ++np;
+            progress = true;
+          } else if (nq < n) {
+            const int tile = tile0 + nq;
+            if (!looked) {
+              new_block = w.advance(a, tile) || nq == 0;
+              looked = true;
             }
-            tc::commit(b_sfull + 8 * sk);
-            tc::commit(b_qempty + 8 * qb);  // the Q tile may be refilled
-          } else if (idx == n) {
-            hist |= 2u << (2 * ((n - 1) & 7));  // the last tile ends its block
+            const int u = use + (new_block ? 1 : 0), sk = nq % NS, qb = nq % NQ;
+            bool ready = !new_block || mbar_test(b_kvfull + 8 * (u & 1), (u >> 1) & 1);
+            ready = ready && mbar_test(b_qfull + 8 * qb, (nq / NQ) & 1);
+            // the slot's previous O has been read out
+            ready = ready && (nq < NS || mbar_test(b_sfree + 8 * sk, ((nq / NS) - 1) & 1));
+            if (ready) {
+              use = u;
+              tc::fence_after_sync();
+              const uint64_t dq = dq0 + qb * (QB >> 4), dk = dk0 + (use & 1) * (KV_BYTES >> 4);
+              const uint32_t sa = tmem + sk * W;
+#pragma unroll
+              for (int ks = 0; ks < D / 16; ++ks) {
+                const uint32_t qoff = (ks >> 2) * (kRows * 128u) + (ks & 3) * 32;
+                const uint32_t koff = (ks >> 2) * HALF + (ks & 3) * 32;
+                tc::mma_bf16(sa, dq + (qoff >> 4), dk + (koff >> 4), id_qk, ks > 0 ? 1u : 0u);
+              }
+              tc::commit(b_sfull + 8 * sk);
+              tc::commit(b_qempty + 8 * qb);  // the Q tile may be refilled
+              const bool last = tile + 1 >= w.t1 || nq == n - 1;
+              hist = (hist & ~(3u << (2 * (nq & 7)))) |
+                     (((uint32_t)(use & 1) | (last ? 2u : 0u)) << (2 * (nq & 7)));
+              ++nq;
+              looked = false;
+              progress = true;
+            }
           }
-          if (!pv_done) issue_pv(idx - 2);
+          if (progress) {
+            stall = 0;
+          } else if (stall == 0) {
+            stall = global_timer_ns();
+          } else if ((++spins & 63u) == 0 && global_timer_ns() - stall > a.wait_ns) {
+            record_error(a.st, kErrTimeout, 0x204u);
+            break;
+          }
         }
         tc::commit(b_done);
         mbar_wait_bounded(b_done, 0, a.st, 0x209u, a.wait_ns);
