@@ -50,7 +50,53 @@ __device__ __forceinline__ RowInfo row_info(const TopkArgs& a, int row) {
   return ri;
 }
 
-// One warp per row; element i = e*32 + lane, E elements per lane.
+// Top-m of one row by one warp, element i = e*32 + lane for e < EE: keys in
+// registers, the threshold found bit by bit, ids emitted in order with ballots.
+template <int EE>
+__device__ __forceinline__ void warp_row_topk(const float* s, int32_t* out, const RowInfo& ri,
+                                              int lane) {
+  uint32_t key[EE];
+#pragma unroll
+  for (int e = 0; e < EE; ++e) {
+    const int i = e * 32 + lane;
+    key[e] = i < ri.F ? order_key(s[i]) : 0u;
+    if (i == ri.own) key[e] = 0xffffffffu;
+  }
+  const int m = ri.m;
+  uint32_t T = 0;
+  for (int bit = 31; bit >= 0; --bit) {
+    const uint32_t cand = T | (1u << bit);
+    unsigned cnt = 0;
+#pragma unroll
+    for (int e = 0; e < EE; ++e) cnt += key[e] >= cand;
+    cnt = __reduce_add_sync(0xffffffffu, cnt);
+    if ((int)cnt >= m) T = cand;
+  }
+  unsigned gt = 0;
+#pragma unroll
+  for (int e = 0; e < EE; ++e) gt += key[e] > T;
+  gt = __reduce_add_sync(0xffffffffu, gt);
+  const int need = m - (int)gt;
+  const unsigned lt = (1u << lane) - 1u;
+  int base = 0, eqbase = 0;
+#pragma unroll
+  for (int e = 0; e < EE; ++e) {
+    const bool eq = key[e] == T;
+    const unsigned be = __ballot_sync(0xffffffffu, eq);
+    const int eqr = eqbase + __popc(be & lt);
+    eqbase += __popc(be);
+    const bool sel = key[e] > T || (eq && eqr < need);
+    const unsigned bs = __ballot_sync(0xffffffffu, sel);
+    if (sel) out[base + __popc(bs & lt)] = e * 32 + lane;
+    base += __popc(bs);
+  }
+}
+
+// One warp per row of up to 32 * E blocks.  A row sees only its F blocks at or
+// before the frontier, so it is handled with the smallest power-of-two number
+// of 32-block groups covering F (blocks past F have key 0 and the threshold is
+// at least 1, so leaving them out changes nothing); a row with m = F keeps all
+// of its visible blocks and needs no threshold.
 template <int E>
 __global__ void __launch_bounds__(256) topk_warp_kernel(TopkArgs a) {
   const int lane = threadIdx.x & 31;
@@ -59,42 +105,21 @@ __global__ void __launch_bounds__(256) topk_warp_kernel(TopkArgs a) {
   const RowInfo ri = row_info(a, row);
   const float* s = a.scores + (int64_t)row * a.nblk;
   int32_t* out = a.ids + (int64_t)row * a.topk;
-  uint32_t key[E];
-#pragma unroll
-  for (int e = 0; e < E; ++e) {
-    const int i = e * 32 + lane;
-    key[e] = i < ri.F ? order_key(s[i]) : 0u;
-    if (i == ri.own) key[e] = 0xffffffffu;
-  }
-  const int m = ri.m;
-  if (m > 0) {
-    uint32_t T = 0;
-    for (int bit = 31; bit >= 0; --bit) {
-      const uint32_t cand = T | (1u << bit);
-      unsigned cnt = 0;
-#pragma unroll
-      for (int e = 0; e < E; ++e) cnt += key[e] >= cand;
-      cnt = __reduce_add_sync(0xffffffffu, cnt);
-      if ((int)cnt >= m) T = cand;
-    }
-    unsigned gt = 0;
-#pragma unroll
-    for (int e = 0; e < E; ++e) gt += key[e] > T;
-    gt = __reduce_add_sync(0xffffffffu, gt);
-    const int need = m - (int)gt;
-    const unsigned lt = (1u << lane) - 1u;
-    int base = 0, eqbase = 0;
-#pragma unroll
-    for (int e = 0; e < E; ++e) {
-      const bool eq = key[e] == T;
-      const unsigned be = __ballot_sync(0xffffffffu, eq);
-      const int eqr = eqbase + __popc(be & lt);
-      eqbase += __popc(be);
-      const bool sel = key[e] > T || (eq && eqr < need);
-      const unsigned bs = __ballot_sync(0xffffffffu, sel);
-      if (sel) out[base + __popc(bs & lt)] = e * 32 + lane;
-      base += __popc(bs);
-    }
+  const int m = ri.m, ne = (ri.F + 31) >> 5;
+  if (m == ri.F) {
+    for (int i = lane; i < m; i += 32) out[i] = i;
+  } else if (ne <= 1 || E == 1) {
+    warp_row_topk<1>(s, out, ri, lane);
+  } else if (ne <= 2 || E == 2) {
+    warp_row_topk<(E < 2 ? E : 2)>(s, out, ri, lane);
+  } else if (ne <= 4 || E == 4) {
+    warp_row_topk<(E < 4 ? E : 4)>(s, out, ri, lane);
+  } else if (ne <= 8 || E == 8) {
+    warp_row_topk<(E < 8 ? E : 8)>(s, out, ri, lane);
+  } else if (ne <= 16 || E == 16) {
+    warp_row_topk<(E < 16 ? E : 16)>(s, out, ri, lane);
+  } else {
+    warp_row_topk<E>(s, out, ri, lane);
   }
   for (int i = m + lane; i < a.topk; i += 32) out[i] = -1;
 }
