@@ -595,9 +595,12 @@ __global__ void __launch_bounds__(kKvThreads, 1)
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            const float p0 = exp2_approx(fmaf(v[c * 32 + 2 * e], a.scale_log2, -msafe));
-            const float p1 = exp2_approx(fmaf(v[c * 32 + 2 * e + 1], a.scale_log2, -msafe));
-            l4[e & 3] += p0 + p1;
+            float x0, x1;
+            fma2(x0, x1, v[c * 32 + 2 * e], v[c * 32 + 2 * e + 1], a.scale_log2, a.scale_log2,
+                 -msafe, -msafe);
+            const float p0 = exp2_approx(x0), p1 = exp2_approx(x1);
+            const int h2 = 2 * (e & 1);  // two packed pairs of partial sums
+            add2(l4[h2], l4[h2 + 1], l4[h2], l4[h2 + 1], p0, p1);
             pk[e] = pack_bf16(p0, p1);
           }
           tc::tmem_st16(pr + c * 16, pk);
