@@ -469,6 +469,9 @@ def main():
     ap.add_argument("--seq", type=int, default=0,
                     help="override the sequence length (prefill: queries and context; decode: "
                          "context) for small profiling captures")
+    ap.add_argument("--queries", type=int, default=0,
+                    help="prefill only: keep the context and take the last N positions as the "
+                         "query rows (chunked prefill), for small profiling captures")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -482,6 +485,8 @@ def main():
                               len_range=None if lr is None else (min(lr[0], args.seq), args.seq))
         else:
             prob = prob.with_(n_q=args.seq, max_kv=args.seq)
+    if args.queries and not prob.is_decode:
+        prob = prob.with_(n_q=min(args.queries, prob.max_kv))
     world, rank, local = dist_setup(args)
     try:
         if args.impl == "reference":
