@@ -63,14 +63,33 @@ __device__ __forceinline__ void warp_row_topk(const float* s, int32_t* out, cons
     if (i == ri.own) key[e] = 0xffffffffu;
   }
   const int m = ri.m;
-  uint32_t T = 0;
-  for (int bit = 31; bit >= 0; --bit) {
-    const uint32_t cand = T | (1u << bit);
-    unsigned cnt = 0;
+  // The threshold lies between the smallest and the largest visible key (the
+  // forced block, key 0xffffffff, always counts): it shares their common high
+  // bits, and the search starts below them.
+  uint32_t kmax = 0u, kmin = 0xffffffffu;
 #pragma unroll
-    for (int e = 0; e < EE; ++e) cnt += key[e] >= cand;
-    cnt = __reduce_add_sync(0xffffffffu, cnt);
-    if ((int)cnt >= m) T = cand;
+  for (int e = 0; e < EE; ++e) {
+    const bool vis = key[e] != 0u && key[e] != 0xffffffffu;
+    kmax = vis ? max(kmax, key[e]) : kmax;
+    kmin = vis ? min(kmin, key[e]) : kmin;
+  }
+  kmax = __reduce_max_sync(0xffffffffu, kmax);
+  kmin = __reduce_min_sync(0xffffffffu, kmin);
+  uint32_t T;
+  if (m <= (ri.own >= 0 ? 1 : 0) || kmax < kmin) {
+    T = 0xffffffffu;  // only the forced block is taken
+  } else {
+    const uint32_t diff = kmax ^ kmin;
+    const int top = diff ? 31 - __clz(diff) : -1;
+    T = top < 0 ? kmax : kmax & ~((2u << top) - 1u);
+    for (int bit = top; bit >= 0; --bit) {
+      const uint32_t cand = T | (1u << bit);
+      unsigned c4[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+      for (int e = 0; e < EE; ++e) c4[e & 3] += key[e] >= cand;
+      const unsigned cnt = __reduce_add_sync(0xffffffffu, (c4[0] + c4[1]) + (c4[2] + c4[3]));
+      if ((int)cnt >= m) T = cand;
+    }
   }
   unsigned gt = 0;
 #pragma unroll
