@@ -285,6 +285,38 @@ def workload_config(prob):
 
 
 # ----------------------------------------------------------------- our arm
+def page_cache(prob, x, seed):
+    """Moves k, v and k_idx into page pools of one block per page, the pages of all
+    sequences shuffled over the pool, and adds the block table [batch, nblk]."""
+    B = prob.block
+    nb = (prob.max_kv + B - 1) // B
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    table = torch.randperm(prob.batch * nb, generator=g).to(torch.int32).view(prob.batch, nb)
+    table = table.to(x["k"].device)
+    flat = table.view(-1).long()
+    for name in ("k", "v", "k_idx"):
+        t = x[name]
+        tail = tuple(t.shape[2:])
+        pool = torch.zeros((prob.batch * nb, B) + tail, dtype=t.dtype, device=t.device)
+        for b in range(prob.batch):  # one sequence at a time bounds the extra memory
+            blocks = torch.zeros((nb * B,) + tail, dtype=t.dtype, device=t.device)
+            blocks[:t.shape[1]] = t[b]
+            pool[flat[b * nb:(b + 1) * nb]] = blocks.view((nb, B) + tail)
+            del blocks
+        x[name] = pool
+        del t
+    x["block_table"] = table
+    return x
+
+
+def cache_row(prob, x, name, b, j):
+    """The cache row of token j of sequence b (contiguous or paged)."""
+    if "block_table" not in x:
+        return x[name][b, j]
+    page = int(x["block_table"][b, j // prob.block])
+    return x[name][page, j % prob.block]
+
+
 def run_ours(args, prob, world, rank, local):
     from block_sparse_gqa_03_b200 import msa
 
@@ -292,6 +324,10 @@ def run_ours(args, prob, world, rank, local):
     x = make_inputs(prob, device=dev, seed=prob.seed + rank)
     sl = x["seq_lens"]
     kw = dict(block=prob.block, causal=prob.causal, seq_lens=sl)
+    if args.paged:
+        x = page_cache(prob, x, seed=prob.seed + 7919 + rank)
+        torch.cuda.empty_cache()
+        kw.update(block_table=x["block_table"], max_kv=prob.max_kv)
     ids = torch.empty((prob.batch, prob.n_q, prob.h, prob.topk), dtype=torch.int32, device=dev)
     out = torch.empty_like(x["q"])
     ws = msa.Workspace(dev)
@@ -375,6 +411,8 @@ def run_ours(args, prob, world, rank, local):
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) bf16%s)" % (", planted blocks" if prob.plant_frac else ""),
         "config": {"workload": prob.name, **workload_config(prob),
+                   "kv_cache": "paged (one block per page, shuffled pool)" if args.paged
+                   else "contiguous",
                    "l2": ("inputs larger than L2 (%.2f GB touched per step)" % (touched / 1e9)
                           if touched else "inputs larger than L2"),
                    "parallelism": "replicas" if world > 1 else "single GPU"},
@@ -388,7 +426,7 @@ def run_ours(args, prob, world, rank, local):
         line["tokens_per_s"] = prob.batch * world / (ms_per_step * 1e-3)
     if rank == 0:
         line["clocks"] = clk.summary()
-        if world == 1 and not args.no_cpu_baseline:
+        if world == 1 and not args.no_cpu_baseline and not args.paged:
             import oracle
             u, s, desc = oracle_sample(prob, {k: v for k, v in x.items()}, args.cpu_budget)
             line["cpu_baseline"] = {"value": u / s / scale, "unit": unit,
@@ -408,8 +446,8 @@ def run_e2e(args, prob, x, dev, world, msa, kw):
         host = {n: x[n].cpu().pin_memory() for n in names}
         L = (x["seq_lens"].cpu().tolist() if x["seq_lens"] is not None
              else [prob.max_kv] * prob.batch)
-        rows = {n: torch.stack([x[n][b, L[b] - 1] for b in range(prob.batch)]).cpu().pin_memory()
-                for n in ("k", "v", "k_idx")}
+        rows = {n: torch.stack([cache_row(prob, x, n, b, L[b] - 1) for b in range(prob.batch)])
+                .cpu().pin_memory() for n in ("k", "v", "k_idx")}
         h2d = sum(t.numel() * t.element_size() for t in host.values())
         h2d += sum(t.numel() * t.element_size() for t in rows.values())
     else:
@@ -423,12 +461,14 @@ def run_e2e(args, prob, x, dev, world, msa, kw):
     ws = msa.Workspace(dev)
     nsteps = max(1, min(args.steps, 20))
 
+    dst = {n: [cache_row(prob, x, n, b, L[b] - 1) for b in range(prob.batch)] for n in rows}
+
     def one():
         for n in names:
             x[n].copy_(host[n], non_blocking=True)
         for n, t in rows.items():
             for b in range(prob.batch):
-                x[n][b, L[b] - 1].copy_(t[b], non_blocking=True)
+                dst[n][b].copy_(t[b], non_blocking=True)
         msa.msa_forward(x["q"], x["k"], x["v"], x["q_idx"], x["k_idx"], topk=prob.topk,
                         force_own_block=prob.force_own, out=out_dev, workspace=ws, **kw)
         out_host.copy_(out_dev, non_blocking=True)
@@ -469,6 +509,9 @@ def main():
     ap.add_argument("--seq", type=int, default=0,
                     help="override the sequence length (prefill: queries and context; decode: "
                          "context) for small profiling captures")
+    ap.add_argument("--paged", action="store_true",
+                    help="keep K, V and K_idx in a paged cache (one block per page, pages "
+                         "shuffled over the pool) addressed through a block table")
     ap.add_argument("--queries", type=int, default=0,
                     help="prefill only: keep the context and take the last N positions as the "
                          "query rows (chunked prefill), for small profiling captures")

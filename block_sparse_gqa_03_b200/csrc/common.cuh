@@ -41,6 +41,40 @@ __device__ __forceinline__ int kv_length(const int32_t* seq_lens, int b, int max
   return L;
 }
 
+// Paged K, V and K_idx: table[b * stride + beta] is the pool page holding tokens
+// [beta * block, (beta + 1) * block) of sequence b.  table == nullptr: the tensors
+// are contiguous per sequence.
+struct KvPages {
+  const int32_t* table;
+  int64_t stride, pages;
+};
+
+// The page of block beta of sequence b, or -1 (recorded as a broken precondition)
+// when the table names a page outside the pool.
+__device__ __forceinline__ int64_t kv_page(const KvPages& pg, int b, int beta, DeviceStatus* st) {
+  const int64_t page = __ldg(pg.table + (int64_t)b * pg.stride + beta);
+  if (page < 0 || page >= pg.pages) {
+    record_error(st, kErrDeviceAssert, 0x20000u | (uint32_t)b);
+    return -1;
+  }
+  return page;
+}
+
+// TMA coordinates (token, plane) of the first token of block beta of sequence b:
+// [beta * block, b] in contiguous tensors, [0, page] in a page pool.  A bad page
+// gives the plane just past the pool, which a TMA load reads as zeros.
+__device__ __forceinline__ void kv_block_coords(const KvPages& pg, int b, int beta, int block,
+                                                DeviceStatus* st, int& tok, int& plane) {
+  if (pg.table == nullptr) {
+    tok = beta * block;
+    plane = b;
+    return;
+  }
+  const int64_t page = kv_page(pg, b, beta, st);
+  tok = 0;
+  plane = page < 0 ? (int)pg.pages : (int)page;
+}
+
 // True once any kernel sharing this status word has recorded an error; kernels
 // check it on entry so that a failure is not repeated by every later CTA.
 __device__ __forceinline__ bool status_failed(const DeviceStatus* st) {

@@ -30,9 +30,19 @@ struct ScanArgs {
   float* scores;
   int fill_tail;
   DeviceStatus* st;
+  KvPages pg;
 };
 
 constexpr int kScanWarps = 8;
+
+// k_idx row of the first token of block beta of sequence b, offset by this lane's
+// 8 dims; nullptr for a page outside the pool (the block then reads as zeros).
+__device__ __forceinline__ const uint16_t* kidx_block(const ScanArgs& a, int b, int beta, int q) {
+  if (a.pg.table == nullptr)
+    return a.k_idx + b * a.ki_s0 + (int64_t)beta * a.block * a.ki_s1 + 8 * q;
+  const int64_t page = kv_page(a.pg, b, beta, a.st);
+  return page < 0 ? nullptr : a.k_idx + page * a.ki_s0 + 8 * q;
+}
 
 // Loads the B fragments (index-query columns) of this lane: column c = nt*8 + r,
 // dims [32kc + 8q, 32kc + 8q + 8).  Columns past `ncols` or t >= n_q are zero.
@@ -55,8 +65,9 @@ __device__ __forceinline__ void load_columns(const ScanArgs& a, int b, int t0, i
 // Block max of the visible token scores of block `beta` for this lane's
 // accumulator columns (c = nt*8 + 2q + e, visible tokens j < lim[nt][e]),
 // reduced over the warp: every lane returns the maxima of its own columns.
+// `kbb` is the block's first k_idx row (kidx_block).
 template <int DI, int NT>
-__device__ __forceinline__ void block_max(const ScanArgs& a, const uint16_t* kb, int L, int beta,
+__device__ __forceinline__ void block_max(const ScanArgs& a, const uint16_t* kbb, int L, int beta,
                                           int r, const uint4 (&bq)[NT][DI / 32],
                                           const int (&lim)[NT][2], float (&cm)[NT][2]) {
   constexpr int KC = DI / 32;
@@ -66,12 +77,14 @@ __device__ __forceinline__ void block_max(const ScanArgs& a, const uint16_t* kb,
   const int nmt = a.block / 16;
 #pragma unroll 2
   for (int mt = 0; mt < nmt; ++mt) {
-    const int jl = beta * a.block + mt * 16 + r, jh = jl + 8;
+    const int ol = mt * 16 + r, oh = ol + 8;  // tokens in the block
+    const int jl = beta * a.block + ol, jh = jl + 8;
+    const bool okl = kbb != nullptr && jl < L, okh = kbb != nullptr && jh < L;
     uint4 X[KC], Y[KC];
 #pragma unroll
     for (int kc = 0; kc < KC; ++kc) {
-      X[kc] = jl < L ? ld_stream_u4(kb + (int64_t)jl * a.ki_s1 + 32 * kc) : make_uint4(0, 0, 0, 0);
-      Y[kc] = jh < L ? ld_stream_u4(kb + (int64_t)jh * a.ki_s1 + 32 * kc) : make_uint4(0, 0, 0, 0);
+      X[kc] = okl ? ld_stream_u4(kbb + (int64_t)ol * a.ki_s1 + 32 * kc) : make_uint4(0, 0, 0, 0);
+      Y[kc] = okh ? ld_stream_u4(kbb + (int64_t)oh * a.ki_s1 + 32 * kc) : make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
@@ -117,13 +130,14 @@ __global__ void __launch_bounds__(kScanWarps * 32) index_scan_decode_kernel(Scan
     if (a.fill_tail && lane < a.h) a.scores[((int64_t)b * a.h + lane) * a.nblk + beta] = ninf;
     return;
   }
+  const uint16_t* kbb = kidx_block(a, b, beta, q);  // the page lookup overlaps the q loads
   uint4 bq[NT][DI / 32];
   load_columns<DI, NT>(a, b, 0, r, q, bq);
   int lim[NT][2];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) lim[nt][0] = lim[nt][1] = L;  // p = L - 1: all j < L visible
   float cm[NT][2];
-  block_max<DI, NT>(a, a.k_idx + b * a.ki_s0 + 8 * q, L, beta, r, bq, lim, cm);
+  block_max<DI, NT>(a, kbb, L, beta, r, bq, lim, cm);
   if (r == 0) {
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
@@ -164,11 +178,10 @@ __global__ void __launch_bounds__(kScanWarps * 32) index_scan_kernel(ScanArgs a)
   const int F = a.causal ? (p_last < 0 ? 0 : min(nb_b, p_last / a.block + 1)) : nb_b;
   const int nw = gridDim.y * kScanWarps;
   const int wid = blockIdx.y * kScanWarps + warp;
-  const uint16_t* kb = a.k_idx + b * a.ki_s0 + 8 * q;
   const float ninf = -__int_as_float(0x7f800000);
   for (int beta = wid; beta < F; beta += nw) {
     float cm[NT][2];
-    block_max<DI, NT>(a, kb, L, beta, r, bq, lim, cm);
+    block_max<DI, NT>(a, kidx_block(a, b, beta, q), L, beta, r, bq, lim, cm);
     if (r == 0) {
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt)
@@ -229,6 +242,7 @@ cudaError_t launch_index_scores(const Shape& s, const uint16_t* q_idx, const uin
   a.qi_s2 = s.qi_s[2];
   a.ki_s0 = s.ki_s[0];
   a.ki_s1 = s.ki_s[1];
+  a.pg = s.pages;
   a.seq_lens = s.seq_lens;
   a.batch = s.batch;
   a.n_q = s.n_q;

@@ -39,6 +39,7 @@ struct TcArgs {
   int fill_tail;
   DeviceStatus* st;
   uint64_t wait_ns;
+  KvPages pg;  // table == nullptr: contiguous K_idx
 };
 
 template <int DI, int BLK>
@@ -119,10 +120,25 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                                a.wait_ns))
           break;
         mbar_arrive_expect_tx(b_kfull + 8 * s, K_BYTES);
+        if (a.pg.table == nullptr) {
 #pragma unroll
-        for (int at = 0; at < NATOM; ++at)
-          tma_load_3d(k_base + s * K_BYTES + at * ATOM, &tmk, b_kfull + 8 * s, at * 64, kt * kKT,
-                      b);
+          for (int at = 0; at < NATOM; ++at)
+            tma_load_3d(k_base + s * K_BYTES + at * ATOM, &tmk, b_kfull + 8 * s, at * 64,
+                        kt * kKT, b);
+        } else {
+          // one box per page of BLK tokens; blocks past the sequence end are not
+          // looked up and read as zeros (their keys are masked anyway)
+          const int nb_b = (L + BLK - 1) / BLK;
+          for (int pi = 0; pi < kKT / BLK; ++pi) {
+            const int beta = kt * (kKT / BLK) + pi;
+            const int64_t page = beta < nb_b ? kv_page(a.pg, b, beta, a.st) : -1;
+            const int plane = page < 0 ? (int)a.pg.pages : (int)page;
+#pragma unroll
+            for (int at = 0; at < NATOM; ++at)
+              tma_load_3d(k_base + s * K_BYTES + at * ATOM + pi * BLK * 128u, &tmk,
+                          b_kfull + 8 * s, at * 64, 0, plane);
+          }
+        }
         ++issued;
       }
       // Drain: the last stages are released by the MMA commits, i.e. after their
@@ -256,9 +272,13 @@ cudaError_t run_tc(const Shape& s, const uint16_t* q_idx, const uint16_t* k_idx,
       return cudaErrorInvalidValue;
   }
   {
-    cuuint64_t dims[3] = {(cuuint64_t)s.d_idx, (cuuint64_t)s.max_kv, (cuuint64_t)s.batch};
+    // contiguous [d_idx, token, batch] with 128-token boxes, or a page pool
+    // [d_idx, token in page, page] with one-page boxes
+    const bool paged = s.pages.table != nullptr;
+    cuuint64_t dims[3] = {(cuuint64_t)s.d_idx, (cuuint64_t)(paged ? BLK : s.max_kv),
+                          (cuuint64_t)(paged ? s.pages.pages : s.batch)};
     cuuint64_t str[2] = {(cuuint64_t)s.ki_s[1] * 2, (cuuint64_t)s.ki_s[0] * 2};
-    cuuint32_t box[3] = {64, (cuuint32_t)kKT, 1};
+    cuuint32_t box[3] = {64, (cuuint32_t)(paged ? BLK : kKT), 1};
     cuuint32_t es[3] = {1, 1, 1};
     if (enc(&tmk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<uint16_t*>(k_idx), dims, str,
             box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -300,6 +320,7 @@ cudaError_t launch_index_scores_tc(const Shape& s, const uint16_t* q_idx, const 
   a.fill_tail = fill_tail ? 1 : 0;
   a.st = st;
   a.wait_ns = 4000000000ull;
+  a.pg = s.pages;
 #define MSA_TC_CASE(DI_, BLK_) \
   if (s.d_idx == DI_ && s.block == BLK_) return run_tc<DI_, BLK_>(s, q_idx, k_idx, a, stream);
   MSA_TC_CASE(128, 16)

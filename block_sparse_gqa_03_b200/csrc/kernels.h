@@ -16,6 +16,7 @@ struct Shape {
   float scale;
   const int32_t* seq_lens;
   int64_t q_s[3], k_s[3], v_s[3], qi_s[3], ki_s[2], o_s[3];
+  KvPages pages;  // table == nullptr: contiguous K/V/K_idx
 };
 
 // Stage 1a/1b: block-max-pooled index scores, fp32 [batch, n_q, h, nblk].

@@ -97,6 +97,15 @@ msa_status_t make_shape(const msa_params_t* p, Shape* s) {
   }
   s->ki_s[0] = p->ki_strides[0];
   s->ki_s[1] = p->ki_strides[1];
+  s->pages.table = p->block_table;
+  s->pages.stride = p->table_stride;
+  s->pages.pages = p->num_pages;
+  if (p->block_table != nullptr) {
+    // one page per block; page coordinates are int32 in the tensor maps
+    if ((reinterpret_cast<uintptr_t>(p->block_table) & 3u) != 0 || p->table_stride < nblk ||
+        p->num_pages < 1 || p->num_pages > (int64_t)INT32_MAX - 1)
+      return MSA_ERR_INVALID_ARG;
+  }
   return MSA_OK;
 }
 

@@ -54,6 +54,7 @@ struct AttnArgs {
   float* lse;
   DeviceStatus* st;
   uint64_t wait_ns;
+  KvPages pg;  // table == nullptr: contiguous K/V
 };
 
 constexpr float kLn2 = 0.69314718055994531f;
@@ -259,15 +260,33 @@ __device__ __forceinline__ void consumer_sync(int nthreads) {
 // the producer waits for its copies still in flight.
 template <int D>
 __device__ __forceinline__ void produce(const AttnArgs& a, const CUtensorMap* tmk,
-                                        const CUtensorMap* tmv, const int32_t* list, int n,
-                                        int64_t row0, uint32_t sbase, uint32_t full0,
-                                        uint32_t empty0) {
+                                        const CUtensorMap* tmv, const int32_t* list,
+                                        const int32_t* plist, int n, int64_t row0,
+                                        uint32_t sbase, uint32_t full0, uint32_t empty0) {
   constexpr int NH = D / 64;
   const uint32_t half_bytes = (uint32_t)a.block * 128u;
   prefetch_tensormap(tmk);
   prefetch_tensormap(tmv);
+  // (head, token, plane) of entry i; a paged cache's pages were looked up when the
+  // list was built (plist, -1 for a page outside the pool)
+  auto coords = [&](int i, int& g, int& tok, int& plane) {
+    const int e = list[i];
+    const int64_t rowg = row0 + (e >> 16);
+    g = (int)(rowg % a.h);
+    if (a.pg.table == nullptr) {
+      tok = (e & 0xffff) * a.block;
+      plane = (int)(rowg / a.h) / a.n_q;
+    } else {
+      tok = 0;
+      plane = plist[i] < 0 ? (int)a.pg.pages : plist[i];
+    }
+  };
+  int g_n = 0, tok_n = 0, plane_n = 0;
+  if (n > 0) coords(0, g_n, tok_n, plane_n);
   int issued = 0;
   for (int i = 0; i < n; ++i) {
+    const int g = g_n, tok = tok_n, plane = plane_n;
+    if (i + 1 < n) coords(i + 1, g_n, tok_n, plane_n);
     const int s = i % a.stages;
     if (i >= a.stages &&
         !mbar_wait_bounded(empty0 + 8 * s, ((i / a.stages) - 1) & 1, a.st, 1u, a.wait_ns))
@@ -276,15 +295,10 @@ __device__ __forceinline__ void produce(const AttnArgs& a, const CUtensorMap* tm
     mbar_arrive_expect_tx(full, a.stage_bytes);
     const uint32_t kdst = sbase + (uint32_t)s * a.stage_bytes;
     const uint32_t vdst = kdst + NH * half_bytes;
-    const int e = list[i];
-    const int64_t rowg = row0 + (e >> 16);
-    const int g = (int)(rowg % a.h);
-    const int b = (int)(rowg / a.h) / a.n_q;
-    const int tok = (e & 0xffff) * a.block;
 #pragma unroll
     for (int hh = 0; hh < NH; ++hh) {
-      tma_load_4d(kdst + hh * half_bytes, tmk, full, hh * 64, g, tok, b);
-      tma_load_4d(vdst + hh * half_bytes, tmv, full, hh * 64, g, tok, b);
+      tma_load_4d(kdst + hh * half_bytes, tmk, full, hh * 64, g, tok, plane);
+      tma_load_4d(vdst + hh * half_bytes, tmv, full, hh * 64, g, tok, plane);
     }
     ++issued;
   }
@@ -293,9 +307,12 @@ __device__ __forceinline__ void produce(const AttnArgs& a, const CUtensorMap* tm
 }
 
 // Compacts slots [s0, s1) of the flattened id array into the entry list: only
-// blocks holding a visible token are kept.  Run by one full warp; returns the count.
+// blocks holding a visible token are kept, and with a paged cache each kept
+// block's page goes to plist (the lanes look their pages up in parallel).  Run
+// by one full warp; returns the count.
 __device__ __forceinline__ int compact_ids(const AttnArgs& a, int64_t s0, int64_t s1,
-                                           int64_t row0, int32_t* list, int lane) {
+                                           int64_t row0, int32_t* list, int32_t* plist,
+                                           int lane) {
   const unsigned lt = (1u << lane) - 1u;
   int n = 0;
   int64_t cached_row = -1;
@@ -316,7 +333,11 @@ __device__ __forceinline__ int compact_ids(const AttnArgs& a, int64_t s0, int64_
     if (bad) record_error(a.st, kErrDeviceAssert, (uint32_t)rowg);
     const bool keep = beta >= 0 && !bad && (int64_t)beta * a.block < lim;
     const unsigned msk = __ballot_sync(0xffffffffu, keep);
-    if (keep) list[n + __popc(msk & lt)] = beta | (int)((rowg - row0) << 16);
+    if (keep) {
+      const int at = n + __popc(msk & lt);
+      list[at] = beta | (int)((rowg - row0) << 16);
+      if (a.pg.table != nullptr) plist[at] = (int)kv_page(a.pg, (int)(rowg / a.h) / a.n_q, beta, a.st);
+    }
     n += __popc(msk);
   }
   return n;
@@ -336,6 +357,7 @@ __global__ void __launch_bounds__(5 * 32, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + a.region_bytes);
   int32_t* list = reinterpret_cast<int32_t*>(bars + 2 * a.stages);
   int32_t* n_list = list + a.list_cap;
+  int32_t* plist = n_list + 1;  // [list_cap] pages, paged cache only
   const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + a.stages);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t rowg = blockIdx.x;
@@ -350,13 +372,13 @@ __global__ void __launch_bounds__(5 * 32, 1)
     fence_mbar_init();
   }
   if (warp == NC) {
-    const int n = compact_ids(a, rowg * a.topk, (rowg + 1) * a.topk, rowg, list, lane);
+    const int n = compact_ids(a, rowg * a.topk, (rowg + 1) * a.topk, rowg, list, plist, lane);
     if (lane == 0) *n_list = n;
   }
   __syncthreads();
   const int n = *n_list;
   if (warp == NC) {
-    if (lane == 0 && n > 0) produce<D>(a, &tmk, &tmv, list, n, rowg, sbase, full0, empty0);
+    if (lane == 0 && n > 0) produce<D>(a, &tmk, &tmv, list, plist, n, rowg, sbase, full0, empty0);
     return;
   }
   const RowGeo rg = row_geo(a, rowg);
@@ -416,6 +438,7 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + a.region_bytes);
   int32_t* list = reinterpret_cast<int32_t*>(bars + 2 * a.stages);
   int32_t* n_list = list + a.list_cap;
+  int32_t* plist = n_list + 1;  // [list_cap] pages, paged cache only
   const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + a.stages);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nsub = a.block / 16;
@@ -434,13 +457,13 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1)
     fence_mbar_init();
   }
   if (warp == NC) {
-    const int n = compact_ids(a, s0, s1, r0, list, lane);
+    const int n = compact_ids(a, s0, s1, r0, list, plist, lane);
     if (lane == 0) *n_list = n;
   }
   __syncthreads();
   const int n = *n_list;
   if (warp == NC) {
-    if (lane == 0 && n > 0) produce<D>(a, &tmk, &tmv, list, n, r0, sbase, full0, empty0);
+    if (lane == 0 && n > 0) produce<D>(a, &tmk, &tmv, list, plist, n, r0, sbase, full0, empty0);
     return;
   }
 
@@ -570,13 +593,16 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// K or V as a 4-D tensor [batch][token][kv head][dim]; one box is 64 dims x 1
-// head x `block` tokens (128 bytes per row, 128-byte swizzle).
+// K or V as a 4-D tensor [batch][token][kv head][dim], or for a paged cache
+// [page][token in page][kv head][dim]; one box is 64 dims x 1 head x `block`
+// tokens (128 bytes per row, 128-byte swizzle).
 bool make_kv_map(CUtensorMap* map, const uint16_t* base, const Shape& s, const int64_t* str) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
-  cuuint64_t dims[4] = {(cuuint64_t)s.d, (cuuint64_t)s.h, (cuuint64_t)s.max_kv,
-                        (cuuint64_t)s.batch};
+  const bool paged = s.pages.table != nullptr;
+  cuuint64_t dims[4] = {(cuuint64_t)s.d, (cuuint64_t)s.h,
+                        (cuuint64_t)(paged ? s.block : s.max_kv),
+                        (cuuint64_t)(paged ? s.pages.pages : s.batch)};
   cuuint64_t strides[3] = {(cuuint64_t)str[2] * 2, (cuuint64_t)str[1] * 2,
                            (cuuint64_t)str[0] * 2};
   cuuint32_t box[4] = {64, 1, (cuuint32_t)s.block, 1};
@@ -658,7 +684,8 @@ AttnPlan plan_attn(const Shape& s) {
     pl.smax = 1;
     pl.list_cap = s.topk;
   }
-  pl.smem_bytes = 1024 + pl.region_bytes + 16 * pl.stages + 4 * (pl.list_cap + 1);
+  pl.smem_bytes = 1024 + pl.region_bytes + 16 * pl.stages + 4 * (pl.list_cap + 1) +
+                  (s.pages.table != nullptr ? 4 * (size_t)pl.list_cap : 0);
   return pl;
 }
 
@@ -733,6 +760,7 @@ cudaError_t launch_sparse_attn(const Shape& s, const uint16_t* q, const uint16_t
   a.lse = lse;
   a.st = st;
   a.wait_ns = 4000000000ull;  // 4 s: far above any healthy wait, even under a profiler
+  a.pg = s.pages;
   cudaError_t err;
   if (!pl.stream && kv_attn_supported(s)) {
     CUtensorMap tmq;

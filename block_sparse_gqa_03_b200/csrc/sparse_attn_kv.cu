@@ -82,6 +82,7 @@ struct KvArgs {
   float* lse;
   DeviceStatus* st;
   uint64_t wait_ns;
+  KvPages pg;  // table == nullptr: contiguous K/V
 };
 
 __device__ __forceinline__ int visible_from_length(const KvArgs& a, int L, int t) {
@@ -373,11 +374,13 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         const uint32_t bar = (fix ? b_kvland : b_kvfull) + 8 * s;
         const uint32_t kd = skv + s * KV_BYTES, vd = kd + NH * HALF;
         if (lane == 0) {
+          int tok, plane;
+          kv_block_coords(a.pg, w.b, w.beta, BLK, a.st, tok, plane);
           mbar_arrive_expect_tx(bar, KV_BYTES);
 #pragma unroll
           for (int hh = 0; hh < NH; ++hh) {
-            tma_load_4d(kd + hh * HALF, &tmk, bar, hh * 64, w.g, w.beta * BLK, w.b);
-            tma_load_4d(vd + hh * HALF, &tmv, bar, hh * 64, w.g, w.beta * BLK, w.b);
+            tma_load_4d(kd + hh * HALF, &tmk, bar, hh * 64, w.g, tok, plane);
+            tma_load_4d(vd + hh * HALF, &tmv, bar, hh * 64, w.g, tok, plane);
           }
         }
         if (fix) {
@@ -926,6 +929,7 @@ cudaError_t launch_kv_attn(const Shape& s, const CUtensorMap& tmq, const CUtenso
   a.lse = lse;
   a.st = st;
   a.wait_ns = 4000000000ull;
+  a.pg = s.pages;
   CUtensorMap tmo;
   if (!make_rows_map(&tmo, a.part_o, p.max_tiles * kRows, s.d)) return cudaErrorInvalidValue;
   if (s.d == 128 && s.block == 128) return run_kv<128, 128>(s, a, p, tmq, tmk, tmv, tmo, w, stream);

@@ -58,6 +58,9 @@ class Params(ctypes.Structure):
         ("qi_strides", ctypes.c_int64 * 3),
         ("ki_strides", ctypes.c_int64 * 2),
         ("o_strides", ctypes.c_int64 * 3),
+        ("block_table", ctypes.c_void_p),
+        ("table_stride", ctypes.c_int64),
+        ("num_pages", ctypes.c_int64),
     ]
 
 
@@ -120,7 +123,10 @@ def _outer(t: torch.Tensor, n: int):
 
 def make_params(*, batch, n_q, max_kv, H, h, d, d_idx, block, topk, causal=True,
                 force_own_block=False, softmax_scale=0.0, seq_lens=None, q=None, k=None, v=None,
-                q_idx=None, k_idx=None, out=None) -> Params:
+                q_idx=None, k_idx=None, out=None, block_table=None, num_pages=0) -> Params:
+    """With ``block_table`` (int32 [batch, table_stride]) k, v and k_idx are page pools
+    ([num_pages, block, h, d] and [num_pages, block, d_idx]) and their strides are
+    taken over (page, token in page, head)."""
     p = Params()
     p.batch, p.n_q, p.max_kv, p.H, p.h = batch, n_q, max_kv, H, h
     p.d, p.d_idx, p.block, p.topk = d, d_idx, block, topk
@@ -139,6 +145,10 @@ def make_params(*, batch, n_q, max_kv, H, h, d, d_idx, block, topk, causal=True,
         p.ki_strides[:] = _outer(k_idx, 2)
     if out is not None:
         p.o_strides[:] = _outer(out, 3)
+    if block_table is not None:
+        p.block_table = _ptr(block_table)
+        p.table_stride = block_table.stride(0)
+        p.num_pages = int(num_pages)
     return p
 
 
@@ -197,16 +207,29 @@ def _check(rc: int, what: str):
         raise MsaError(rc, what)
 
 
+def _kv_extent(k, block_table, max_kv):
+    """max_kv and the page count: the tensor's token axis, or for a page pool the
+    caller's max_kv and the pool's first axis."""
+    if block_table is None:
+        return k.shape[1], 0
+    if max_kv is None:
+        raise ValueError("a paged KV cache needs max_kv")
+    return int(max_kv), k.shape[0]
+
+
 def msa_index_select(q_idx, k_idx, *, block, topk, causal=True, force_own_block=False,
                      seq_lens=None, return_scores=False, block_ids=None, block_scores=None,
-                     workspace: Workspace | None = None, stream=None):
-    """Stage 1: block ids int32 [b, n_q, h, topk] (and fp32 block scores if asked)."""
+                     block_table=None, max_kv=None, workspace: Workspace | None = None,
+                     stream=None):
+    """Stage 1: block ids int32 [b, n_q, h, topk] (and fp32 block scores if asked).
+    With ``block_table``, ``k_idx`` is a page pool [num_pages, block, d_idx]."""
     b, n_q, h, d_idx = q_idx.shape
-    max_kv = k_idx.shape[1]
+    max_kv, num_pages = _kv_extent(k_idx, block_table, max_kv)
     nblk = (max_kv + block - 1) // block
     p = make_params(batch=b, n_q=n_q, max_kv=max_kv, H=h, h=h, d=64, d_idx=d_idx, block=block,
                     topk=topk, causal=causal, force_own_block=force_own_block,
-                    seq_lens=seq_lens, q_idx=q_idx, k_idx=k_idx)
+                    seq_lens=seq_lens, q_idx=q_idx, k_idx=k_idx, block_table=block_table,
+                    num_pages=num_pages)
     dev = q_idx.device
     if block_ids is None:
         block_ids = torch.empty((b, n_q, h, topk), dtype=torch.int32, device=dev)
@@ -223,11 +246,13 @@ def msa_index_select(q_idx, k_idx, *, block, topk, causal=True, force_own_block=
 
 
 def msa_sparse_attn(q, k, v, block_ids, *, block, causal=True, seq_lens=None, softmax_scale=0.0,
-                    return_lse=False, out=None, lse=None, workspace: Workspace | None = None,
-                    stream=None):
-    """Stage 2: bf16 output [b, n_q, H, d] (and fp32 lse [b, n_q, H] if asked)."""
+                    return_lse=False, out=None, lse=None, block_table=None, max_kv=None,
+                    workspace: Workspace | None = None, stream=None):
+    """Stage 2: bf16 output [b, n_q, H, d] (and fp32 lse [b, n_q, H] if asked).
+    With ``block_table``, ``k`` and ``v`` are page pools [num_pages, block, h, d]."""
     b, n_q, H, d = q.shape
-    max_kv, h = k.shape[1], k.shape[2]
+    h = k.shape[2]
+    max_kv, num_pages = _kv_extent(k, block_table, max_kv)
     topk = block_ids.shape[-1]
     if out is None:
         out = torch.empty_like(q)
@@ -235,7 +260,7 @@ def msa_sparse_attn(q, k, v, block_ids, *, block, causal=True, seq_lens=None, so
         lse = torch.empty((b, n_q, H), dtype=torch.float32, device=q.device)
     p = make_params(batch=b, n_q=n_q, max_kv=max_kv, H=H, h=h, d=d, d_idx=32, block=block,
                     topk=topk, causal=causal, softmax_scale=softmax_scale, seq_lens=seq_lens,
-                    q=q, k=k, v=v, out=out)
+                    q=q, k=k, v=v, out=out, block_table=block_table, num_pages=num_pages)
     need = msa_workspace_size(p, MSA_OP_SPARSE_ATTN)
     if need == 0:
         raise MsaError(MSA_ERR_INVALID_ARG, "msa_workspace_size")
@@ -267,10 +292,13 @@ def msa_sparse_attn_noalloc(q, k, v, block_ids, *, block, causal=True, seq_lens=
 def msa_forward(q, k, v, q_idx, k_idx, *, block, topk, causal=True, force_own_block=False,
                 seq_lens=None, softmax_scale=0.0, out=None, block_ids=None, block_scores=None,
                 lse=None, return_ids=False, return_scores=False, return_lse=False,
-                workspace: Workspace | None = None, stream=None, params: Params | None = None):
-    """Both stages; returns out, plus (ids, scores, lse) when asked, in that order."""
+                block_table=None, max_kv=None, workspace: Workspace | None = None, stream=None,
+                params: Params | None = None):
+    """Both stages; returns out, plus (ids, scores, lse) when asked, in that order.
+    With ``block_table``, ``k``, ``v`` and ``k_idx`` are page pools."""
     b, n_q, H, d = q.shape
-    max_kv, h = k.shape[1], k.shape[2]
+    h = k.shape[2]
+    max_kv, num_pages = _kv_extent(k, block_table, max_kv)
     d_idx = q_idx.shape[-1]
     nblk = (max_kv + block - 1) // block
     dev = q.device
@@ -285,7 +313,8 @@ def msa_forward(q, k, v, q_idx, k_idx, *, block, topk, causal=True, force_own_bl
     p = params or make_params(batch=b, n_q=n_q, max_kv=max_kv, H=H, h=h, d=d, d_idx=d_idx,
                               block=block, topk=topk, causal=causal,
                               force_own_block=force_own_block, softmax_scale=softmax_scale,
-                              seq_lens=seq_lens, q=q, k=k, v=v, q_idx=q_idx, k_idx=k_idx, out=out)
+                              seq_lens=seq_lens, q=q, k=k, v=v, q_idx=q_idx, k_idx=k_idx, out=out,
+                              block_table=block_table, num_pages=num_pages)
     need = msa_workspace_size(p, MSA_OP_FORWARD)
     if need == 0:
         raise MsaError(MSA_ERR_INVALID_ARG, "msa_workspace_size")

@@ -33,6 +33,17 @@
  *   block_scores fp32  [batch, n_q, h, nblk]   dense, row-major
  *   lse          fp32  [batch, n_q, H]         dense, row-major (natural log)
  *
+ * Paged KV cache (optional; block_table != NULL): k, v and k_idx are pools of
+ * pages of `block` tokens each,
+ *   k, v   bf16 [num_pages, block, h, d]    k_idx  bf16 [num_pages, block, d_idx]
+ * with k/v_strides = [page, token in page, kv head] and ki_strides = [page, token
+ * in page], and block_table (device int32 [batch, table_stride]) gives the page of
+ * each logical block: block_table[b * table_stride + beta] holds tokens
+ * [beta * block, (beta + 1) * block) of sequence b.  Only rows beta <
+ * ceil(L_b / block) are read, so table_stride >= ceil(max_kv / block).  A page
+ * id outside [0, num_pages) is recorded as MSA_ERR_DEVICE_ASSERT and that block
+ * reads as zeros.  Results are the same as with the contiguous layout.
+ *
  * Supported sizes: d in {64, 128}; d_idx in {32, 64, 128}; block in {16, 32, 64,
  * 128}; 1 <= G <= 16; 1 <= topk <= 4096; h <= 16; n_q <= max_kv; all base pointers
  * 16-byte aligned and every outer stride a multiple of 8 elements.  Anything else
@@ -96,6 +107,10 @@ typedef struct msa_params {
   int64_t qi_strides[3];   /* q_idx: [b, t, group] */
   int64_t ki_strides[2];   /* k_idx: [b, token] */
   int64_t o_strides[3];    /* out:   [b, t, head] */
+  /* paged K/V/K_idx (see above); block_table NULL means contiguous tensors */
+  const int32_t* block_table; /* device [batch, table_stride] */
+  int64_t table_stride;       /* entries per sequence row of block_table */
+  int64_t num_pages;          /* pages in each of the k, v and k_idx pools */
 } msa_params_t;
 
 /* Bytes of workspace `op` needs for these shapes (0 on invalid params).  The

@@ -106,6 +106,22 @@ def test_bad_pointers_and_workspace_rejected(lib):
     assert lib.msa_selftest_wait_timeout(fake, 4096, 0, None) == msa.MSA_ERR_INVALID_ARG
 
 
+def test_paged_params_validated(lib):
+    p = valid_params()
+    assert msa.msa_workspace_size(p, msa.MSA_OP_FORWARD) > 0
+    fake = 1 << 20
+    p.block_table, p.num_pages = fake, 64
+    p.table_stride = 16  # = ceil(1024 / 64) blocks per sequence
+    assert msa.msa_workspace_size(p, msa.MSA_OP_FORWARD) > 0
+    p.table_stride = 15  # too short for max_kv
+    assert msa.msa_workspace_size(p, msa.MSA_OP_FORWARD) == 0
+    p.table_stride, p.num_pages = 16, 0  # empty pool
+    assert msa.msa_workspace_size(p, msa.MSA_OP_FORWARD) == 0
+    p.num_pages, p.block_table = 64, fake + 2  # misaligned table
+    assert lib.msa_forward(ctypes.byref(p), fake, fake, fake, fake, fake, fake, None, None, None,
+                           fake, 1 << 30, None) == msa.MSA_ERR_INVALID_ARG
+
+
 def test_binding_fails_loudly_without_library(monkeypatch):
     monkeypatch.setattr(msa, "LIB_PATH", "/nonexistent/libmsa.so")
     monkeypatch.setattr(msa, "_lib", None)
