@@ -14,8 +14,10 @@
 //   warp 0     TMA producer (query tiles once, then the key ring);
 //   warp 1     tensor-memory allocation, and one thread issuing the MMAs
 //              (M = 128 queries, N = 128 keys, K = 16 per instruction);
-//   warps 2-5  epilogue: each owns 32 tensor-memory lanes (= 32 query rows),
-//              masks invisible keys, takes the block maxima, stores them.
+//   warps 2-9  epilogue: one warp per (group, 32 tensor-memory lanes = 32
+//              query rows); masks invisible keys, takes the block maxima,
+//              stores them.  Tiles wholly below the causal frontier skip the
+//              mask.
 // Accumulators are double-buffered (2 x 2 groups x 128 columns = 512 columns), so
 // the epilogue of one key tile overlaps the MMAs of the next.  Every mbarrier wait
 // is bounded and records an error instead of hanging.
@@ -28,7 +30,7 @@ namespace {
 constexpr int kQT = 128;  // queries per tile (MMA M, tensor-memory lanes)
 constexpr int kKT = 128;  // keys per tile (MMA N)
 constexpr int kNG = 2;    // groups per CTA
-constexpr int kTcThreads = 6 * 32;
+constexpr int kTcThreads = (2 + 4 * kNG) * 32;
 constexpr uint32_t kTmemCols = 512;
 
 struct TcArgs {
@@ -87,7 +89,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(b_afull + 8 * i, 1);
-      mbar_init(b_aempty + 8 * i, 4);
+      mbar_init(b_aempty + 8 * i, 4 * ng_valid);
     }
     mbar_init(b_done, 1);
     fence_mbar_init();
@@ -179,6 +181,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   } else {
     // ------------------------------------------------------------ epilogue
     const int quarter = warp & 3;  // tensor-memory lanes [32q, 32q + 32)
+    const int ng = (warp - 2) >> 2;  // this warp's group of the pair
     const int row = quarter * 32 + lane;
     const int t = t0 + row;
     const bool row_ok = t < a.n_q;
@@ -187,45 +190,48 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     constexpr int bpt = kKT / BLK;  // blocks per key tile
     const float ninf = -__int_as_float(0x7f800000);
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
-    float* srow = a.scores + ((int64_t)b * a.n_q + t) * a.h * (int64_t)a.nblk;
-    for (int kt = 0; kt < n_kt; ++kt) {
+    float* srow = a.scores + (((int64_t)b * a.n_q + t) * a.h + gp * kNG + ng) * (int64_t)a.nblk;
+    for (int kt = 0; kt < n_kt && ng < ng_valid; ++kt) {
       const int buf = kt & 1;
       if (!mbar_wait_warp(b_afull + 8 * buf, (kt >> 1) & 1, a.st, 0x106u, a.wait_ns)) break;
       tc::fence_after_sync();
       const int j0 = kt * kKT;
       const int vis = lim - j0;  // columns [0, vis) of this tile are visible keys
-      for (int ng = 0; ng < ng_valid; ++ng) {
-        float bm[bpt];
+      float v[kKT];
 #pragma unroll
-        for (int k = 0; k < bpt; ++k) bm[k] = ninf;
-#pragma unroll
-        for (int c = 0; c < kKT / 32; ++c) {
-          float v[32];
-          tc::tmem_ld32(lane_base + (uint32_t)(buf * kNG * kKT + ng * kKT + c * 32), v);
-          tc::tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int col = c * 32 + i;
-            bm[col / BLK] = fmaxf(bm[col / BLK], col < vis ? v[i] : ninf);
-          }
-        }
-        if (row_ok) {
-          float* dst = srow + (int64_t)(gp * kNG + ng) * a.nblk + j0 / BLK;
-#pragma unroll
-          for (int k = 0; k < bpt; ++k)
-            if (j0 / BLK + k < a.nblk) dst[k] = bm[k];
-        }
-      }
+      for (int c = 0; c < kKT / 32; ++c)
+        tc::tmem_ld32_at(lane_base + (uint32_t)(buf * kNG * kKT + ng * kKT + c * 32), v + c * 32);
+      tc::tmem_wait_ld();
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(b_aempty + 8 * buf);
-    }
-    if (a.fill_tail && row_ok) {
-      for (int ng = 0; ng < ng_valid; ++ng) {
-        float* dst = srow + (int64_t)(gp * kNG + ng) * a.nblk;
-        for (int beta = n_kt * bpt; beta < a.nblk; ++beta) dst[beta] = ninf;
+      float bm[bpt];
+      if (vis >= kKT) {
+#pragma unroll
+        for (int k = 0; k < bpt; ++k) {
+          float m0 = fmaxf(v[k * BLK], v[k * BLK + 1]), m1 = fmaxf(v[k * BLK + 2], v[k * BLK + 3]);
+#pragma unroll
+          for (int i = 4; i + 3 < BLK; i += 4) {
+            m0 = fmax3(m0, v[k * BLK + i], v[k * BLK + i + 1]);
+            m1 = fmax3(m1, v[k * BLK + i + 2], v[k * BLK + i + 3]);
+          }
+          bm[k] = fmaxf(m0, m1);
+        }
+      } else {
+#pragma unroll
+        for (int k = 0; k < bpt; ++k) bm[k] = ninf;
+#pragma unroll
+        for (int col = 0; col < kKT; ++col)
+          bm[col / BLK] = fmaxf(bm[col / BLK], col < vis ? v[col] : ninf);
+      }
+      if (row_ok) {
+#pragma unroll
+        for (int k = 0; k < bpt; ++k)
+          if (j0 / BLK + k < a.nblk) srow[j0 / BLK + k] = bm[k];
       }
     }
+    if (a.fill_tail && row_ok && ng < ng_valid)
+      for (int beta = n_kt * bpt; beta < a.nblk; ++beta) srow[beta] = ninf;
   }
   tc::fence_before_sync();
   __syncthreads();
