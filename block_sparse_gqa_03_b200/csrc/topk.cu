@@ -8,12 +8,17 @@
 // the causal frontier.
 //
 // Method: scores become order-preserving 32-bit keys (blocks past the frontier
-// get key 0, a forced own block the largest key).  The k-th largest key T is
-// found bit by bit from the most significant end: T is the largest value with
-// count(key >= T) >= m.  Keys above T are all taken; keys equal to T are taken
-// in ascending id order until m are chosen.  Rows of up to 1024 blocks use one
-// warp per row with keys in registers (counts by warp reductions, ids emitted in
-// order with ballots); wider rows (long-context decode) use one CTA per row.
+// get key 0, a forced own block the largest key).  T, the m-th largest key
+// (counted with multiplicity), is found from the most significant bit down: the
+// visible keys share the high bits of the row's largest and smallest key, and
+// each step halves the bucket of keys that can still be T by counting the keys
+// at or above its midpoint.  Once at most 32 keys remain in the bucket they are
+// gathered in id order and T is the one of the right rank among them (exact
+// ranks by key, ties by id), so the count steps stop long before the last bit.
+// Keys above T are all taken; keys equal to T are taken in ascending id order
+// until m are chosen.  Rows of up to 1024 blocks use one warp
+// per row with keys in registers (ids emitted in order with ballots); wider rows
+// (long-context decode) use one CTA per row.
 #include "kernels.h"
 
 namespace msa {
@@ -50,54 +55,139 @@ __device__ __forceinline__ RowInfo row_info(const TopkArgs& a, int row) {
   return ri;
 }
 
+// Search state: T's bits above `hi` are known (`prefix`); the bucket is the keys
+// sharing them (`cnt` keys, the forced block excluded), `above` keys (the forced
+// block included) are larger than the whole bucket, and T is the key of rank
+// `need` = m - above in the bucket.  Keys 0 (past the frontier) and 0xffffffff
+// (the forced block) are never in the bucket.
+struct Bucket {
+  uint32_t prefix;
+  int hi, cnt, above;
+};
+
+// Mask of the bits above `hi` (hi in [-1, 31]).
+__device__ __forceinline__ uint32_t bits_above(int hi) {
+  return hi >= 31 ? 0u : (hi < 0 ? 0xffffffffu : ~((2u << hi) - 1u));
+}
+
+__device__ __forceinline__ bool in_bucket(uint32_t key, const Bucket& r) {
+  return key != 0u && key != 0xffffffffu && (key & bits_above(r.hi)) == r.prefix;
+}
+
+// Bucket of a row whose visible keys lie in [kmin, kmax] (kmin <= kmax): their
+// common high bits are known, all `cnt` visible keys are in it.
+__device__ __forceinline__ Bucket bucket_start(uint32_t kmax, uint32_t kmin, int cnt, int above) {
+  const uint32_t diff = kmax ^ kmin;
+  Bucket r;
+  r.hi = diff ? 31 - __clz(diff) : -1;
+  r.prefix = kmax & bits_above(r.hi);
+  r.cnt = cnt;
+  r.above = above;
+  return r;
+}
+
+// One halving step at bit r.hi, given c = count(key >= prefix | 1 << hi) over all
+// of the row's keys.
+__device__ __forceinline__ void bucket_split(Bucket& r, int c, int m) {
+  if (c >= m) {
+    r.prefix |= 1u << r.hi;  // T is in the upper half
+    r.cnt = c - r.above;
+  } else {
+    r.cnt -= c - r.above;  // lower half; the upper half is above T
+    r.above = c;
+  }
+  --r.hi;
+}
+
+// Among the (at most 32) bucket keys gathered in id order in `ck` (lane i holds
+// the i-th, `n` of them), the key of rank need - 1 by (key desc, id asc).
+__device__ __forceinline__ uint32_t rank_pick(uint32_t ck, int n, int need, int lane) {
+  int rank = 0;
+  for (int j = 0; j < n; ++j) {
+    const uint32_t o = __shfl_sync(0xffffffffu, ck, j);
+    rank += (o > ck) || (o == ck && j < lane);
+  }
+  const unsigned hit = __ballot_sync(0xffffffffu, lane < n && rank == need - 1);
+  return __shfl_sync(0xffffffffu, ck, __ffs(hit) - 1);
+}
+
 // Top-m of one row by one warp, element i = e*32 + lane for e < EE: keys in
-// registers, the threshold found bit by bit, ids emitted in order with ballots.
+// registers, counts by warp reductions, the last bucket gathered in `cbuf` (32
+// words private to the warp), ids emitted in order with ballots.
 template <int EE>
 __device__ __forceinline__ void warp_row_topk(const float* s, int32_t* out, const RowInfo& ri,
-                                              int lane) {
+                                              int lane, uint32_t* cbuf) {
+  // The threshold lies between the smallest and the largest visible key: it
+  // shares their common high bits, and the search starts below them.  (The
+  // forced block's own score may widen that range; that is harmless.)  Keys
+  // past the frontier are 0, which k - 1 turns into the largest value for the
+  // minimum.
   uint32_t key[EE];
+  uint32_t kmax = 0u, kmin1 = 0xffffffffu;
 #pragma unroll
   for (int e = 0; e < EE; ++e) {
     const int i = e * 32 + lane;
     key[e] = i < ri.F ? order_key(s[i]) : 0u;
+    kmax = max(kmax, key[e]);
+    kmin1 = min(kmin1, key[e] - 1u);
     if (i == ri.own) key[e] = 0xffffffffu;
   }
   const int m = ri.m;
-  // The threshold lies between the smallest and the largest visible key (the
-  // forced block, key 0xffffffff, always counts): it shares their common high
-  // bits, and the search starts below them.
-  uint32_t kmax = 0u, kmin = 0xffffffffu;
-#pragma unroll
-  for (int e = 0; e < EE; ++e) {
-    const bool vis = key[e] != 0u && key[e] != 0xffffffffu;
-    kmax = vis ? max(kmax, key[e]) : kmax;
-    kmin = vis ? min(kmin, key[e]) : kmin;
-  }
+  const int forced = ri.own >= 0 ? 1 : 0;
   kmax = __reduce_max_sync(0xffffffffu, kmax);
-  kmin = __reduce_min_sync(0xffffffffu, kmin);
+  const uint32_t kmin = __reduce_min_sync(0xffffffffu, kmin1) + 1u;
+  const unsigned lt = (1u << lane) - 1u;
   uint32_t T;
-  if (m <= (ri.own >= 0 ? 1 : 0) || kmax < kmin) {
+  if (m <= forced || kmax < kmin) {
     T = 0xffffffffu;  // only the forced block is taken
   } else {
-    const uint32_t diff = kmax ^ kmin;
-    const int top = diff ? 31 - __clz(diff) : -1;
-    T = top < 0 ? kmax : kmax & ~((2u << top) - 1u);
-    for (int bit = top; bit >= 0; --bit) {
-      const uint32_t cand = T | (1u << bit);
+    Bucket r = bucket_start(kmax, kmin, ri.F - forced, forced);
+    while (r.cnt > 32 && r.hi >= 0) {
+      const uint32_t cand = r.prefix | (1u << r.hi);
       unsigned c4[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
       for (int e = 0; e < EE; ++e) c4[e & 3] += key[e] >= cand;
-      const unsigned cnt = __reduce_add_sync(0xffffffffu, (c4[0] + c4[1]) + (c4[2] + c4[3]));
-      if ((int)cnt >= m) T = cand;
+      bucket_split(r, (int)__reduce_add_sync(0xffffffffu, (c4[0] + c4[1]) + (c4[2] + c4[3])), m);
     }
+    if (r.cnt > 32) {
+      T = r.prefix;  // every bit resolved: the remaining keys all equal T
+    } else {
+      int base = 0;
+#pragma unroll
+      for (int e = 0; e < EE; ++e) {
+        const bool u = in_bucket(key[e], r);
+        const unsigned bu = __ballot_sync(0xffffffffu, u);
+        if (u) cbuf[base + __popc(bu & lt)] = key[e];
+        base += __popc(bu);
+      }
+      __syncwarp();
+      const uint32_t ck = lane < r.cnt ? cbuf[lane] : 0u;
+      __syncwarp();
+      T = rank_pick(ck, r.cnt, m - r.above, lane);
+    }
+  }
+  unsigned ge = 0;
+#pragma unroll
+  for (int e = 0; e < EE; ++e) ge += key[e] >= T;
+  ge = __reduce_add_sync(0xffffffffu, ge);
+  int base = 0;
+  if ((int)ge == m) {
+    // every key equal to T is taken (the usual case: T is unique)
+#pragma unroll
+    for (int e = 0; e < EE; ++e) {
+      const bool sel = key[e] >= T;
+      const unsigned bs = __ballot_sync(0xffffffffu, sel);
+      if (sel) out[base + __popc(bs & lt)] = e * 32 + lane;
+      base += __popc(bs);
+    }
+    return;
   }
   unsigned gt = 0;
 #pragma unroll
   for (int e = 0; e < EE; ++e) gt += key[e] > T;
   gt = __reduce_add_sync(0xffffffffu, gt);
   const int need = m - (int)gt;
-  const unsigned lt = (1u << lane) - 1u;
-  int base = 0, eqbase = 0;
+  int eqbase = 0;
 #pragma unroll
   for (int e = 0; e < EE; ++e) {
     const bool eq = key[e] == T;
@@ -117,9 +207,10 @@ __device__ __forceinline__ void warp_row_topk(const float* s, int32_t* out, cons
 // at least 1, so leaving them out changes nothing); a row with m = F keeps all
 // of its visible blocks and needs no threshold.
 template <int E>
-__global__ void __launch_bounds__(256) topk_warp_kernel(TopkArgs a) {
-  const int lane = threadIdx.x & 31;
-  const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
+__global__ void __launch_bounds__(256, 3) topk_warp_kernel(TopkArgs a) {
+  __shared__ uint32_t cbuf[8][32];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int row = blockIdx.x * 8 + w;
   if (row >= a.rows) return;
   const RowInfo ri = row_info(a, row);
   const float* s = a.scores + (int64_t)row * a.nblk;
@@ -128,17 +219,17 @@ __global__ void __launch_bounds__(256) topk_warp_kernel(TopkArgs a) {
   if (m == ri.F) {
     for (int i = lane; i < m; i += 32) out[i] = i;
   } else if (ne <= 1 || E == 1) {
-    warp_row_topk<1>(s, out, ri, lane);
+    warp_row_topk<1>(s, out, ri, lane, cbuf[w]);
   } else if (ne <= 2 || E == 2) {
-    warp_row_topk<(E < 2 ? E : 2)>(s, out, ri, lane);
+    warp_row_topk<(E < 2 ? E : 2)>(s, out, ri, lane, cbuf[w]);
   } else if (ne <= 4 || E == 4) {
-    warp_row_topk<(E < 4 ? E : 4)>(s, out, ri, lane);
+    warp_row_topk<(E < 4 ? E : 4)>(s, out, ri, lane, cbuf[w]);
   } else if (ne <= 8 || E == 8) {
-    warp_row_topk<(E < 8 ? E : 8)>(s, out, ri, lane);
+    warp_row_topk<(E < 8 ? E : 8)>(s, out, ri, lane, cbuf[w]);
   } else if (ne <= 16 || E == 16) {
-    warp_row_topk<(E < 16 ? E : 16)>(s, out, ri, lane);
+    warp_row_topk<(E < 16 ? E : 16)>(s, out, ri, lane, cbuf[w]);
   } else {
-    warp_row_topk<E>(s, out, ri, lane);
+    warp_row_topk<E>(s, out, ri, lane, cbuf[w]);
   }
   for (int i = m + lane; i < a.topk; i += 32) out[i] = -1;
 }
@@ -174,34 +265,78 @@ __device__ __forceinline__ unsigned cta_exclusive_scan(unsigned v, unsigned* wsu
   return before + inc - v;
 }
 
-// One CTA of NT threads per row; thread i holds elements [i*E, i*E + E).
+// One CTA of NT threads per row; thread i holds elements [i*E, i*E + E).  Counts
+// are CTA sums; warp 0 ranks the last bucket.
 template <int NT, int E>
 __global__ void __launch_bounds__(NT) topk_cta_kernel(TopkArgs a) {
   constexpr int NW = NT / 32;
+  __shared__ uint32_t cbuf[32];
   __shared__ unsigned red[2][32];
   __shared__ unsigned wsum[32];
+  __shared__ uint32_t wmax[NW], wmin[NW];
+  __shared__ uint32_t Ts;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int row = blockIdx.x;
   const RowInfo ri = row_info(a, row);
   const float* s = a.scores + (int64_t)row * a.nblk;
   int32_t* out = a.ids + (int64_t)row * a.topk;
   const int i0 = threadIdx.x * E;
-  uint32_t key[E];
+  const int m = ri.m, forced = ri.own >= 0 ? 1 : 0;
+  if (m == ri.F) {
+    for (int i = threadIdx.x; i < m; i += NT) out[i] = i;
+  } else {
+    uint32_t key[E];
+    uint32_t kmax = 0u, kmin = 0xffffffffu;
 #pragma unroll
-  for (int e = 0; e < E; ++e) {
-    const int i = i0 + e;
-    key[e] = i < ri.F ? order_key(s[i]) : 0u;
-    if (i == ri.own) key[e] = 0xffffffffu;
-  }
-  const int m = ri.m;
-  int buf = 0;
-  if (m > 0) {
-    uint32_t T = 0;
-    for (int bit = 31; bit >= 0; --bit) {
-      const uint32_t cand = T | (1u << bit);
-      unsigned cnt = 0;
+    for (int e = 0; e < E; ++e) {
+      const int i = i0 + e;
+      key[e] = i < ri.F ? order_key(s[i]) : 0u;
+      if (i == ri.own) key[e] = 0xffffffffu;
+      const bool vis = key[e] != 0u && key[e] != 0xffffffffu;
+      kmax = vis ? max(kmax, key[e]) : kmax;
+      kmin = vis ? min(kmin, key[e]) : kmin;
+    }
+    kmax = __reduce_max_sync(0xffffffffu, kmax);
+    kmin = __reduce_min_sync(0xffffffffu, kmin);
+    if (lane == 0) {
+      wmax[warp] = kmax;
+      wmin[warp] = kmin;
+    }
+    __syncthreads();
+    kmax = __reduce_max_sync(0xffffffffu, lane < NW ? wmax[lane] : 0u);
+    kmin = __reduce_min_sync(0xffffffffu, lane < NW ? wmin[lane] : 0xffffffffu);
+    uint32_t T;
+    int buf = 0;
+    if (m <= forced || kmax < kmin) {
+      T = 0xffffffffu;  // only the forced block is taken
+    } else {
+      Bucket r = bucket_start(kmax, kmin, ri.F - forced, forced);
+      while (r.cnt > 32 && r.hi >= 0) {
+        const uint32_t cand = r.prefix | (1u << r.hi);
+        unsigned c = 0;
 #pragma unroll
-      for (int e = 0; e < E; ++e) cnt += key[e] >= cand;
-      if ((int)cta_sum<NW>(cnt, red, buf) >= m) T = cand;
+        for (int e = 0; e < E; ++e) c += key[e] >= cand;
+        bucket_split(r, (int)cta_sum<NW>(c, red, buf), m);
+      }
+      if (r.cnt > 32) {
+        T = r.prefix;  // every bit resolved: the remaining keys all equal T
+      } else {
+        unsigned nu = 0;
+#pragma unroll
+        for (int e = 0; e < E; ++e) nu += in_bucket(key[e], r);
+        unsigned pos = cta_exclusive_scan<NW>(nu, wsum);
+#pragma unroll
+        for (int e = 0; e < E; ++e)
+          if (in_bucket(key[e], r)) cbuf[pos++] = key[e];
+        __syncthreads();
+        if (warp == 0) {
+          const uint32_t ck = lane < r.cnt ? cbuf[lane] : 0u;
+          const uint32_t t = rank_pick(ck, r.cnt, m - r.above, lane);
+          if (lane == 0) Ts = t;
+        }
+        __syncthreads();
+        T = Ts;
+      }
     }
     unsigned gt = 0, eq = 0;
 #pragma unroll
