@@ -61,5 +61,6 @@ cudaError_t launch_kv_attn(const Shape& s, const CUtensorMap& tmq, const CUtenso
 cudaError_t launch_wait_timeout_probe(DeviceStatus* st, uint64_t wait_ns, cudaStream_t stream);
 
 int num_sms();
+int max_smem_optin();
 
 }  // namespace msa

@@ -9,6 +9,21 @@
 
 namespace msa {
 
+// Largest dynamic shared memory a CTA may opt in to (227 KB on sm_100).
+int max_smem_optin() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 232448;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
+        n <= 0)
+      n = 232448;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
 int num_sms() {
   static int cached[64] = {0};
   int dev = 0;

@@ -204,19 +204,23 @@ struct WarpState {
   }
 
   // Stores this warp's state in the merge buffer: o [16][D], m [16], l [16].
-  __device__ __forceinline__ void stash(float* mo, float* mm, float* ml, int warp, int lane) {
+  // Writes this warp's state for the merge: O rows [warp][gr][D] (only the gr
+  // head rows in use), running max and sum [warp][16].
+  __device__ __forceinline__ void stash(float* mo, float* mm, float* ml, int warp, int lane,
+                                        int gr) {
     const int r = lane >> 2, q4 = lane & 3;
     float la = l_a, lb = l_b;
     la += __shfl_xor_sync(0xffffffffu, la, 1);
     la += __shfl_xor_sync(0xffffffffu, la, 2);
     lb += __shfl_xor_sync(0xffffffffu, lb, 1);
     lb += __shfl_xor_sync(0xffffffffu, lb, 2);
-    float* mw = mo + warp * 16 * D;
+    float* mw = mo + warp * gr * D;
 #pragma unroll
     for (int nt = 0; nt < D / 8; ++nt) {
       const int c = nt * 8 + 2 * q4;
-      *reinterpret_cast<float2*>(mw + r * D + c) = make_float2(o[nt][0], o[nt][1]);
-      *reinterpret_cast<float2*>(mw + (r + 8) * D + c) = make_float2(o[nt][2], o[nt][3]);
+      if (r < gr) *reinterpret_cast<float2*>(mw + r * D + c) = make_float2(o[nt][0], o[nt][1]);
+      if (r + 8 < gr)
+        *reinterpret_cast<float2*>(mw + (r + 8) * D + c) = make_float2(o[nt][2], o[nt][3]);
     }
     if (q4 == 0) {
       mm[warp * 16 + r] = m_a;
@@ -231,7 +235,7 @@ struct WarpState {
 // and natural-log LSE (-inf and 0 when no key was seen).
 template <int D, int NC>
 __device__ __forceinline__ void merge_warps(const float* mo, const float* mm, const float* ml,
-                                            int row, int dim, float& val, float& lsev) {
+                                            int gr, int row, int dim, float& val, float& lsev) {
   const float ninf = neg_inf();
   float M = ninf;
 #pragma unroll
@@ -244,7 +248,7 @@ __device__ __forceinline__ void merge_warps(const float* mo, const float* mm, co
   for (int w = 0; w < NC; ++w) {
     const float f = exp2f(mm[w * 16 + row] - M);
     wsum += f * ml[w * 16 + row];
-    acc += f * mo[(w * 16 + row) * D + dim];
+    acc += f * mo[(w * gr + row) * D + dim];
   }
   val = acc / wsum;
   lsev = (M + log2f(wsum)) * kLn2;
@@ -261,21 +265,21 @@ __device__ __forceinline__ void consumer_sync(int nthreads) {
 template <int D>
 __device__ __forceinline__ void produce(const AttnArgs& a, const CUtensorMap* tmk,
                                         const CUtensorMap* tmv, const int32_t* list,
-                                        const int32_t* plist, int n, int64_t row0,
+                                        const int32_t* plist, const int32_t* glist, int n,
                                         uint32_t sbase, uint32_t full0, uint32_t empty0) {
   constexpr int NH = D / 64;
   const uint32_t half_bytes = (uint32_t)a.block * 128u;
   prefetch_tensormap(tmk);
   prefetch_tensormap(tmv);
-  // (head, token, plane) of entry i; a paged cache's pages were looked up when the
-  // list was built (plist, -1 for a page outside the pool)
+  // (head, token, plane) of entry i: the head and the plane (sequence, or page of
+  // a paged cache, -1 for a page outside the pool) were resolved when the list
+  // was built
   auto coords = [&](int i, int& g, int& tok, int& plane) {
     const int e = list[i];
-    const int64_t rowg = row0 + (e >> 16);
-    g = (int)(rowg % a.h);
+    g = glist[i];
     if (a.pg.table == nullptr) {
       tok = (e & 0xffff) * a.block;
-      plane = (int)(rowg / a.h) / a.n_q;
+      plane = plist[i];
     } else {
       tok = 0;
       plane = plist[i] < 0 ? (int)a.pg.pages : plist[i];
@@ -307,38 +311,59 @@ __device__ __forceinline__ void produce(const AttnArgs& a, const CUtensorMap* tm
 }
 
 // Compacts slots [s0, s1) of the flattened id array into the entry list: only
-// blocks holding a visible token are kept, and with a paged cache each kept
-// block's page goes to plist (the lanes look their pages up in parallel).  Run
+// blocks holding a visible token are kept.  For each kept block, glist gets its
+// KV head and plist its sequence (with a paged cache: its page, looked up by the
+// lanes in parallel), so that the producer's loop does no index arithmetic.  Run
 // by one full warp; returns the count.
 __device__ __forceinline__ int compact_ids(const AttnArgs& a, int64_t s0, int64_t s1,
                                            int64_t row0, int32_t* list, int32_t* plist,
-                                           int lane) {
+                                           int32_t* glist, int lane) {
+  constexpr int PF = 8;  // 32-slot groups whose ids are loaded together
   const unsigned lt = (1u << lane) - 1u;
+  // visible-token limit of rows row0 .. row0 + 31, one per lane
+  const int64_t span = (s1 - 1) / a.topk - row0 + 1;
+  const int nrows = span < 32 ? (int)span : 32;
+  // visible-token limit, head and sequence of rows row0 .. row0 + 31, one per lane
+  RowGeo geo_l;
+  geo_l.lim = geo_l.g = geo_l.b = 0;
+  if (lane < nrows) geo_l = row_geo(a, row0 + lane);
   int n = 0;
-  int64_t cached_row = -1;
-  int lim = 0;
-  for (int64_t base = s0; base < s1; base += 32) {
-    const int64_t i = base + lane;
-    int beta = -1;
-    int64_t rowg = row0;
-    if (i < s1) {
-      beta = a.ids[i];
-      rowg = i / a.topk;
-      if (rowg != cached_row) {
-        lim = row_geo(a, rowg).lim;
-        cached_row = rowg;
+  for (int64_t base = s0; base < s1; base += 32 * PF) {
+    int ids[PF];
+#pragma unroll
+    for (int k = 0; k < PF; ++k) {
+      const int64_t i = base + k * 32 + lane;
+      ids[k] = i < s1 ? __ldg(a.ids + i) : -1;
+    }
+#pragma unroll
+    for (int k = 0; k < PF; ++k) {
+      if (base + k * 32 >= s1) break;
+      const int64_t i = base + k * 32 + lane;
+      const int beta = ids[k];
+      const int64_t rowg = i < s1 ? i / a.topk : row0;
+      const int64_t rr = rowg - row0;
+      const int src = rr < 31 ? (int)rr : 31;
+      int lim = __shfl_sync(0xffffffffu, geo_l.lim, src);
+      int g = __shfl_sync(0xffffffffu, geo_l.g, src);
+      int b = __shfl_sync(0xffffffffu, geo_l.b, src);
+      if (rr >= 32) {
+        const RowGeo gr = row_geo(a, rowg);
+        lim = gr.lim;
+        g = gr.g;
+        b = gr.b;
       }
+      const bool bad = beta >= a.nblk;
+      if (bad) record_error(a.st, kErrDeviceAssert, (uint32_t)rowg);
+      const bool keep = beta >= 0 && !bad && (int64_t)beta * a.block < lim;
+      const unsigned msk = __ballot_sync(0xffffffffu, keep);
+      if (keep) {
+        const int at = n + __popc(msk & lt);
+        list[at] = beta | (int)(rr << 16);
+        glist[at] = g;
+        plist[at] = a.pg.table != nullptr ? (int)kv_page(a.pg, b, beta, a.st) : b;
+      }
+      n += __popc(msk);
     }
-    const bool bad = beta >= a.nblk;
-    if (bad) record_error(a.st, kErrDeviceAssert, (uint32_t)rowg);
-    const bool keep = beta >= 0 && !bad && (int64_t)beta * a.block < lim;
-    const unsigned msk = __ballot_sync(0xffffffffu, keep);
-    if (keep) {
-      const int at = n + __popc(msk & lt);
-      list[at] = beta | (int)((rowg - row0) << 16);
-      if (a.pg.table != nullptr) plist[at] = (int)kv_page(a.pg, (int)(rowg / a.h) / a.n_q, beta, a.st);
-    }
-    n += __popc(msk);
   }
   return n;
 }
@@ -349,7 +374,6 @@ __global__ void __launch_bounds__(5 * 32, 1)
     sparse_attn_rows_kernel(const __grid_constant__ CUtensorMap tmk,
                             const __grid_constant__ CUtensorMap tmv, AttnArgs a) {
   constexpr int NC = 4;
-  if (status_failed(a.st)) return;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -357,7 +381,8 @@ __global__ void __launch_bounds__(5 * 32, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + a.region_bytes);
   int32_t* list = reinterpret_cast<int32_t*>(bars + 2 * a.stages);
   int32_t* n_list = list + a.list_cap;
-  int32_t* plist = n_list + 1;  // [list_cap] pages, paged cache only
+  int32_t* plist = n_list + 1;       // [list_cap] sequence or page of each entry
+  int32_t* glist = plist + a.list_cap;  // [list_cap] KV head of each entry
   const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + a.stages);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t rowg = blockIdx.x;
@@ -371,20 +396,26 @@ __global__ void __launch_bounds__(5 * 32, 1)
     }
     fence_mbar_init();
   }
+  // the consumers load their queries while the list is built
+  WarpState<D> ws;
+  const RowGeo rg = row_geo(a, rowg);
   if (warp == NC) {
-    const int n = compact_ids(a, rowg * a.topk, (rowg + 1) * a.topk, rowg, list, plist, lane);
-    if (lane == 0) *n_list = n;
+    // after an earlier timeout the kernel does nothing (status read first: its
+    // latency overlaps the compaction)
+    const bool skip = status_failed(a.st);
+    const int n = compact_ids(a, rowg * a.topk, (rowg + 1) * a.topk, rowg, list, plist, glist, lane);
+    if (lane == 0) *n_list = skip ? -1 : n;
+  } else {
+    ws.reset();
+    ws.load_q(a, rg, lane);
   }
   __syncthreads();
   const int n = *n_list;
+  if (n < 0) return;
   if (warp == NC) {
-    if (lane == 0 && n > 0) produce<D>(a, &tmk, &tmv, list, plist, n, rowg, sbase, full0, empty0);
+    if (lane == 0 && n > 0) produce<D>(a, &tmk, &tmv, list, plist, glist, n, sbase, full0, empty0);
     return;
   }
-  const RowGeo rg = row_geo(a, rowg);
-  WarpState<D> ws;
-  ws.reset();
-  ws.load_q(a, rg, lane);
   for (int i = 0; i < n; ++i) {
     const int u0 = i * nsub;
     const int st0 = (warp - (u0 % NC) + NC) % NC;  // first slice of block i owned by this warp
@@ -406,14 +437,14 @@ __global__ void __launch_bounds__(5 * 32, 1)
   // Merge the warps' states (the stages are free: every load was consumed).
   consumer_sync(NC * 32);
   float* mo = reinterpret_cast<float*>(smem);
-  float* mm = mo + NC * 16 * D;
+  float* mm = mo + NC * a.G * D;
   float* ml = mm + NC * 16;
-  ws.stash(mo, mm, ml, warp, lane);
+  ws.stash(mo, mm, ml, warp, lane, a.G);
   consumer_sync(NC * 32);
   for (int x = tid; x < a.G * D; x += NC * 32) {
     const int row = x / D, dim = x % D;
     float val, lsev;
-    merge_warps<D, NC>(mo, mm, ml, row, dim, val, lsev);
+    merge_warps<D, NC>(mo, mm, ml, a.G, row, dim, val, lsev);
     const int hq = rg.g * a.G + row;
     a.out[rg.b * a.o_s0 + (int64_t)rg.t * a.o_s1 + (int64_t)hq * a.o_s2 + dim] =
         __bfloat16_as_ushort(__float2bfloat16_rn(val));
@@ -426,19 +457,19 @@ template <int D, int NC>
 __global__ void __launch_bounds__((NC + 1) * 32, 1)
     sparse_attn_stream_kernel(const __grid_constant__ CUtensorMap tmk,
                               const __grid_constant__ CUtensorMap tmv, AttnArgs a) {
-  if (status_failed(a.st)) return;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
-  float* mo = reinterpret_cast<float*>(smem + a.merge_off);  // [NC][16][D]
-  float* mm = mo + NC * 16 * D;                               // [NC][16]
+  float* mo = reinterpret_cast<float*>(smem + a.merge_off);  // [NC][G][D]
+  float* mm = mo + NC * a.G * D;                              // [NC][16]
   float* ml = mm + NC * 16;                                   // [NC][16]
   int* flag = reinterpret_cast<int*>(ml + NC * 16);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + a.region_bytes);
   int32_t* list = reinterpret_cast<int32_t*>(bars + 2 * a.stages);
   int32_t* n_list = list + a.list_cap;
-  int32_t* plist = n_list + 1;  // [list_cap] pages, paged cache only
+  int32_t* plist = n_list + 1;       // [list_cap] sequence or page of each entry
+  int32_t* glist = plist + a.list_cap;  // [list_cap] KV head of each entry
   const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + a.stages);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nsub = a.block / 16;
@@ -456,29 +487,34 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1)
     }
     fence_mbar_init();
   }
+  // the consumers load their first row's queries while the list is built
+  WarpState<D> ws;
+  int64_t cur = r0;
+  RowGeo rg = row_geo(a, cur);
   if (warp == NC) {
-    const int n = compact_ids(a, s0, s1, r0, list, plist, lane);
-    if (lane == 0) *n_list = n;
+    // after an earlier timeout the kernel does nothing; the status load is issued
+    // first so that its latency overlaps the compaction
+    const bool skip = status_failed(a.st);
+    const int n = compact_ids(a, s0, s1, r0, list, plist, glist, lane);
+    if (lane == 0) *n_list = skip ? -1 : n;
+  } else {
+    ws.reset();
+    ws.load_q(a, rg, lane);
   }
   __syncthreads();
   const int n = *n_list;
+  if (n < 0) return;
   if (warp == NC) {
-    if (lane == 0 && n > 0) produce<D>(a, &tmk, &tmv, list, plist, n, r0, sbase, full0, empty0);
+    if (lane == 0 && n > 0) produce<D>(a, &tmk, &tmv, list, plist, glist, n, sbase, full0, empty0);
     return;
   }
-
-  WarpState<D> ws;
   bool failed = false;
-  int64_t cur = r0;
-  RowGeo rg = row_geo(a, cur);
-  ws.reset();
-  ws.load_q(a, rg, lane);
 
   // Ends the segment of row `cur` held by this CTA: merge the warps, then write
   // the output (row entirely in this CTA) or a partial (and merge the row's
   // partials if this CTA is the last of the row to finish).
   auto flush = [&]() {
-    ws.stash(mo, mm, ml, warp, lane);
+    ws.stash(mo, mm, ml, warp, lane, a.G);
     consumer_sync(NC * 32);
     const int64_t c_first = (cur * a.topk) / a.per;
     const int64_t c_last = ((cur + 1) * a.topk - 1) / a.per;
@@ -487,7 +523,7 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1)
     for (int x = tid; x < a.G * D; x += NC * 32) {
       const int row = x / D, dim = x % D;
       float val, lsev;
-      merge_warps<D, NC>(mo, mm, ml, row, dim, val, lsev);
+      merge_warps<D, NC>(mo, mm, ml, a.G, row, dim, val, lsev);
       const int hq = rg.g * a.G + row;
       if (nseg == 1) {
         a.out[rg.b * a.o_s0 + (int64_t)rg.t * a.o_s1 + (int64_t)hq * a.o_s2 + dim] =
@@ -504,7 +540,48 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1)
       consumer_sync(NC * 32);
       if (tid == 0) *flag = atomicAdd(&a.counters[cur], 1);
       consumer_sync(NC * 32);
-      if (*flag == nseg - 1) {
+      if (*flag == nseg - 1 && nseg <= NC) {
+        // Last CTA of the row: stage the row's partials in the (now free) merge
+        // buffer with independent loads, then merge them from shared memory.
+        __threadfence();
+        float* so = mo;              // [G][nseg][D]
+        float* sl = mo + NC * a.G * D;  // [G][nseg], over the free max/sum arrays
+        const int64_t pr_g = ((int64_t)rg.bt * a.H + rg.g * a.G) * a.smax;
+        const int q4n = nseg * (D / 4);
+#pragma unroll 4
+        for (int y = tid; y < a.G * q4n; y += NC * 32) {
+          const int row = y / q4n, sp = (y % q4n) / (D / 4), c4 = y % (D / 4);
+          const float4 v = __ldcg(reinterpret_cast<const float4*>(
+                                      a.part_o + (pr_g + (int64_t)row * a.smax + sp) * D) +
+                                  c4);
+          reinterpret_cast<float4*>(so)[(row * nseg + sp) * (D / 4) + c4] = v;
+        }
+        for (int y = tid; y < a.G * nseg; y += NC * 32)
+          sl[y] = __ldcg(a.part_lse + pr_g + (int64_t)(y / nseg) * a.smax + y % nseg);
+        consumer_sync(NC * 32);
+        for (int x = tid; x < a.G * D; x += NC * 32) {
+          const int row = x / D, dim = x % D;
+          const int hq = rg.g * a.G + row;
+          const float ninf = neg_inf();
+          float M = ninf;
+          for (int sp = 0; sp < nseg; ++sp) M = fmaxf(M, sl[row * nseg + sp]);
+          float val = 0.f, lsev = ninf;
+          if (M != ninf) {
+            float den = 0.f, acc = 0.f;
+            for (int sp = 0; sp < nseg; ++sp) {
+              const float w = exp2f((sl[row * nseg + sp] - M) * kLog2e);
+              den += w;
+              acc += w * so[(row * nseg + sp) * D + dim];
+            }
+            val = acc / den;
+            lsev = M + log2f(den) * kLn2;
+          }
+          a.out[rg.b * a.o_s0 + (int64_t)rg.t * a.o_s1 + (int64_t)hq * a.o_s2 + dim] =
+              __bfloat16_as_ushort(__float2bfloat16_rn(val));
+          if (dim == 0 && a.lse) a.lse[(int64_t)rg.bt * a.H + hq] = lsev;
+        }
+      } else if (*flag == nseg - 1) {
+        // more segments than the merge buffer holds: merge from global memory
         __threadfence();
         for (int x = tid; x < a.G * D; x += NC * 32) {
           const int row = x / D, dim = x % D;
@@ -629,7 +706,7 @@ bool make_q_group_map(CUtensorMap* map, const uint16_t* base, const Shape& s) {
          CUDA_SUCCESS;
 }
 
-constexpr int kStreamNC = 4;       // consumer warps of the streaming kernel
+constexpr int kStreamNC = 8;       // consumer warps of the streaming kernel
 constexpr int kMaxList = 4096;     // entries a streaming CTA compacts up front
 constexpr uint32_t kSmemCap = 227u * 1024u;
 
@@ -656,13 +733,12 @@ AttnPlan plan_attn(const Shape& s) {
   const int nsub = s.block / 16;
   const int64_t rows_g = (int64_t)s.batch * s.n_q * s.h;
   pl.total = rows_g * s.topk;
-  const uint32_t merge_bytes = (uint32_t)kStreamNC * 16 * (s.d + 2) * 4 + 16;
+  // merge buffer: O [warps][G][d], max and sum [warps][16], one flag word
+  const uint32_t merge_bytes =
+      (uint32_t)kStreamNC * s.G * s.d * 4 + (uint32_t)kStreamNC * 16 * 2 * 4 + 16;
   // Few rows with many blocks (decode): the persistent streaming kernel.
   pl.stream = rows_g < 4LL * num_sms();
   if (pl.stream) {
-    pl.stages = stage_count((int)((160u * 1024u) / pl.stage_bytes), nsub, kStreamNC);
-    pl.region_bytes = pl.stages * pl.stage_bytes + ((merge_bytes + 1023) & ~1023u);
-    pl.merge_off = pl.stages * pl.stage_bytes;
     pl.ctas = num_sms();
     pl.per = (int)((pl.total + pl.ctas - 1) / pl.ctas);
     if (pl.per > kMaxList) {
@@ -672,6 +748,15 @@ AttnPlan plan_attn(const Shape& s) {
     pl.ctas = (int)((pl.total + pl.per - 1) / pl.per);
     pl.smax = (s.topk - 1) / pl.per + 2;
     pl.list_cap = pl.per;
+    // as many stages as the shared memory holds: the bytes in flight per SM set
+    // the streaming rate
+    const size_t merge_r = (merge_bytes + 1023) & ~1023u;
+    const size_t fixed = 1024 + merge_r + 4 * (3 * (size_t)pl.list_cap + 1);
+    const size_t cap = (size_t)max_smem_optin();
+    const int fit = cap > fixed ? (int)((cap - fixed) / (pl.stage_bytes + 16)) : 0;
+    pl.stages = stage_count(fit, nsub, kStreamNC);  // fit >= 3 for every supported shape
+    pl.region_bytes = pl.stages * pl.stage_bytes + merge_r;
+    pl.merge_off = pl.stages * pl.stage_bytes;
   } else {
     // Two CTAs per SM when the stages allow it, else one with deeper buffering.
     int want = (int)((100u * 1024u) / pl.stage_bytes);
@@ -684,8 +769,7 @@ AttnPlan plan_attn(const Shape& s) {
     pl.smax = 1;
     pl.list_cap = s.topk;
   }
-  pl.smem_bytes = 1024 + pl.region_bytes + 16 * pl.stages + 4 * (pl.list_cap + 1) +
-                  (s.pages.table != nullptr ? 4 * (size_t)pl.list_cap : 0);
+  pl.smem_bytes = 1024 + pl.region_bytes + 16 * pl.stages + 4 * (3 * (size_t)pl.list_cap + 1);
   return pl;
 }
 
