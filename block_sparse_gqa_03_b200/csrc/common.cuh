@@ -96,6 +96,37 @@ __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
 }
 
+// Programmatic dependent launch.  Every kernel of the library starts with
+// grid_dep_wait(), which returns once the grid launched before it on the stream
+// has completed and its writes are visible (immediately when the kernel was not
+// launched as a dependent), and then allows its own dependent to be scheduled:
+// the next kernel's CTAs take free SM slots and wait there, so its launch overlaps
+// this kernel's tail.
+__device__ __forceinline__ void grid_dep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dep_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Launches `kernel` on `stream` as a programmatic dependent of the previous
+// kernel on the stream (see grid_dep_wait).
+template <typename... K, typename... A>
+inline cudaError_t launch_pdl(void (*kernel)(K...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t stream, A... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 __device__ __forceinline__ void fence_mbar_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }

@@ -118,6 +118,8 @@ __device__ __forceinline__ void block_max(const ScanArgs& a, const uint16_t* kbb
 // the h groups of the sequence's query.
 template <int DI, int NT>
 __global__ void __launch_bounds__(kScanWarps * 32) index_scan_decode_kernel(ScanArgs a) {
+  grid_dep_wait();
+  grid_dep_launch();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int r = lane >> 2, q = lane & 3;
   const int64_t item = (int64_t)blockIdx.x * kScanWarps + warp;
@@ -153,6 +155,8 @@ __global__ void __launch_bounds__(kScanWarps * 32) index_scan_decode_kernel(Scan
 // (query, group) pairs and each warp walks the blocks up to the tile's frontier.
 template <int DI, int NT>
 __global__ void __launch_bounds__(kScanWarps * 32) index_scan_kernel(ScanArgs a) {
+  grid_dep_wait();
+  grid_dep_launch();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int r = lane >> 2, q = lane & 3;
   const int tile = blockIdx.x % a.ntiles;
@@ -213,9 +217,9 @@ template <int DI, int NT>
 cudaError_t run_scan(const ScanArgs& a, int batch, cudaStream_t stream) {
   if (a.n_q == 1) {
     const int64_t items = (int64_t)batch * a.nblk;
-    index_scan_decode_kernel<DI, NT>
-        <<<(unsigned)((items + kScanWarps - 1) / kScanWarps), kScanWarps * 32, 0, stream>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(index_scan_decode_kernel<DI, NT>,
+                      dim3((unsigned)((items + kScanWarps - 1) / kScanWarps)), dim3(kScanWarps * 32),
+                      0, stream, a);
   }
   const int ctas_per_row = a.ntiles * batch;
   // Spread the block range of each query tile over enough warps to fill the
@@ -225,8 +229,7 @@ cudaError_t run_scan(const ScanArgs& a, int batch, cudaStream_t stream) {
   const int max_split = (a.nblk + kScanWarps - 1) / kScanWarps;
   split = max(1, min(split, max_split));
   dim3 grid(ctas_per_row, split);
-  index_scan_kernel<DI, NT><<<grid, kScanWarps * 32, 0, stream>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(index_scan_kernel<DI, NT>, grid, dim3(kScanWarps * 32), 0, stream, a);
 }
 
 }  // namespace

@@ -48,6 +48,8 @@ template <int DI, int BLK>
 __global__ void __launch_bounds__(kTcThreads, 1)
     index_score_tc_kernel(const __grid_constant__ CUtensorMap tmq,
                           const __grid_constant__ CUtensorMap tmk, TcArgs a) {
+  grid_dep_wait();
+  grid_dep_launch();
   constexpr int NATOM = DI / 64;               // 128-byte K atoms per row
   constexpr uint32_t ATOM = 128u * 128u;       // one atom of a 128-row tile
   constexpr uint32_t Q_BYTES = NATOM * ATOM;   // one group's query tile
@@ -298,8 +300,8 @@ cudaError_t run_tc(const Shape& s, const uint16_t* q_idx, const uint16_t* k_idx,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   const unsigned grid = (unsigned)((int64_t)s.batch * a.n_gpairs * a.n_mtiles);
-  index_score_tc_kernel<DI, BLK><<<grid, kTcThreads, smem, stream>>>(tmq, tmk, a);
-  return cudaGetLastError();
+  return launch_pdl(index_score_tc_kernel<DI, BLK>, dim3(grid), dim3(kTcThreads), smem, stream,
+                    tmq, tmk, a);
 }
 
 }  // namespace

@@ -31,17 +31,24 @@ cudaError_t launch_index_scores_tc(const Shape& s, const uint16_t* q_idx, const 
                                    float* scores, bool fill_tail, DeviceStatus* st,
                                    cudaStream_t stream);
 
-// Stage 1c: top-k block ids, int32 [batch, n_q, h, topk], from the scores.
+// Stage 1c: top-k block ids, int32 [batch, n_q, h, topk], from the scores.  When
+// `zero` is given, the kernel also clears zero[0, nzero) (the attention's merge
+// counters, so that a fused forward needs no separate memset between the stages).
 cudaError_t launch_topk(const Shape& s, const float* scores, int32_t* ids, DeviceStatus* st,
-                        cudaStream_t stream);
+                        cudaStream_t stream, int* zero = nullptr, int nzero = 0);
 
 // Stage 2: workspace bytes for the split-KV partials, then the attention.
 size_t attn_partial_bytes(const Shape& s);
 int attn_launches(const Shape& s);
+// The streaming (decode) kernel's per-row merge counters inside `partials`, or
+// nullptr when the shape takes another kernel; *count receives their number.
+int* attn_merge_counters(const Shape& s, void* partials, int* count);
+// counters_zeroed: the merge counters were cleared on the stream already (by the
+// top-k kernel of the same forward), so no memset is issued.
 cudaError_t launch_sparse_attn(const Shape& s, const uint16_t* q, const uint16_t* k,
                                const uint16_t* v, const int32_t* ids, uint16_t* out, float* lse,
                                void* partials, size_t partial_bytes, DeviceStatus* st,
-                               cudaStream_t stream);
+                               cudaStream_t stream, bool counters_zeroed = false);
 
 // Stage 2 for prefill, KV-major on tcgen05 (d 64/128, block 64/128, n_q > 1):
 // inverted index, tiles of gathered (query, head) rows per selected block,

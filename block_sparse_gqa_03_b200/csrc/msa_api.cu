@@ -199,7 +199,7 @@ uint8_t* at(void* ws, size_t off) { return reinterpret_cast<uint8_t*>(ws) + off;
 
 msa_status_t run_select(const Shape& s, const msa_bf16_t* q_idx, const msa_bf16_t* k_idx,
                         int32_t* ids, float* user_scores, void* ws, const Layout& l,
-                        cudaStream_t stream) {
+                        cudaStream_t stream, int* zero = nullptr, int nzero = 0) {
   msa::DeviceStatus* st = reinterpret_cast<msa::DeviceStatus*>(ws);
   float* scores = user_scores ? user_scores : reinterpret_cast<float*>(at(ws, l.scores_off));
   cudaError_t e = msa::index_scores_tc_supported(s)
@@ -208,7 +208,7 @@ msa_status_t run_select(const Shape& s, const msa_bf16_t* q_idx, const msa_bf16_
                       : msa::launch_index_scores(s, q_idx, k_idx, scores, user_scores != nullptr,
                                                  st, stream);
   if (e != cudaSuccess) return MSA_ERR_CUDA;
-  return cuda_status(msa::launch_topk(s, scores, ids, st, stream));
+  return cuda_status(msa::launch_topk(s, scores, ids, st, stream, zero, nzero));
 }
 
 }  // namespace
@@ -264,10 +264,17 @@ msa_status_t msa_forward(const msa_params_t* params, const msa_bf16_t* q, const 
   const Layout l = layout(s, MSA_OP_FORWARD);
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   int32_t* ids = block_ids ? block_ids : reinterpret_cast<int32_t*>(at(workspace, l.ids_off));
-  if ((rc = run_select(s, q_idx, k_idx, ids, block_scores, workspace, l, cs)) != MSA_OK) return rc;
+  // the top-k kernel clears the attention's merge counters, so that the two
+  // stages follow each other with no memset in between
+  int ncounters = 0;
+  int* counters = msa::attn_merge_counters(s, at(workspace, l.part_off), &ncounters);
+  if ((rc = run_select(s, q_idx, k_idx, ids, block_scores, workspace, l, cs, counters,
+                       ncounters)) != MSA_OK)
+    return rc;
   return cuda_status(msa::launch_sparse_attn(s, q, k, v, ids, out, lse, at(workspace, l.part_off),
                                              l.part_bytes,
-                                             reinterpret_cast<msa::DeviceStatus*>(workspace), cs));
+                                             reinterpret_cast<msa::DeviceStatus*>(workspace), cs,
+                                             counters != nullptr));
 }
 
 msa_status_t msa_get_device_status(void* workspace, msa_stream_t stream) {

@@ -373,6 +373,8 @@ template <int D>
 __global__ void __launch_bounds__(5 * 32, 1)
     sparse_attn_rows_kernel(const __grid_constant__ CUtensorMap tmk,
                             const __grid_constant__ CUtensorMap tmv, AttnArgs a) {
+  grid_dep_wait();
+  grid_dep_launch();
   constexpr int NC = 4;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -457,6 +459,8 @@ template <int D, int NC>
 __global__ void __launch_bounds__((NC + 1) * 32, 1)
     sparse_attn_stream_kernel(const __grid_constant__ CUtensorMap tmk,
                               const __grid_constant__ CUtensorMap tmv, AttnArgs a) {
+  grid_dep_wait();
+  grid_dep_launch();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -800,10 +804,21 @@ int attn_launches(const Shape& s) {
   return !pl.stream && kv_attn_supported(s) ? kv_launches(s) : 1;
 }
 
+int* attn_merge_counters(const Shape& s, void* partials, int* count) {
+  const AttnPlan pl = plan_attn(s);
+  *count = 0;
+  if (!pl.stream || partials == nullptr) return nullptr;
+  const size_t nrow_h = (size_t)s.batch * s.n_q * s.H;
+  const float* part_lse = reinterpret_cast<float*>(partials) + nrow_h * pl.smax * s.d;
+  *count = s.batch * s.n_q * s.h;
+  return reinterpret_cast<int*>(
+      (reinterpret_cast<uintptr_t>(part_lse + nrow_h * pl.smax) + 255) & ~uintptr_t(255));
+}
+
 cudaError_t launch_sparse_attn(const Shape& s, const uint16_t* q, const uint16_t* k,
                                const uint16_t* v, const int32_t* ids, uint16_t* out, float* lse,
                                void* partials, size_t partial_bytes, DeviceStatus* st,
-                               cudaStream_t stream) {
+                               cudaStream_t stream, bool counters_zeroed) {
   const AttnPlan pl = plan_attn(s);
   if (pl.smem_bytes > kSmemCap) return cudaErrorInvalidValue;
   CUtensorMap tmk, tmv;
@@ -857,37 +872,43 @@ cudaError_t launch_sparse_attn(const Shape& s, const uint16_t* q, const uint16_t
       err = cudaFuncSetAttribute(sparse_attn_rows_kernel<128>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem_bytes);
       if (err != cudaSuccess) return err;
-      sparse_attn_rows_kernel<128><<<grid, 5 * 32, pl.smem_bytes, stream>>>(tmk, tmv, a);
+      err = launch_pdl(sparse_attn_rows_kernel<128>, grid, dim3(5 * 32), pl.smem_bytes, stream, tmk,
+                       tmv, a);
     } else {
       err = cudaFuncSetAttribute(sparse_attn_rows_kernel<64>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem_bytes);
       if (err != cudaSuccess) return err;
-      sparse_attn_rows_kernel<64><<<grid, 5 * 32, pl.smem_bytes, stream>>>(tmk, tmv, a);
+      err = launch_pdl(sparse_attn_rows_kernel<64>, grid, dim3(5 * 32), pl.smem_bytes, stream, tmk,
+                       tmv, a);
     }
-    return cudaGetLastError();
+    return err;
   }
   const size_t nrow_h = (size_t)s.batch * s.n_q * s.H;
   if (partials == nullptr || partial_bytes < attn_partial_bytes(s)) return cudaErrorInvalidValue;
   a.part_o = reinterpret_cast<float*>(partials);
   a.part_lse = a.part_o + nrow_h * pl.smax * s.d;
-  a.counters = reinterpret_cast<int*>(
-      (reinterpret_cast<uintptr_t>(a.part_lse + nrow_h * pl.smax) + 255) & ~uintptr_t(255));
-  err = cudaMemsetAsync(a.counters, 0, (size_t)s.batch * s.n_q * s.h * sizeof(int), stream);
-  if (err != cudaSuccess) return err;
+  int ncounters = 0;
+  a.counters = attn_merge_counters(s, partials, &ncounters);
+  if (!counters_zeroed) {
+    err = cudaMemsetAsync(a.counters, 0, (size_t)ncounters * sizeof(int), stream);
+    if (err != cudaSuccess) return err;
+  }
   const dim3 grid((unsigned)pl.ctas);
   constexpr int NT = (kStreamNC + 1) * 32;
   if (s.d == 128) {
     err = cudaFuncSetAttribute(sparse_attn_stream_kernel<128, kStreamNC>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem_bytes);
     if (err != cudaSuccess) return err;
-    sparse_attn_stream_kernel<128, kStreamNC><<<grid, NT, pl.smem_bytes, stream>>>(tmk, tmv, a);
+    err = launch_pdl(sparse_attn_stream_kernel<128, kStreamNC>, grid, dim3(NT), pl.smem_bytes,
+                     stream, tmk, tmv, a);
   } else {
     err = cudaFuncSetAttribute(sparse_attn_stream_kernel<64, kStreamNC>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem_bytes);
     if (err != cudaSuccess) return err;
-    sparse_attn_stream_kernel<64, kStreamNC><<<grid, NT, pl.smem_bytes, stream>>>(tmk, tmv, a);
+    err = launch_pdl(sparse_attn_stream_kernel<64, kStreamNC>, grid, dim3(NT), pl.smem_bytes,
+                     stream, tmk, tmv, a);
   }
-  return cudaGetLastError();
+  return err;
 }
 
 }  // namespace msa

@@ -30,7 +30,15 @@ struct TopkArgs {
   const int32_t* seq_lens;
   int rows, n_q, max_kv, h, block, nblk, topk, causal, force_own;
   DeviceStatus* st;
+  int* zero;  // cleared by CTA 0 when not null (nzero words)
+  int nzero;
 };
+
+// CTA 0 clears the words the caller asked for (before any early exit).
+__device__ __forceinline__ void clear_words(const TopkArgs& a) {
+  if (blockIdx.x == 0 && a.zero != nullptr)
+    for (int i = threadIdx.x; i < a.nzero; i += blockDim.x) a.zero[i] = 0;
+}
 
 __device__ __forceinline__ uint32_t order_key(float f) {
   const uint32_t u = __float_as_uint(f);
@@ -208,6 +216,9 @@ __device__ __forceinline__ void warp_row_topk(const float* s, int32_t* out, cons
 // of its visible blocks and needs no threshold.
 template <int E>
 __global__ void __launch_bounds__(256, 3) topk_warp_kernel(TopkArgs a) {
+  grid_dep_wait();
+  grid_dep_launch();
+  clear_words(a);
   __shared__ uint32_t cbuf[8][32];
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const int row = blockIdx.x * 8 + w;
@@ -269,6 +280,9 @@ __device__ __forceinline__ unsigned cta_exclusive_scan(unsigned v, unsigned* wsu
 // are CTA sums; warp 0 ranks the last bucket.
 template <int NT, int E>
 __global__ void __launch_bounds__(NT) topk_cta_kernel(TopkArgs a) {
+  grid_dep_wait();
+  grid_dep_launch();
+  clear_words(a);
   constexpr int NW = NT / 32;
   __shared__ uint32_t cbuf[32];
   __shared__ unsigned red[2][32];
@@ -366,7 +380,7 @@ __global__ void __launch_bounds__(NT) topk_cta_kernel(TopkArgs a) {
 }  // namespace
 
 cudaError_t launch_topk(const Shape& s, const float* scores, int32_t* ids, DeviceStatus* st,
-                        cudaStream_t stream) {
+                        cudaStream_t stream, int* zero, int nzero) {
   TopkArgs a;
   a.scores = scores;
   a.ids = ids;
@@ -381,13 +395,14 @@ cudaError_t launch_topk(const Shape& s, const float* scores, int32_t* ids, Devic
   a.causal = s.causal;
   a.force_own = s.force_own;
   a.st = st;
+  a.zero = zero;
+  a.nzero = nzero;
   const int n = s.nblk;
   if (n <= 1024) {
     const dim3 grid((a.rows + 7) / 8);
 #define MSA_TOPK_WARP(E_)                                             \
   if (n <= 32 * E_) {                                                 \
-    topk_warp_kernel<E_><<<grid, 256, 0, stream>>>(a);                \
-    return cudaGetLastError();                                        \
+    return launch_pdl(topk_warp_kernel<E_>, grid, dim3(256), 0, stream, a); \
   }
     MSA_TOPK_WARP(1)
     MSA_TOPK_WARP(2)
@@ -400,8 +415,7 @@ cudaError_t launch_topk(const Shape& s, const float* scores, int32_t* ids, Devic
   const dim3 grid(a.rows);
 #define MSA_TOPK_CTA(NT_, E_)                                      \
   if (n <= NT_ * E_) {                                             \
-    topk_cta_kernel<NT_, E_><<<grid, NT_, 0, stream>>>(a);         \
-    return cudaGetLastError();                                     \
+    return launch_pdl(topk_cta_kernel<NT_, E_>, grid, dim3(NT_), 0, stream, a); \
   }
   MSA_TOPK_CTA(256, 8)
   MSA_TOPK_CTA(256, 16)
