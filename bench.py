@@ -40,10 +40,10 @@ L2_BYTES = 126 * 2**20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # Per-launch DRAM traffic (read + write bytes) of the dominant kernel, from one ncu
-# capture (profiles/sparse_attn_stream_decode128k_b4.md: batch 4, 134.42 MB read +
-# 4.57 MB written, scaled by 4 to the batch of 16, the work growing in proportion).
+# capture (profiles/sparse_attn_stream_decode128k_b4.md: batch 4, 134.46 MB read +
+# 3.49 MB written, scaled by 4 to the batch of 16, the work growing in proportion).
 # Absent entries report null; an entry is removed when its kernel changes.
-TRAFFIC = {("decode_128k", "attn"): 4 * (134.422016e6 + 4.572928e6)}
+TRAFFIC = {("decode_128k", "attn"): 4 * (134.462208e6 + 3.493888e6)}
 
 
 def load_peaks():
