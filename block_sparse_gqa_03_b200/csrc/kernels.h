@@ -37,6 +37,13 @@ cudaError_t launch_index_scores_tc(const Shape& s, const uint16_t* q_idx, const 
 cudaError_t launch_topk(const Shape& s, const float* scores, int32_t* ids, DeviceStatus* st,
                         cudaStream_t stream, int* zero = nullptr, int nzero = 0);
 
+// Decode-step cache write: the n_q new tokens of every sequence (dense
+// [batch, n_q, h, d] K and V, [batch, n_q, d_idx] K_idx; any may be null) go to
+// positions L_b - n_q + t of the contiguous or paged cache.
+cudaError_t launch_append_kv(const Shape& s, const uint16_t* k_new, const uint16_t* v_new,
+                             const uint16_t* ki_new, uint16_t* k, uint16_t* v, uint16_t* ki,
+                             DeviceStatus* st, cudaStream_t stream);
+
 // Stage 2: workspace bytes for the split-KV partials, then the attention.
 size_t attn_partial_bytes(const Shape& s);
 int attn_launches(const Shape& s);

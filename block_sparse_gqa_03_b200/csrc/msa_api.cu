@@ -189,7 +189,8 @@ Layout layout(const Shape& s, msa_op_t op) {
 msa_status_t check_ws(const Shape& s, msa_op_t op, void* ws, size_t bytes) {
   if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) != 0)
     return MSA_ERR_WORKSPACE;
-  if (bytes < layout(s, op).total) return MSA_ERR_WORKSPACE;
+  if (bytes < (op == MSA_OP_APPEND_KV ? msa::kStatusBytes : layout(s, op).total))
+    return MSA_ERR_WORKSPACE;
   return MSA_OK;
 }
 
@@ -218,6 +219,7 @@ extern "C" {
 size_t msa_workspace_size(const msa_params_t* params, msa_op_t op) {
   Shape s;
   if (make_shape(params, &s) != MSA_OK) return 0;
+  if (op == MSA_OP_APPEND_KV) return msa::kStatusBytes;
   if (op != MSA_OP_INDEX_SELECT && op != MSA_OP_SPARSE_ATTN && op != MSA_OP_FORWARD) return 0;
   return layout(s, op).total;
 }
@@ -277,6 +279,27 @@ msa_status_t msa_forward(const msa_params_t* params, const msa_bf16_t* q, const 
                                              counters != nullptr));
 }
 
+msa_status_t msa_append_kv(const msa_params_t* params, const msa_bf16_t* k_new,
+                           const msa_bf16_t* v_new, const msa_bf16_t* k_idx_new, msa_bf16_t* k,
+                           msa_bf16_t* v, msa_bf16_t* k_idx, void* workspace,
+                           size_t workspace_bytes, msa_stream_t stream) {
+  Shape s;
+  msa_status_t rc = make_shape(params, &s);
+  if (rc != MSA_OK) return rc;
+  if ((k_new != nullptr && (!k || !aligned16(k) || !aligned16(k_new) ||
+                            check_strides3(s.k_s) != MSA_OK || s.k_s[2] < s.d)) ||
+      (v_new != nullptr && (!v || !aligned16(v) || !aligned16(v_new) ||
+                            check_strides3(s.v_s) != MSA_OK || s.v_s[2] < s.d)) ||
+      (k_idx_new != nullptr &&
+       (!k_idx || !aligned16(k_idx) || !aligned16(k_idx_new) || !good_stride(s.ki_s[0]) ||
+        !good_stride(s.ki_s[1]) || s.ki_s[1] < s.d_idx)))
+    return MSA_ERR_INVALID_ARG;
+  if ((rc = check_ws(s, MSA_OP_APPEND_KV, workspace, workspace_bytes)) != MSA_OK) return rc;
+  return cuda_status(msa::launch_append_kv(s, k_new, v_new, k_idx_new, k, v, k_idx,
+                                           reinterpret_cast<msa::DeviceStatus*>(workspace),
+                                           reinterpret_cast<cudaStream_t>(stream)));
+}
+
 msa_status_t msa_get_device_status(void* workspace, msa_stream_t stream) {
   if (workspace == nullptr) return MSA_ERR_WORKSPACE;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
@@ -317,6 +340,7 @@ int msa_launch_count(const msa_params_t* params, msa_op_t op) {
     case MSA_OP_INDEX_SELECT: return 2;
     case MSA_OP_SPARSE_ATTN: return msa::attn_launches(s);
     case MSA_OP_FORWARD: return 2 + msa::attn_launches(s);
+    case MSA_OP_APPEND_KV: return 1;
   }
   return -1;
 }

@@ -32,10 +32,11 @@ MSA_ERR_DEVICE_ASSERT = 6
 MSA_OP_INDEX_SELECT = 0
 MSA_OP_SPARSE_ATTN = 1
 MSA_OP_FORWARD = 2
+MSA_OP_APPEND_KV = 3
 
 EXPORTED = ("msa_workspace_size", "msa_index_select", "msa_sparse_attn", "msa_forward",
             "msa_get_device_status", "msa_workspace_init", "msa_selftest_wait_timeout",
-            "msa_launch_count", "msa_sparse_attn_noalloc", "msa_status_string")
+            "msa_launch_count", "msa_sparse_attn_noalloc", "msa_status_string", "msa_append_kv")
 
 
 class MsaError(RuntimeError):
@@ -86,6 +87,8 @@ def load_library():
             lib.msa_sparse_attn.restype = I
             lib.msa_forward.argtypes = [P, P, P, P, P, P, P, P, P, P, P, S, P]
             lib.msa_forward.restype = I
+            lib.msa_append_kv.argtypes = [P, P, P, P, P, P, P, P, S, P]
+            lib.msa_append_kv.restype = I
             lib.msa_get_device_status.argtypes = [P, P]
             lib.msa_get_device_status.restype = I
             lib.msa_workspace_init.argtypes = [P, S, P]
@@ -287,6 +290,36 @@ def msa_sparse_attn_noalloc(q, k, v, block_ids, *, block, causal=True, seq_lens=
                                                   _ptr(block_ids), _ptr(out), _ptr(lse),
                                                   _stream(stream)), "msa_sparse_attn_noalloc")
     return out
+
+
+def msa_append_kv(k, v, k_idx, k_new=None, v_new=None, k_idx_new=None, *, block,
+                  seq_lens=None, block_table=None, max_kv=None,
+                  workspace: Workspace | None = None, stream=None):
+    """Writes the new tokens' rows into the cache: k_new / v_new [b, n_new, h, d] and
+    k_idx_new [b, n_new, d_idx] (dense) go to positions L_b - n_new + t of k / v
+    [b, max_kv, h, d] and k_idx [b, max_kv, d_idx] (or of the page pools, with
+    ``block_table``).  Any of the new tensors may be None, and then its cache too
+    (``k`` or ``v`` must be given for the shapes)."""
+    ref = next(t for t in (k_new, v_new, k_idx_new) if t is not None)
+    b, n_new = ref.shape[0], ref.shape[1]
+    kv = k if k is not None else v
+    h, d = kv.shape[2], kv.shape[3]
+    max_kv, num_pages = _kv_extent(kv, block_table, max_kv)
+    for t in (k_new, v_new, k_idx_new):
+        if t is not None and not t.is_contiguous():
+            raise ValueError("new rows must be dense")
+    d_idx = k_idx.shape[-1] if k_idx is not None else 32
+    p = make_params(batch=b, n_q=n_new, max_kv=max_kv, H=h, h=h, d=d, d_idx=d_idx,
+                    block=block, topk=1, seq_lens=seq_lens, k=k, v=v, k_idx=k_idx,
+                    block_table=block_table, num_pages=num_pages)
+    need = msa_workspace_size(p, MSA_OP_APPEND_KV)
+    if need == 0:
+        raise MsaError(MSA_ERR_INVALID_ARG, "msa_workspace_size")
+    ws = _workspace(workspace, kv.device).get(need)
+    _check(load_library().msa_append_kv(ctypes.byref(p), _ptr(k_new), _ptr(v_new),
+                                        _ptr(k_idx_new), _ptr(k), _ptr(v), _ptr(k_idx),
+                                        ws.data_ptr(), ws.numel(), _stream(stream)),
+           "msa_append_kv")
 
 
 def msa_forward(q, k, v, q_idx, k_idx, *, block, topk, causal=True, force_own_block=False,

@@ -92,7 +92,8 @@ typedef enum msa_status {
 typedef enum msa_op {
   MSA_OP_INDEX_SELECT = 0,
   MSA_OP_SPARSE_ATTN = 1,
-  MSA_OP_FORWARD = 2
+  MSA_OP_FORWARD = 2,
+  MSA_OP_APPEND_KV = 3
 } msa_op_t;
 
 typedef struct msa_params {
@@ -152,6 +153,27 @@ MSA_API msa_status_t msa_forward(const msa_params_t* params, const msa_bf16_t* q
                          const msa_bf16_t* v, const msa_bf16_t* q_idx, const msa_bf16_t* k_idx,
                          msa_bf16_t* out, int32_t* block_ids, float* block_scores, float* lse,
                          void* workspace, size_t workspace_bytes, msa_stream_t stream);
+
+/* Decode-step cache write, so that a step needs no per-row copies: for every
+ * sequence b and new token t < n_q (params->n_q new tokens per sequence, already
+ * counted in seq_lens), at position pos = L_b - n_q + t:
+ *   k[b, pos, g, :] = k_new[b, t, g, :]   v[b, pos, g, :] = v_new[b, t, g, :]
+ *   k_idx[b, pos, :] = k_idx_new[b, t, :]
+ * k_new, v_new: bf16 [batch, n_q, h, d] and k_idx_new: bf16 [batch, n_q, d_idx],
+ * dense row-major and 16-byte aligned; any of the three may be NULL (that cache
+ * is not written, and its cache pointer may then be NULL).  k, v, k_idx and their
+ * strides (k_strides, v_strides, ki_strides) are those the other calls take,
+ * paged caches included (row pos % block of page block_table[b, pos / block]).
+ * A position < 0 or a page id outside the pool is recorded as
+ * MSA_ERR_DEVICE_ASSERT and that token is not written.  The workspace holds the
+ * status word only (msa_workspace_size(params, MSA_OP_APPEND_KV) bytes).
+ * The cache keeps the plain GQA layout ("MiniMax M3 的 MSA ...", section
+ * "三条有意为之的减法", first item), one block per physical block ("深度解析M3多模态
+ * 模型与Token Plan", list of MSA's innovations, first item). */
+MSA_API msa_status_t msa_append_kv(const msa_params_t* params, const msa_bf16_t* k_new,
+                                   const msa_bf16_t* v_new, const msa_bf16_t* k_idx_new,
+                                   msa_bf16_t* k, msa_bf16_t* v, msa_bf16_t* k_idx,
+                                   void* workspace, size_t workspace_bytes, msa_stream_t stream);
 
 /* Synchronises `stream`, returns the first error a kernel recorded in this
  * workspace since the last reset (MSA_OK if none) and clears it. */

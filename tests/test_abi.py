@@ -122,6 +122,24 @@ def test_paged_params_validated(lib):
                            fake, 1 << 30, None) == msa.MSA_ERR_INVALID_ARG
 
 
+def test_append_args_validated(lib):
+    p = valid_params()
+    fake = 1 << 20
+    assert msa.msa_workspace_size(p, msa.MSA_OP_APPEND_KV) == 256
+    assert msa.msa_launch_count(p, msa.MSA_OP_APPEND_KV) == 1
+    # new K rows without a K cache, misaligned new rows, a workspace without room
+    # for the status word
+    assert lib.msa_append_kv(ctypes.byref(p), fake, None, None, None, None, None, fake, 256,
+                             None) == msa.MSA_ERR_INVALID_ARG
+    assert lib.msa_append_kv(ctypes.byref(p), fake + 2, None, None, fake, None, None, fake, 256,
+                             None) == msa.MSA_ERR_INVALID_ARG
+    assert lib.msa_append_kv(ctypes.byref(p), fake, fake, fake, fake, fake, fake, fake, 128,
+                             None) == msa.MSA_ERR_WORKSPACE
+    p.ki_strides[1] = 16  # index-key rows closer than d_idx
+    assert lib.msa_append_kv(ctypes.byref(p), None, None, fake, None, None, fake, fake, 256,
+                             None) == msa.MSA_ERR_INVALID_ARG
+
+
 def test_binding_fails_loudly_without_library(monkeypatch):
     monkeypatch.setattr(msa, "LIB_PATH", "/nonexistent/libmsa.so")
     monkeypatch.setattr(msa, "_lib", None)
