@@ -436,42 +436,55 @@ def run_ours(args, prob, world, rank, local):
 
 
 def run_e2e(args, prob, x, dev, world, msa, kw):
-    """Same metric through msa_forward with host buffers: pinned host -> device copies
-    of the step's inputs, the call, and the output read back, inside the timed region."""
+    """Same metric through the public API with host buffers: pinned host -> device
+    copies of the step's inputs, the calls, and the output read back, inside the
+    timed region."""
     stream = torch.cuda.current_stream(dev)
-    if prob.is_decode:
-        # a decode step's inputs: the new token's queries, and its K/V/K_idx rows
-        # written into the resident cache at position L_b - 1
-        names = ["q", "q_idx"]
-        host = {n: x[n].cpu().pin_memory() for n in names}
-        L = (x["seq_lens"].cpu().tolist() if x["seq_lens"] is not None
-             else [prob.max_kv] * prob.batch)
-        rows = {n: torch.stack([cache_row(prob, x, n, b, L[b] - 1) for b in range(prob.batch)])
-                .cpu().pin_memory() for n in ("k", "v", "k_idx")}
-        h2d = sum(t.numel() * t.element_size() for t in host.values())
-        h2d += sum(t.numel() * t.element_size() for t in rows.values())
-    else:
-        names = ["q", "k", "v", "q_idx", "k_idx"]
-        host = {n: x[n].cpu().pin_memory() for n in names}
-        rows, L = {}, None
-        h2d = sum(t.numel() * t.element_size() for t in host.values())
     out_dev = torch.empty_like(x["q"])
     out_host = torch.empty(out_dev.shape, dtype=out_dev.dtype, pin_memory=True)
     d2h = out_host.numel() * out_host.element_size()
     ws = msa.Workspace(dev)
     nsteps = max(1, min(args.steps, 20))
+    if prob.is_decode:
+        # A decode step's inputs are the new token's queries and its K/V/K_idx rows:
+        # packed in one pinned buffer, copied once, the rows written into the
+        # resident cache at position L_b - 1 by msa_append_kv, then msa_forward.
+        # (The rows are the cache's own, so the cache is unchanged step to step.)
+        L = (x["seq_lens"].cpu().tolist() if x["seq_lens"] is not None
+             else [prob.max_kv] * prob.batch)
+        parts = {"q": x["q"], "q_idx": x["q_idx"]}
+        for n in ("k", "v", "k_idx"):
+            parts[n + "_new"] = torch.stack([cache_row(prob, x, n, b, L[b] - 1)
+                                             for b in range(prob.batch)]).unsqueeze(1)
+        flat = [t.reshape(-1) for t in parts.values()]
+        host = torch.cat(flat).cpu().pin_memory()
+        staging = torch.empty_like(host, device=dev)
+        views, off = {}, 0
+        for n, t in parts.items():
+            views[n] = staging[off:off + t.numel()].view(t.shape)
+            off += t.numel()
+        h2d = host.numel() * host.element_size()
+        akw = {k: kw[k] for k in ("block", "seq_lens", "block_table", "max_kv") if k in kw}
 
-    dst = {n: [cache_row(prob, x, n, b, L[b] - 1) for b in range(prob.batch)] for n in rows}
+        def one():
+            staging.copy_(host, non_blocking=True)
+            msa.msa_append_kv(x["k"], x["v"], x["k_idx"], views["k_new"], views["v_new"],
+                              views["k_idx_new"], workspace=ws, **akw)
+            msa.msa_forward(views["q"], x["k"], x["v"], views["q_idx"], x["k_idx"],
+                            topk=prob.topk, force_own_block=prob.force_own, out=out_dev,
+                            workspace=ws, **kw)
+            out_host.copy_(out_dev, non_blocking=True)
+    else:
+        names = ["q", "k", "v", "q_idx", "k_idx"]
+        host = {n: x[n].cpu().pin_memory() for n in names}
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
 
-    def one():
-        for n in names:
-            x[n].copy_(host[n], non_blocking=True)
-        for n, t in rows.items():
-            for b in range(prob.batch):
-                dst[n][b].copy_(t[b], non_blocking=True)
-        msa.msa_forward(x["q"], x["k"], x["v"], x["q_idx"], x["k_idx"], topk=prob.topk,
-                        force_own_block=prob.force_own, out=out_dev, workspace=ws, **kw)
-        out_host.copy_(out_dev, non_blocking=True)
+        def one():
+            for n in names:
+                x[n].copy_(host[n], non_blocking=True)
+            msa.msa_forward(x["q"], x["k"], x["v"], x["q_idx"], x["k_idx"], topk=prob.topk,
+                            force_own_block=prob.force_own, out=out_dev, workspace=ws, **kw)
+            out_host.copy_(out_dev, non_blocking=True)
 
     one()
     torch.cuda.synchronize(dev)
