@@ -474,6 +474,49 @@ def run_e2e(args, prob, x, dev, world, msa, kw):
                             topk=prob.topk, force_own_block=prob.force_own, out=out_dev,
                             workspace=ws, **kw)
             out_host.copy_(out_dev, non_blocking=True)
+    elif x["seq_lens"] is None and "block_table" not in kw:
+        # Prefill as a chunked prefill through the same API: the inputs are copied
+        # chunk by chunk in token order on a copy stream, msa_forward runs query
+        # chunk c (the context up to the chunk's last query) as soon as its rows
+        # have landed, and each chunk's output is read back on a third stream, so
+        # that the copies overlap the compute.
+        names = ["q", "k", "v", "q_idx", "k_idx"]
+        host = {n: x[n].cpu().pin_memory() for n in names}
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        qc = min(prob.n_q, 16384 if prob.batch == 1 else 8192)
+        off = prob.max_kv - prob.n_q  # query t sits at position off + t
+        chunks = []
+        for c0 in range(0, prob.n_q, qc):
+            c1 = min(c0 + qc, prob.n_q)
+            k0 = 0 if c0 == 0 else off + c0
+            chunks.append((c0, c1, k0, off + c1,
+                           torch.full((prob.batch,), off + c1, dtype=torch.int32, device=dev)))
+        s_copy, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        landed = [torch.cuda.Event() for _ in chunks]
+        done = [torch.cuda.Event() for _ in chunks]
+        ckw = {k: v for k, v in kw.items() if k != "seq_lens"}
+
+        def one():
+            s_copy.wait_stream(stream)
+            with torch.cuda.stream(s_copy):
+                for (c0, c1, k0, k1, _), ev in zip(chunks, landed):
+                    for b in range(prob.batch):
+                        for n in ("q", "q_idx"):
+                            x[n][b, c0:c1].copy_(host[n][b, c0:c1], non_blocking=True)
+                        for n in ("k", "v", "k_idx"):
+                            x[n][b, k0:k1].copy_(host[n][b, k0:k1], non_blocking=True)
+                    ev.record(s_copy)
+            for (c0, c1, _, _, sl), ev, dn in zip(chunks, landed, done):
+                stream.wait_event(ev)
+                msa.msa_forward(x["q"][:, c0:c1], x["k"], x["v"], x["q_idx"][:, c0:c1], x["k_idx"],
+                                topk=prob.topk, force_own_block=prob.force_own,
+                                out=out_dev[:, c0:c1], workspace=ws, seq_lens=sl, **ckw)
+                dn.record(stream)
+                s_out.wait_event(dn)
+                with torch.cuda.stream(s_out):
+                    for b in range(prob.batch):
+                        out_host[b, c0:c1].copy_(out_dev[b, c0:c1], non_blocking=True)
+            stream.wait_stream(s_out)
     else:
         names = ["q", "k", "v", "q_idx", "k_idx"]
         host = {n: x[n].cpu().pin_memory() for n in names}
