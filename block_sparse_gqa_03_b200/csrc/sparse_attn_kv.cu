@@ -701,136 +701,101 @@ __global__ void __launch_bounds__(kKvThreads, 1)
 }
 
 // -------------------------------------------------------------- combine
-// m[base + rl] for rl < RPI, as selects (an indexed pick would put m in local memory).
-template <int RPI>
-__device__ __forceinline__ float pick_row(const float* m, int base, int rl) {
-  if constexpr (RPI == 2) {
-    return rl ? m[base + 1] : m[base];
-  } else {
-    static_assert(RPI == 4, "rows per load");
-    return (rl & 2) ? ((rl & 1) ? m[base + 3] : m[base + 2]) : ((rl & 1) ? m[base + 1] : m[base]);
-  }
-}
-
-// One warp per (query, group): merge the G heads' partials over the group's valid
-// slots by log-sum-exp weights; bf16 output and the natural-log LSE.
-template <int D, int GM>
-__global__ void __launch_bounds__(256, GM * D <= 1024 ? 2 : 1) kv_combine_kernel(KvArgs a, int BLK) {
+// One warp per (query, head): merge the head's partials over the group's valid
+// slots by log-sum-exp weights; bf16 output and the natural-log LSE.  Lanes
+// take 32 slots at a time, so the loads of many partials are in flight at once.
+template <int D>
+__global__ void __launch_bounds__(256) kv_combine_kernel(KvArgs a, int BLK) {
   grid_dep_wait();
   grid_dep_launch();
-  // One warp per (query, group): a slot's G partial rows are consecutive rows of
-  // its tile, read as one contiguous piece, 16 bytes per lane.  Lane = (row rl of
-  // a load, 16-byte chunk c); a load covers RPI rows, ni loads cover the G heads.
-  constexpr int LPR = D / 8;         // lanes per partial row
-  constexpr int RPI = 32 / LPR;      // rows per warp-wide load
-  constexpr int MI = GM / RPI;       // loads per slot at most
-  constexpr int U = MI <= 2 ? 4 : 2;  // slots whose loads are in flight together
   const int lane = threadIdx.x & 31;
   const int64_t wid = blockIdx.x * 8LL + (threadIdx.x >> 5);
-  if (wid >= (int64_t)a.nbt * a.h) return;
-  const int g = (int)(wid % a.h);
-  const int bt_rel = (int)(wid / a.h);
+  const int64_t n = (int64_t)a.nbt * a.H;
+  if (wid >= n) return;
+  const int hq = (int)(wid % a.H);
+  const int bt_rel = (int)(wid / a.H);
+  const int g = hq / a.G, hi = hq - g * a.G;
   const int bt = (int)a.bt0 + bt_rel;
   const int b = bt / a.n_q, t = bt % a.n_q;
   const int lim = visible_limit(a, b, t);
-  const int G = a.G;
-  const int rl = lane / LPR, c = lane % LPR;
   const int32_t* row_ids = a.ids + ((int64_t)bt * a.h + g) * a.topk;
   const int64_t p0 = ((int64_t)bt_rel * a.h + g) * a.topk;
   const float ninf = -__int_as_float(0x7f800000);
-  // pass 1: per-head maximum of the valid slots' LSEs, slots spread over the lanes
-  float M[GM];
-#pragma unroll
-  for (int h = 0; h < GM; ++h) M[h] = ninf;
+  constexpr int PER = D / 32;  // dims per lane
+  float M = ninf;
   for (int s0 = 0; s0 < a.topk; s0 += 32) {
     const int s = s0 + lane;
+    float l = ninf;
     if (s < a.topk) {
       const int beta = __ldg(row_ids + s);
-      if (beta >= 0 && beta < a.nblk && beta * BLK < lim) {
-        const float* l = a.part_lse + (p0 + s) * G;
-#pragma unroll
-        for (int h = 0; h < GM; ++h)
-          if (h < G) M[h] = fmaxf(M[h], __ldg(l + h));
-      }
+      if (beta >= 0 && beta < a.nblk && beta * BLK < lim) l = __ldg(a.part_lse + (p0 + s) * a.G + hi);
     }
+    M = fmaxf(M, l);
   }
 #pragma unroll
-  for (int h = 0; h < GM; ++h)
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  float acc[PER];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M[h] = fmaxf(M[h], __shfl_xor_sync(0xffffffffu, M[h], o));
-  // this lane's heads hi = i * RPI + rl
-  float Mi[MI], den[MI], acc[MI][8];
-#pragma unroll
-  for (int i = 0; i < MI; ++i) {
-    Mi[i] = pick_row<RPI>(M, i * RPI, rl);
-    den[i] = 0.f;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) acc[i][e] = 0.f;
-  }
-  // pass 2: weighted sum, slot by slot (the warp on one slot at a time, U slots'
-  // loads in flight); an empty slot reads row 0 with weight 0, through a select,
-  // so that whatever row 0 holds cannot leak into the sum
-  for (int s0 = 0; s0 < a.topk; s0 += 32) {
-    const int s = s0 + lane;
-    int prow = 0;
-    bool ok = false;
-    if (s < a.topk) {
-      const int beta = __ldg(row_ids + s);
-      ok = beta >= 0 && beta < a.nblk && beta * BLK < lim;
-      if (ok) prow = __ldg(a.slot_row + p0 + s);
-    }
-    const int cnt = min(32, a.topk - s0);
-    for (int j0 = 0; j0 < cnt; j0 += U) {
-      uint4 u[U][MI];
-      float l[U][MI];
-      bool use[U];
-#pragma unroll
-      for (int jj = 0; jj < U; ++jj) {
-        const int j = min(j0 + jj, cnt - 1);
-        use[jj] = j0 + jj < cnt && __shfl_sync(0xffffffffu, ok ? 1 : 0, j) != 0;
-        const int rj = __shfl_sync(0xffffffffu, prow, j);
-        const float* lp = a.part_lse + (p0 + s0 + j) * G;
-#pragma unroll
-        for (int i = 0; i < MI; ++i) {
-          const int hi = i * RPI + rl;
-          const bool live = use[jj] && hi < G;
-          u[jj][i] = __ldg(reinterpret_cast<const uint4*>(
-                             a.part_o + (int64_t)(live ? rj + hi : 0) * D) +
-                         c);
-          l[jj][i] = live ? __ldg(lp + hi) : ninf;
+  for (int e = 0; e < PER; ++e) acc[e] = 0.f;
+  float den = 0.f;
+  if (M != ninf) {
+    for (int s0 = 0; s0 < a.topk; s0 += 32) {
+      const int s = s0 + lane;
+      float wgt = 0.f;
+      int prow = 0;  // partial row of this lane's slot (row 0 stands in for none)
+      if (s < a.topk) {
+        const int beta = __ldg(row_ids + s);
+        if (beta >= 0 && beta < a.nblk && beta * BLK < lim) {
+          prow = __ldg(a.slot_row + p0 + s) + hi;
+          wgt = __expf(__ldg(a.part_lse + (p0 + s) * a.G + hi) - M);
         }
       }
+      den += wgt;
+      // Loads are issued for every slot of the pass (a slot without a partial reads
+      // row 0, which exists); such a slot contributes through a select, never a
+      // multiply, so whatever that row holds cannot leak into the sum.  Sixteen slots
+      // per round keep several loads in flight per lane.
+      const int cnt = min(32, a.topk - s0);
+      for (int j0 = 0; j0 < cnt; j0 += 16) {
+        uint2 u[16];
+        float wj[16];
 #pragma unroll
-      for (int jj = 0; jj < U; ++jj)
-#pragma unroll
-        for (int i = 0; i < MI; ++i) {
-          const bool live = l[jj][i] != ninf;
-          const float w = live ? __expf(l[jj][i] - Mi[i]) : 0.f;
-          den[i] += w;
-          const uint32_t x[4] = {u[jj][i].x, u[jj][i].y, u[jj][i].z, u[jj][i].w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            acc[i][2 * e] += live ? w * __uint_as_float(x[e] << 16) : 0.f;
-            acc[i][2 * e + 1] += live ? w * __uint_as_float(x[e] & 0xffff0000u) : 0.f;
+        for (int j = 0; j < 16; ++j) {
+          const int jj = min(j0 + j, cnt - 1);
+          wj[j] = __shfl_sync(0xffffffffu, wgt, jj);
+          if (j0 + j >= cnt) wj[j] = 0.f;
+          const int rj = __shfl_sync(0xffffffffu, prow, jj);
+          const uint16_t* src = a.part_o + (int64_t)rj * D + lane * PER;
+          if constexpr (PER == 4) {
+            u[j] = __ldg(reinterpret_cast<const uint2*>(src));
+          } else {
+            u[j] = make_uint2(__ldg(reinterpret_cast<const uint32_t*>(src)), 0u);
           }
         }
-    }
-  }
-  uint16_t* ob = a.out + (int64_t)b * a.o_s0 + (int64_t)t * a.o_s1 + c * 8;
 #pragma unroll
-  for (int i = 0; i < MI; ++i) {
-    const int hi = i * RPI + rl;
-    if (hi >= G) continue;
-    const int hq = g * G + hi;
-    const float inv = den[i] > 0.f ? 1.f / den[i] : 0.f;
-    *reinterpret_cast<uint4*>(ob + (int64_t)hq * a.o_s2) =
-        make_uint4(pack_bf16(acc[i][0] * inv, acc[i][1] * inv),
-                   pack_bf16(acc[i][2] * inv, acc[i][3] * inv),
-                   pack_bf16(acc[i][4] * inv, acc[i][5] * inv),
-                   pack_bf16(acc[i][6] * inv, acc[i][7] * inv));
-    if (c == 0 && a.lse)
-      a.lse[(int64_t)bt * a.H + hq] = Mi[i] != ninf && den[i] > 0.f ? Mi[i] + __logf(den[i]) : ninf;
+        for (int j = 0; j < 16; ++j) {
+          const bool use = wj[j] != 0.f;
+          acc[0] += use ? wj[j] * __uint_as_float(u[j].x << 16) : 0.f;
+          acc[1] += use ? wj[j] * __uint_as_float(u[j].x & 0xffff0000u) : 0.f;
+          if constexpr (PER == 4) {
+            acc[2] += use ? wj[j] * __uint_as_float(u[j].y << 16) : 0.f;
+            acc[3] += use ? wj[j] * __uint_as_float(u[j].y & 0xffff0000u) : 0.f;
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
   }
+  const float inv = den > 0.f ? 1.f / den : 0.f;
+  uint16_t* o = a.out + (int64_t)b * a.o_s0 + (int64_t)t * a.o_s1 + (int64_t)hq * a.o_s2 + lane * PER;
+  if constexpr (PER == 4) {
+    *reinterpret_cast<uint2*>(o) = make_uint2(pack_bf16(acc[0] * inv, acc[1] * inv),
+                                              pack_bf16(acc[2] * inv, acc[3] * inv));
+  } else {
+    *reinterpret_cast<uint32_t*>(o) = pack_bf16(acc[0] * inv, acc[1] * inv);
+  }
+  if (lane == 0 && a.lse) a.lse[(int64_t)bt * a.H + hq] = M != ninf ? M + __logf(den) : ninf;
 }
 
 }  // namespace
@@ -911,7 +876,7 @@ cudaError_t run_kv(const Shape& s, KvArgs& a, const KvPlan& p, const CUtensorMap
     if (err != cudaSuccess) return err;
     const int64_t n = (int64_t)a.nbt * s.h * s.topk;
     const int grid = (int)((n + 255) / 256 < (int64_t)sms * 8 ? (n + 255) / 256 : (int64_t)sms * 8);
-    const int64_t warps = (int64_t)a.nbt * s.h;  // combine: one warp per (query, group)
+    const int64_t warps = (int64_t)a.nbt * s.H;
     if ((err = launch_pdl(kv_count_kernel, dim3(grid), dim3(256), 0, stream, a, BLK)) !=
             cudaSuccess ||
         (err = launch_pdl(kv_scan_kernel, dim3(1), dim3(1024), 0, stream, a)) != cudaSuccess ||
@@ -922,10 +887,7 @@ cudaError_t run_kv(const Shape& s, KvArgs& a, const KvPlan& p, const CUtensorMap
       return err;
     // The combine is launched plainly: as a programmatic dependent of kv_attn
     // (its CTAs taking the SMs that kv_attn leaves early) it measured ~6% slower.
-    if (s.G <= 8)
-      kv_combine_kernel<D, 8><<<(unsigned)((warps + 7) / 8), 256, 0, stream>>>(a, BLK);
-    else
-      kv_combine_kernel<D, 16><<<(unsigned)((warps + 7) / 8), 256, 0, stream>>>(a, BLK);
+    kv_combine_kernel<D><<<(unsigned)((warps + 7) / 8), 256, 0, stream>>>(a, BLK);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
   }
   return cudaSuccess;
