@@ -334,7 +334,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
       mbar_init(b_sfree + 8 * i, 4);
     }
     for (int i = 0; i < NQ; ++i) {
-      mbar_init(b_qfull + 8 * i, 2);
+      mbar_init(b_qfull + 8 * i, 3);
       mbar_init(b_qempty + 8 * i, 1);
     }
     for (int i = 0; i < 4; ++i) mbar_init(b_lfull + 8 * i, 4);
@@ -353,64 +353,119 @@ __global__ void __launch_bounds__(kKvThreads, 1)
   // code under each limit is exactly that branch.
   const int wg = warp >> 2;
   Walker w;
-  if (warp == kWarpProd) {
-    // ---------------------------------------------------------- K/V producer
+  if (warp == kWarpProd || warp == kWarpGather || warp == kWarpGather + 1) {
+    // ------------------------------------------ K/V producer (warp 0), Q gather
+    // Warp 0 loads a block's K/V when the tile walk reaches a new block.  The Q
+    // gather: one TMA load per (query, 64-dim atom) brings the query's G heads,
+    // i.e. G consecutive tile rows, into the swizzled operand layout; a tile's
+    // loads are dealt round-robin to warps 0, 2 and 3 (a warp issues its loads one
+    // lane after another, so the more warps, the sooner a tile's Q is requested).
+    // A tile's query positions are read while the previous tile is issued.
     tc::regs_dec<kRegsLoad>();
     if (n > 0) {
+      const bool kv_role = warp == kWarpProd;
+      const int gi = kv_role ? 0 : warp - kWarpGather + 1;  // gather share
       w.seek(a, tile0);
       if (lane == 0) {
-        prefetch_tensormap(&tmk);
-        prefetch_tensormap(&tmv);
+        prefetch_tensormap(&tmq);
+        if (kv_role) {
+          prefetch_tensormap(&tmk);
+          prefetch_tensormap(&tmv);
+        }
       }
+      const uint32_t rows_bytes = (uint32_t)a.G * 128u;
+      // loads o = gi + 3 (lane + 32 k) of a tile: query o / NH, atom o % NH
+      auto load_t = [&](int first, int nq, int (&tq)[3]) {
+#pragma unroll
+        for (int k = 0; k < 3; ++k) {
+          const int o = gi + 3 * (lane + 32 * k);
+          tq[k] = o < NH * nq ? __ldg(&a.entries[first + o / NH].y) : 0;
+        }
+      };
+      int nq = w.count(a, tile0), qg = w.g, qbb = w.b;
+      bool new_block = true;
+      int tq[3];
+      load_t(w.first(a, tile0), nq, tq);
       int use = -1;
       uint32_t land_par = 0;  // bit s: parity of the next wait on kv_land[s]
-      bool ok = true;
-      for (int idx = 0; idx < n && ok; ++idx) {
-        const int tile = tile0 + idx;
-        if (!w.advance(a, tile) && idx > 0) continue;
-        ++use;
-        const int s = use & 1;
-        if (use >= 2)
-          ok = mbar_wait_warp(b_kvempty + 8 * s, ((use >> 1) - 1) & 1, a.st, 0x201u, a.wait_ns);
-        if (!ok) break;
-        // V rows [r0, BLK) lie past the sequence end and may hold anything: they
-        // are zeroed once the block has landed, so that a zero probability never
-        // meets a non-finite value.
-        const int L = kv_length(a.seq_lens, w.b, a.max_kv, a.st);
-        const int r0 = max(0, L - w.beta * BLK);
-        const bool fix = r0 < BLK;
-        const uint32_t bar = (fix ? b_kvland : b_kvfull) + 8 * s;
-        const uint32_t kd = skv + s * KV_BYTES, vd = kd + NH * HALF;
-        if (lane == 0) {
-          int tok, plane;
-          kv_block_coords(a.pg, w.b, w.beta, BLK, a.st, tok, plane);
-          mbar_arrive_expect_tx(bar, KV_BYTES);
+      bool ok = true, q_ok = true;
+      for (int idx = 0; idx < n; ++idx) {
+        if (kv_role && new_block && ok) {
+          ++use;
+          const int s = use & 1;
+          if (use >= 2)
+            ok = mbar_wait_warp(b_kvempty + 8 * s, ((use >> 1) - 1) & 1, a.st, 0x201u, a.wait_ns);
+          if (ok) {
+          // V rows [r0, BLK) lie past the sequence end and may hold anything: they
+          // are zeroed once the block has landed, so that a zero probability never
+          // meets a non-finite value.
+          const int L = kv_length(a.seq_lens, w.b, a.max_kv, a.st);
+          const int r0 = max(0, L - w.beta * BLK);
+          const bool fix = r0 < BLK;
+          const uint32_t bar = (fix ? b_kvland : b_kvfull) + 8 * s;
+          const uint32_t kd = skv + s * KV_BYTES, vd = kd + NH * HALF;
+          if (lane == 0) {
+            int tok, plane;
+            kv_block_coords(a.pg, w.b, w.beta, BLK, a.st, tok, plane);
+            mbar_arrive_expect_tx(bar, KV_BYTES);
 #pragma unroll
-          for (int hh = 0; hh < NH; ++hh) {
-            tma_load_4d(kd + hh * HALF, &tmk, bar, hh * 64, w.g, tok, plane);
-            tma_load_4d(vd + hh * HALF, &tmv, bar, hh * 64, w.g, tok, plane);
+            for (int hh = 0; hh < NH; ++hh) {
+              tma_load_4d(kd + hh * HALF, &tmk, bar, hh * 64, w.g, tok, plane);
+              tma_load_4d(vd + hh * HALF, &tmv, bar, hh * 64, w.g, tok, plane);
+            }
+          }
+          if (fix) {
+            ok = mbar_wait_warp(b_kvland + 8 * s, (land_par >> s) & 1u, a.st, 0x202u, a.wait_ns);
+            land_par ^= 1u << s;
+            if (ok) {
+              const int per_h = (BLK - r0) * 8;  // 16-byte pieces per 64-dim atom
+              uint8_t* vb = smem + (vd - sq);
+              for (int x = lane; x < per_h * NH; x += 32) {
+                const int hh = x / per_h, rem = x - hh * per_h;
+                *reinterpret_cast<uint4*>(vb + hh * HALF + (r0 + rem / 8) * 128 + (rem % 8) * 16) =
+                    make_uint4(0, 0, 0, 0);
+              }
+              fence_proxy_async_smem();
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(b_kvfull + 8 * s);
+          }
           }
         }
-        if (fix) {
-          ok = mbar_wait_warp(b_kvland + 8 * s, (land_par >> s) & 1u, a.st, 0x202u, a.wait_ns);
-          land_par ^= 1u << s;
-          if (ok) {
-            const int per_h = (BLK - r0) * 8;  // 16-byte pieces per 64-dim atom
-            uint8_t* vb = smem + (vd - sq);
-            for (int x = lane; x < per_h * NH; x += 32) {
-              const int hh = x / per_h, rem = x - hh * per_h;
-              *reinterpret_cast<uint4*>(vb + hh * HALF + (r0 + rem / 8) * 128 + (rem % 8) * 16) =
-                  make_uint4(0, 0, 0, 0);
+        // this warp's share of the tile's Q loads
+        const int qb = idx % NQ;
+        if (idx >= NQ && q_ok)
+          q_ok = mbar_wait_warp(b_qempty + 8 * qb, ((idx / NQ) - 1) & 1, a.st, 0x20au, a.wait_ns);
+        const int total = NH * nq;
+        const int mine = q_ok ? (total - gi + 2) / 3 : 0;
+        const uint32_t bar = b_qfull + 8 * qb;
+        if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)mine * rows_bytes);
+        __syncwarp();
+        if (q_ok) {
+#pragma unroll
+          for (int k = 0; k < 3; ++k) {
+            const int o = gi + 3 * (lane + 32 * k);
+            if (o < total) {
+              const int qi = o / NH, hh = o % NH;
+              tma_load_4d(sq + qb * QB + hh * (kRows * 128u) + qi * rows_bytes, &tmq, bar, hh * 64,
+                          qg * a.G, tq[k], qbb);
             }
-            fence_proxy_async_smem();
           }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(b_kvfull + 8 * s);
+        }
+        if (idx + 1 < n) {
+          const int tile = tile0 + idx + 1;
+          new_block = w.advance(a, tile);
+          nq = w.count(a, tile);
+          qg = w.g;
+          qbb = w.b;
+          load_t(w.first(a, tile), nq, tq);
         }
       }
-      // drain: the last two stages are released once their products complete
-      for (int u = max(0, use - 1); u <= use; ++u)
-        mbar_wait_warp(b_kvempty + 8 * (u & 1), (u >> 1) & 1, a.st, 0x203u, a.wait_ns);
+      if (kv_role) {
+        // drain: the last two stages are released once their products complete
+        for (int u = max(0, use - 1); u <= use; ++u)
+          mbar_wait_warp(b_kvempty + 8 * (u & 1), (u >> 1) & 1, a.st, 0x203u, a.wait_ns);
+      }
     }
   } else if (warp == kWarpMma) {
     // ----------------------------------------------- MMA issue (one thread)
@@ -495,56 +550,6 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         }
         tc::commit(b_done);
         mbar_wait_bounded(b_done, 0, a.st, 0x209u, a.wait_ns);
-      }
-    }
-  } else if (warp == kWarpGather || warp == kWarpGather + 1) {
-    // -------------------------------------------------------------- Q gather
-    // One TMA load per (query, 64-dim atom) brings the query's G heads, i.e. G
-    // consecutive tile rows, into the swizzled operand layout.  Two warps share
-    // the loads (one atom each, or alternate queries when d = 64); the query
-    // positions of the next tile are read while the current one is issued.
-    tc::regs_dec<kRegsLoad>();
-    if (n > 0) {
-      w.seek(a, tile0);
-      const int gw = warp - kWarpGather;
-      if (lane == 0) prefetch_tensormap(&tmq);
-      const uint32_t rows_bytes = (uint32_t)a.G * 128u;
-      // query positions of a tile's (at most 128) queries: query 32 k + lane in tq[k]
-      auto load_t = [&](int first, int nq, int (&tq)[4]) {
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-          tq[k] = 32 * k + lane < nq ? __ldg(&a.entries[first + 32 * k + lane].y) : 0;
-      };
-      int first = w.first(a, tile0), nq = w.count(a, tile0), b = w.b, g = w.g;
-      int tq[4];
-      load_t(first, nq, tq);
-      const int hh = NH == 2 ? gw : 0;
-      bool ok = true;
-      for (int idx = 0; idx < n; ++idx) {
-        const int qb = idx % NQ;
-        if (idx >= NQ && ok)
-          ok = mbar_wait_warp(b_qempty + 8 * qb, ((idx / NQ) - 1) & 1, a.st, 0x20au, a.wait_ns);
-        const int mine = !ok ? 0 : NH == 2 ? nq : (nq + 1 - gw) / 2;  // loads of this warp
-        const uint32_t bar = b_qfull + 8 * qb, qd = sq + qb * QB + hh * (kRows * 128u);
-        if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)mine * rows_bytes);
-        __syncwarp();
-        if (ok) {
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const int qi = 32 * k + lane;
-            if (qi < nq && (NH == 2 || (qi & 1) == gw))
-              tma_load_4d(qd + qi * rows_bytes, &tmq, bar, hh * 64, g * a.G, tq[k], b);
-          }
-        }
-        if (idx + 1 < n) {
-          const int tile = tile0 + idx + 1;
-          w.advance(a, tile);
-          first = w.first(a, tile);
-          nq = w.count(a, tile);
-          b = w.b;
-          g = w.g;
-          load_t(first, nq, tq);
-        }
       }
     }
   } else if (wg < 3) {
