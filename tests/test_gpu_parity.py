@@ -87,6 +87,11 @@ SMALL_CASES = [
             block=128, topk=3, causal=True, seed=112, len_range=(300, 700)),
     Problem("prefill_kv_d64_b64", batch=1, n_q=1500, max_kv=1500, H=16, h=1, d=64, d_idx=128,
             block=64, topk=5, causal=True, force_own=True, seed=113),
+    # groups of 8 heads: the combine takes one warp per (query, group)
+    Problem("prefill_kv_g8_d64", batch=2, n_q=600, max_kv=900, H=16, h=2, d=64, d_idx=64,
+            block=64, topk=6, causal=True, seed=114),
+    Problem("prefill_kv_g8_d128", batch=1, n_q=777, max_kv=777, H=8, h=1, d=128, d_idx=128,
+            block=128, topk=3, causal=True, force_own=True, seed=115),
     Problem("decode_many_splits", batch=2, n_q=1, max_kv=65536, H=64, h=8, d=128, d_idx=128,
             block=64, topk=600, causal=True, seed=109, len_range=(40000, 65536)),
 ]
