@@ -40,10 +40,12 @@ L2_BYTES = 126 * 2**20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # Per-launch DRAM traffic (read + write bytes) of the dominant kernel, from one ncu
-# capture (profiles/sparse_attn_stream_decode128k_b4.md: batch 4, 134.46 MB read +
-# 3.49 MB written, scaled by 4 to the batch of 16, the work growing in proportion).
-# Absent entries report null; an entry is removed when its kernel changes.
-TRAFFIC = {("decode_128k", "attn"): 4 * (134.462208e6 + 3.493888e6)}
+# capture at batch 4 scaled by 4 to the batch of 16 (the work grows in proportion):
+# profiles/sparse_attn_stream_decode128k_b4.md (134.46 MB read + 3.49 MB written) and
+# profiles/index_scan_decode128k_b4.md (134.26 MB read + 3.81 MB written).  Absent
+# entries report null; an entry is removed when its kernel changes.
+TRAFFIC = {("decode_128k", "attn"): 4 * (134.462208e6 + 3.493888e6),
+           ("decode_128k", "select"): 4 * (134.258176e6 + 3.808768e6)}
 
 
 def load_peaks():
@@ -392,7 +394,12 @@ def run_ours(args, prob, world, rank, local):
     peaks, peak_kind = load_peaks()
     dom = "attn" if attn_ms >= sel_ms else "select"
     dom_ms = attn_ms if dom == "attn" else sel_ms
-    kernel = {"attn": "sparse_attn_kernel (+combine)", "select": "index_scan_kernel (+topk)"}[dom]
+    if prob.is_decode:
+        kernel = {"attn": "sparse_attn_stream_kernel",
+                  "select": "index_scan_decode_kernel (+topk)"}[dom]
+    else:
+        kernel = {"attn": "kv_attn_kernel (+count/scan/scatter, combine)",
+                  "select": "index_score_tc_kernel (+topk)"}[dom]
     if prob.is_decode:
         roof = {"bound": "hbm", "achieved": units[dom] / (dom_ms * 1e-3) / 1e9,
                 "peak": peaks["hbm_gbs"], "unit": "GB/s"}
