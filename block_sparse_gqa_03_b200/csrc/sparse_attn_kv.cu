@@ -23,15 +23,18 @@
 // CTA roles (persistent CTAs, each a contiguous share of the chunk's tiles), four
 // warpgroups with registers moved from the first and last to the softmax ones:
 //   warp 0        TMA producer of K and V (a new load only when the block changes;
-//                 V rows past the sequence end are zeroed after the load lands);
-//   warp 1        tensor-memory allocation and the thread issuing all MMAs: S of
-//                 tile i, then O of tile i - 2, so that a softmax warpgroup finds
-//                 its next scores computed;
-//   warps 2-3     gather the tile's Q rows with TMA, one load per (query, 64-dim
-//                 atom) bringing the query's G heads into the swizzled layout;
+//                 V rows past the sequence end are zeroed after the load lands),
+//                 and a third of the Q gather;
+//   warp 1        tensor-memory allocation and the thread issuing all MMAs: S and
+//                 O = P V as two in-order streams, each issued as soon as its
+//                 inputs are ready;
+//   warps 0, 2-3  gather the tile's Q rows with TMA, one load per (query, 64-dim
+//                 atom) bringing the query's G heads into the swizzled layout, the
+//                 loads dealt round-robin to the three warps;
 //   warps 4-11    two softmax warpgroups taking tiles in turn, one thread per tile
 //                 row, each owning one P region in tensor memory;
-//   warps 12-15   output warpgroup: O / l from tensor memory to the partials.
+//   warps 12-15   output warpgroup: O / l from tensor memory to the partials
+//                 (staged per warp in shared memory, written by TMA stores).
 // Buffers: 2-4 Q tiles (released when S is computed), 2 K/V stages, and in tensor
 // memory 3-4 slots, each holding a tile's S and then its O, plus the two P
 // regions.  Every wait is bounded.
