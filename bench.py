@@ -74,10 +74,12 @@ def dist_setup(args):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """The largest of the ranks' values (step times are reported as the slowest rank's)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
