@@ -231,31 +231,60 @@ struct WarpState {
   }
 };
 
-// Merge of NC warp states for tile row `row` and dim `dim`: normalised output
-// and natural-log LSE (-inf and 0 when no key was seen).
+// Merge of NC warp states for tile row `row`, dims [dim, dim + 4) (dim a
+// multiple of 4): normalised output and natural-log LSE (-inf and 0 when no key
+// was seen).  The warps' weights are computed once for the four dims.
 template <int D, int NC>
-__device__ __forceinline__ void merge_warps(const float* mo, const float* mm, const float* ml,
-                                            int gr, int row, int dim, float& val, float& lsev) {
+__device__ __forceinline__ void merge_warps4(const float* mo, const float* mm, const float* ml,
+                                             int gr, int row, int dim, float4& val, float& lsev) {
   const float ninf = neg_inf();
   float M = ninf;
 #pragma unroll
   for (int w = 0; w < NC; ++w) M = fmaxf(M, mm[w * 16 + row]);
-  val = 0.f;
+  val = make_float4(0.f, 0.f, 0.f, 0.f);
   lsev = ninf;
   if (M == ninf) return;
-  float wsum = 0.f, acc = 0.f;
+  float wsum = 0.f;
+  float4 acc = val;
 #pragma unroll
   for (int w = 0; w < NC; ++w) {
     const float f = exp2f(mm[w * 16 + row] - M);
     wsum += f * ml[w * 16 + row];
-    acc += f * mo[(w * gr + row) * D + dim];
+    const float4 o = *reinterpret_cast<const float4*>(mo + (w * gr + row) * D + dim);
+    acc.x += f * o.x;
+    acc.y += f * o.y;
+    acc.z += f * o.z;
+    acc.w += f * o.w;
   }
-  val = acc / wsum;
+  val = make_float4(acc.x / wsum, acc.y / wsum, acc.z / wsum, acc.w / wsum);
   lsev = (M + log2f(wsum)) * kLn2;
+}
+
+// Four consecutive bf16 outputs of head hq (one 8-byte store when aligned).
+__device__ __forceinline__ void store_out4(const AttnArgs& a, const RowGeo& rg, int hq, int dim,
+                                           const float4& v) {
+  uint16_t* p = a.out + rg.b * a.o_s0 + (int64_t)rg.t * a.o_s1 + (int64_t)hq * a.o_s2 + dim;
+  const uint32_t lo = pack_bf16(v.x, v.y), hi = pack_bf16(v.z, v.w);
+  if ((reinterpret_cast<uintptr_t>(p) & 7u) == 0) {
+    *reinterpret_cast<uint2*>(p) = make_uint2(lo, hi);
+  } else {
+    p[0] = (uint16_t)lo;
+    p[1] = (uint16_t)(lo >> 16);
+    p[2] = (uint16_t)hi;
+    p[3] = (uint16_t)(hi >> 16);
+  }
 }
 
 __device__ __forceinline__ void consumer_sync(int nthreads) {
   asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
+}
+
+// Named barrier `id` over `nthreads` threads: arrive without waiting, or wait.
+__device__ __forceinline__ void named_arrive(int id, int nthreads) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+__device__ __forceinline__ void named_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 // Producer: streams the K and V tiles of list entries [0, n) into the stage ring.
@@ -320,7 +349,18 @@ __device__ __forceinline__ int compact_ids(const AttnArgs& a, int64_t s0, int64_
                                            int32_t* glist, int lane) {
   constexpr int PF = 8;  // 32-slot groups whose ids are loaded together
   const unsigned lt = (1u << lane) - 1u;
-  // visible-token limit of rows row0 .. row0 + 31, one per lane
+  // Slot i belongs to row row0 + (i - first) / topk; the range is one CTA's
+  // list (at most list_cap slots), so the offsets fit 32 bits.
+  const int64_t first = row0 * a.topk;
+  int ids[PF];
+  auto load_ids = [&](int64_t base) {
+#pragma unroll
+    for (int k = 0; k < PF; ++k) {
+      const int64_t i = base + k * 32 + lane;
+      ids[k] = i < s1 ? __ldg(a.ids + i) : -1;
+    }
+  };
+  load_ids(s0);  // issued before the row geometry: the two loads overlap
   const int64_t span = (s1 - 1) / a.topk - row0 + 1;
   const int nrows = span < 32 ? (int)span : 32;
   // visible-token limit, head and sequence of rows row0 .. row0 + 31, one per lane
@@ -329,20 +369,15 @@ __device__ __forceinline__ int compact_ids(const AttnArgs& a, int64_t s0, int64_
   if (lane < nrows) geo_l = row_geo(a, row0 + lane);
   int n = 0;
   for (int64_t base = s0; base < s1; base += 32 * PF) {
-    int ids[PF];
-#pragma unroll
-    for (int k = 0; k < PF; ++k) {
-      const int64_t i = base + k * 32 + lane;
-      ids[k] = i < s1 ? __ldg(a.ids + i) : -1;
-    }
+    if (base != s0) load_ids(base);
 #pragma unroll
     for (int k = 0; k < PF; ++k) {
       if (base + k * 32 >= s1) break;
       const int64_t i = base + k * 32 + lane;
       const int beta = ids[k];
-      const int64_t rowg = i < s1 ? i / a.topk : row0;
-      const int64_t rr = rowg - row0;
-      const int src = rr < 31 ? (int)rr : 31;
+      const int rr = i < s1 ? (int)(i - first) / a.topk : 0;
+      const int64_t rowg = row0 + rr;
+      const int src = rr < 31 ? rr : 31;
       int lim = __shfl_sync(0xffffffffu, geo_l.lim, src);
       int g = __shfl_sync(0xffffffffu, geo_l.g, src);
       int b = __shfl_sync(0xffffffffu, geo_l.b, src);
@@ -358,7 +393,7 @@ __device__ __forceinline__ int compact_ids(const AttnArgs& a, int64_t s0, int64_
       const unsigned msk = __ballot_sync(0xffffffffu, keep);
       if (keep) {
         const int at = n + __popc(msk & lt);
-        list[at] = beta | (int)(rr << 16);
+        list[at] = beta | (rr << 16);
         glist[at] = g;
         plist[at] = a.pg.table != nullptr ? (int)kv_page(a.pg, b, beta, a.st) : b;
       }
@@ -443,13 +478,13 @@ __global__ void __launch_bounds__(5 * 32, 1)
   float* ml = mm + NC * 16;
   ws.stash(mo, mm, ml, warp, lane, a.G);
   consumer_sync(NC * 32);
-  for (int x = tid; x < a.G * D; x += NC * 32) {
-    const int row = x / D, dim = x % D;
-    float val, lsev;
-    merge_warps<D, NC>(mo, mm, ml, a.G, row, dim, val, lsev);
+  for (int x = tid; x < a.G * (D / 4); x += NC * 32) {
+    const int row = x / (D / 4), dim = (x % (D / 4)) * 4;
+    float4 val;
+    float lsev;
+    merge_warps4<D, NC>(mo, mm, ml, a.G, row, dim, val, lsev);
     const int hq = rg.g * a.G + row;
-    a.out[rg.b * a.o_s0 + (int64_t)rg.t * a.o_s1 + (int64_t)hq * a.o_s2 + dim] =
-        __bfloat16_as_ushort(__float2bfloat16_rn(val));
+    store_out4(a, rg, hq, dim, val);
     if (dim == 0 && a.lse) a.lse[(int64_t)rg.bt * a.H + hq] = lsev;
   }
 }
@@ -484,34 +519,36 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1)
   if (s0 >= s1) return;
   const int64_t r0 = s0 / a.topk, r1 = (s1 - 1) / a.topk;
 
-  if (tid == 0) {
-    for (int s = 0; s < a.stages; ++s) {
-      mbar_init(full0 + 8 * s, 1);
-      mbar_init(empty0 + 8 * s, min(NC, nsub));
+  if (warp == NC) {
+    // The producer warp sets up the stage barriers, builds the list and starts
+    // streaming at once; the arrive on barrier 2 publishes both to the consumers.
+    // After an earlier timeout the kernel does nothing; the status load is issued
+    // first so that its latency overlaps the compaction.
+    if (lane == 0) {
+      for (int s = 0; s < a.stages; ++s) {
+        mbar_init(full0 + 8 * s, 1);
+        mbar_init(empty0 + 8 * s, min(NC, nsub));
+      }
+      fence_mbar_init();
     }
-    fence_mbar_init();
+    const bool skip = status_failed(a.st);
+    const int n = compact_ids(a, s0, s1, r0, list, plist, glist, lane);
+    if (lane == 0) *n_list = skip ? -1 : n;
+    __syncwarp();
+    named_arrive(2, (NC + 1) * 32);
+    if (lane == 0 && !skip && n > 0)
+      produce<D>(a, &tmk, &tmv, list, plist, glist, n, sbase, full0, empty0);
+    return;
   }
   // the consumers load their first row's queries while the list is built
   WarpState<D> ws;
   int64_t cur = r0;
   RowGeo rg = row_geo(a, cur);
-  if (warp == NC) {
-    // after an earlier timeout the kernel does nothing; the status load is issued
-    // first so that its latency overlaps the compaction
-    const bool skip = status_failed(a.st);
-    const int n = compact_ids(a, s0, s1, r0, list, plist, glist, lane);
-    if (lane == 0) *n_list = skip ? -1 : n;
-  } else {
-    ws.reset();
-    ws.load_q(a, rg, lane);
-  }
-  __syncthreads();
+  ws.reset();
+  ws.load_q(a, rg, lane);
+  named_sync(2, (NC + 1) * 32);
   const int n = *n_list;
   if (n < 0) return;
-  if (warp == NC) {
-    if (lane == 0 && n > 0) produce<D>(a, &tmk, &tmv, list, plist, glist, n, sbase, full0, empty0);
-    return;
-  }
   bool failed = false;
 
   // Ends the segment of row `cur` held by this CTA: merge the warps, then write
@@ -524,30 +561,36 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1)
     const int64_t c_last = ((cur + 1) * a.topk - 1) / a.per;
     const int nseg = (int)(c_last - c_first + 1);
     const int seg = (int)(c - c_first);
-    for (int x = tid; x < a.G * D; x += NC * 32) {
-      const int row = x / D, dim = x % D;
-      float val, lsev;
-      merge_warps<D, NC>(mo, mm, ml, a.G, row, dim, val, lsev);
+    for (int x = tid; x < a.G * (D / 4); x += NC * 32) {
+      const int row = x / (D / 4), dim = (x % (D / 4)) * 4;
+      float4 val;
+      float lsev;
+      merge_warps4<D, NC>(mo, mm, ml, a.G, row, dim, val, lsev);
       const int hq = rg.g * a.G + row;
       if (nseg == 1) {
-        a.out[rg.b * a.o_s0 + (int64_t)rg.t * a.o_s1 + (int64_t)hq * a.o_s2 + dim] =
-            __bfloat16_as_ushort(__float2bfloat16_rn(val));
+        store_out4(a, rg, hq, dim, val);
         if (dim == 0 && a.lse) a.lse[(int64_t)rg.bt * a.H + hq] = lsev;
       } else {
         const int64_t pr = ((int64_t)rg.bt * a.H + hq) * a.smax + seg;
-        a.part_o[pr * D + dim] = val;
+        *reinterpret_cast<float4*>(a.part_o + pr * D + dim) = val;
         if (dim == 0) a.part_lse[pr] = lsev;
       }
     }
     if (nseg > 1) {
-      __threadfence();
+      // One thread publishes the CTA's partial (its stores ordered before the
+      // fence by the barrier) and learns whether it is the row's last; its
+      // second fence orders the other CTAs' partials before the loads below.
       consumer_sync(NC * 32);
-      if (tid == 0) *flag = atomicAdd(&a.counters[cur], 1);
+      if (tid == 0) {
+        __threadfence();
+        const int f = atomicAdd(&a.counters[cur], 1);
+        __threadfence();
+        *flag = f;
+      }
       consumer_sync(NC * 32);
       if (*flag == nseg - 1 && nseg <= NC) {
         // Last CTA of the row: stage the row's partials in the (now free) merge
         // buffer with independent loads, then merge them from shared memory.
-        __threadfence();
         float* so = mo;              // [G][nseg][D]
         float* sl = mo + NC * a.G * D;  // [G][nseg], over the free max/sum arrays
         const int64_t pr_g = ((int64_t)rg.bt * a.H + rg.g * a.G) * a.smax;
@@ -563,30 +606,34 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1)
         for (int y = tid; y < a.G * nseg; y += NC * 32)
           sl[y] = __ldcg(a.part_lse + pr_g + (int64_t)(y / nseg) * a.smax + y % nseg);
         consumer_sync(NC * 32);
-        for (int x = tid; x < a.G * D; x += NC * 32) {
-          const int row = x / D, dim = x % D;
+        for (int x = tid; x < a.G * (D / 4); x += NC * 32) {
+          const int row = x / (D / 4), dim = (x % (D / 4)) * 4;
           const int hq = rg.g * a.G + row;
           const float ninf = neg_inf();
           float M = ninf;
           for (int sp = 0; sp < nseg; ++sp) M = fmaxf(M, sl[row * nseg + sp]);
-          float val = 0.f, lsev = ninf;
+          float4 val = make_float4(0.f, 0.f, 0.f, 0.f);
+          float lsev = ninf;
           if (M != ninf) {
-            float den = 0.f, acc = 0.f;
+            float den = 0.f;
+            float4 acc = val;
             for (int sp = 0; sp < nseg; ++sp) {
               const float w = exp2f((sl[row * nseg + sp] - M) * kLog2e);
               den += w;
-              acc += w * so[(row * nseg + sp) * D + dim];
+              const float4 o = *reinterpret_cast<const float4*>(so + (row * nseg + sp) * D + dim);
+              acc.x += w * o.x;
+              acc.y += w * o.y;
+              acc.z += w * o.z;
+              acc.w += w * o.w;
             }
-            val = acc / den;
+            val = make_float4(acc.x / den, acc.y / den, acc.z / den, acc.w / den);
             lsev = M + log2f(den) * kLn2;
           }
-          a.out[rg.b * a.o_s0 + (int64_t)rg.t * a.o_s1 + (int64_t)hq * a.o_s2 + dim] =
-              __bfloat16_as_ushort(__float2bfloat16_rn(val));
+          store_out4(a, rg, hq, dim, val);
           if (dim == 0 && a.lse) a.lse[(int64_t)rg.bt * a.H + hq] = lsev;
         }
       } else if (*flag == nseg - 1) {
         // more segments than the merge buffer holds: merge from global memory
-        __threadfence();
         for (int x = tid; x < a.G * D; x += NC * 32) {
           const int row = x / D, dim = x % D;
           const int hq = rg.g * a.G + row;
