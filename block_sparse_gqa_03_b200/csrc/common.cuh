@@ -127,6 +127,14 @@ inline cudaError_t launch_pdl(void (*kernel)(K...), dim3 grid, dim3 block, size_
   return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
+// Named barrier `id` over `nthreads` threads: arrive without waiting, or wait.
+__device__ __forceinline__ void named_arrive(int id, int nthreads) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+__device__ __forceinline__ void named_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 __device__ __forceinline__ void fence_mbar_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }

@@ -16,7 +16,16 @@
 // straight into MMA fragments: each thread loads 8 consecutive dims of a token
 // row, and the same dim permutation is applied to the index-query fragments,
 // which leaves the dot products unchanged.
+//
+// Decode with d_idx 64 or 128 takes a persistent streaming scan instead: one
+// CTA per SM owns an equal, contiguous share of the (sequence, block) items; a
+// producer lane brings each item's K_idx block into a ring of shared-memory
+// stages with TMA (128-byte swizzle, waits bounded), and consumer warp w takes
+// items w, w + 8, ...: token rows as A fragments by ldmatrix, the sequence's h
+// index queries as B fragments held in registers, the block max reduced over
+// the warp.  The ring keeps a steady stream of bulk copies in flight per SM.
 #include "kernels.h"
+#include "sm100.cuh"
 
 namespace msa {
 namespace {
@@ -232,11 +241,284 @@ cudaError_t run_scan(const ScanArgs& a, int batch, cudaStream_t stream) {
   return launch_pdl(index_scan_kernel<DI, NT>, grid, dim3(kScanWarps * 32), 0, stream, a);
 }
 
+
+// ------------------------------------------------ decode: streaming TMA scan
+struct StreamScanArgs {
+  const uint16_t* q_idx;
+  int64_t qi_s0, qi_s2;
+  const int32_t* seq_lens;
+  int batch, max_kv, h, block, nblk, stages;
+  uint32_t stage_bytes;
+  float* scores;
+  int fill_tail;
+  DeviceStatus* st;
+  uint64_t wait_ns;
+  KvPages pg;
+};
+
+constexpr int kStreamScanWarps = 8;  // consumer warps; one more warp produces
+
+__device__ __forceinline__ int seq_blocks(const StreamScanArgs& a, int b) {
+  return (kv_length(a.seq_lens, b, a.max_kv, a.st) + a.block - 1) / a.block;
+}
+
+// B fragments of sequence b's index queries: column c = nt*8 + r is group c,
+// k-step ks holds dims [16ks + 2q, +2) and [16ks + 8 + 2q, +2).
+template <int DI, int NT>
+__device__ __forceinline__ void load_query_frags(const StreamScanArgs& a, int b, int r, int q,
+                                                 uint32_t (&bf)[NT][DI / 16][2]) {
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    const int g = nt * 8 + r;
+    const bool ok = g < a.h;
+    const uint16_t* src = a.q_idx + b * a.qi_s0 + (int64_t)g * a.qi_s2 + 2 * q;
+#pragma unroll
+    for (int ks = 0; ks < DI / 16; ++ks) {
+      bf[nt][ks][0] = ok ? *reinterpret_cast<const uint32_t*>(src + 16 * ks) : 0u;
+      bf[nt][ks][1] = ok ? *reinterpret_cast<const uint32_t*>(src + 16 * ks + 8) : 0u;
+    }
+  }
+}
+
+template <int DI, int NT>
+__global__ void __launch_bounds__((kStreamScanWarps + 1) * 32, 1)
+    index_scan_stream_kernel(const __grid_constant__ CUtensorMap tmk, StreamScanArgs a) {
+  grid_dep_wait();
+  grid_dep_launch();
+  constexpr int NW = kStreamScanWarps;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const int S = a.stages;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)S * a.stage_bytes);
+  int2* info = reinterpret_cast<int2*>(bars + 2 * S);  // [S] (sequence, block) of a stage
+  int* n_items = reinterpret_cast<int*>(info + S);
+  const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + S);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t box_bytes = (uint32_t)a.block * 128u;
+
+  if (warp == NW) {
+    // Producer warp: barriers, this CTA's share of the items (counted over the
+    // sequences' block counts), then one lane streams them.
+    if (lane == 0) {
+      for (int s = 0; s < S; ++s) {
+        mbar_init(full0 + 8 * s, 1);
+        mbar_init(empty0 + 8 * s, 1);
+      }
+      fence_mbar_init();
+      prefetch_tensormap(&tmk);
+    }
+    const bool skip = status_failed(a.st);
+    int total = 0;
+    for (int b = lane; b < a.batch; b += 32) total += seq_blocks(a, b);
+    total = (int)__reduce_add_sync(0xffffffffu, (unsigned)total);
+    const int per = (total + (int)gridDim.x - 1) / (int)gridDim.x;
+    const int i0 = (int)blockIdx.x * per;
+    const int n = max(0, min(total, i0 + per) - i0);
+    // first item: the sequence whose block range holds i0
+    int b0 = 0, beta0 = 0, carry = 0;
+    bool found = false;
+    for (int base = 0; base < a.batch && !found; base += 32) {
+      const int b = base + lane;
+      const int nb = b < a.batch ? seq_blocks(a, b) : 0;
+      int inc = nb;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += v;
+      }
+      const int excl = carry + inc - nb;
+      const unsigned hit = __ballot_sync(0xffffffffu, nb > 0 && i0 >= excl && i0 < excl + nb);
+      if (hit) {
+        const int src = __ffs(hit) - 1;
+        b0 = base + src;
+        beta0 = i0 - __shfl_sync(0xffffffffu, excl, src);
+        found = true;
+      }
+      carry += __shfl_sync(0xffffffffu, inc, 31);
+    }
+    if (lane == 0) *n_items = skip ? -1 : n;
+    __syncwarp();
+    named_arrive(2, (NW + 1) * 32);
+    if (lane != 0 || skip || n == 0) return;
+    int b = b0, beta = beta0, nb = seq_blocks(a, b0);
+    int issued = 0;
+    for (int k = 0; k < n; ++k) {
+      const int s = k % S;
+      if (k >= S && !mbar_wait_bounded(empty0 + 8 * s, ((k / S) - 1) & 1, a.st, 0x201u, a.wait_ns))
+        break;
+      info[s] = make_int2(b, beta);
+      int tok, plane;
+      kv_block_coords(a.pg, b, beta, a.block, a.st, tok, plane);
+      const uint32_t full = full0 + 8 * s, dst = sbase + (uint32_t)s * a.stage_bytes;
+      mbar_arrive_expect_tx(full, a.stage_bytes);
+#pragma unroll
+      for (int hh = 0; hh < DI / 64; ++hh) tma_load_3d(dst + hh * box_bytes, &tmk, full, hh * 64, tok, plane);
+      issued = k + 1;
+      if (++beta == nb) {
+        beta = 0;
+        do {
+          ++b;
+          nb = b < a.batch ? seq_blocks(a, b) : 1;
+        } while (nb == 0);
+      }
+    }
+    // before leaving, wait (bounded) for the copies still in flight
+    for (int k = max(0, issued - S); k < issued; ++k)
+      mbar_wait_bounded(full0 + 8 * (k % S), (k / S) & 1, a.st, 0x203u, a.wait_ns);
+    return;
+  }
+
+  named_sync(2, (NW + 1) * 32);
+  const int n = *n_items;
+  if (n < 0) return;
+  const int r = lane >> 2, q = lane & 3;
+  const float ninf = -__int_as_float(0x7f800000);
+  uint32_t bf[NT][DI / 16][2];
+  int cur_b = -1, L = 0;
+  for (int k = warp; k < n; k += NW) {
+    const int s = k % S;
+    if (!mbar_wait_warp(full0 + 8 * s, (k / S) & 1, a.st, 0x202u, a.wait_ns)) break;
+    const int2 it = info[s];
+    if (it.x != cur_b) {
+      cur_b = it.x;
+      L = kv_length(a.seq_lens, cur_b, a.max_kv, a.st);
+      load_query_frags<DI, NT>(a, cur_b, r, q, bf);
+    }
+    const uint32_t base = sbase + (uint32_t)s * a.stage_bytes;
+    float cm[NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) cm[nt][0] = cm[nt][1] = ninf;
+    for (int mt = 0; mt < a.block / 16; ++mt) {
+      float acc[NT][4];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+      const uint32_t row = (uint32_t)(mt * 16 + (lane & 15));
+#pragma unroll
+      for (int ks = 0; ks < DI / 16; ++ks) {
+        uint32_t a0, a1, a2, a3;
+        ldmatrix_x4(base + (uint32_t)(ks >> 2) * box_bytes +
+                        swz128(row, (uint32_t)((ks & 3) * 2 + (lane >> 4))),
+                    a0, a1, a2, a3);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+          mma_bf16_16816(acc[nt], a0, a1, a2, a3, bf[nt][ks][0], bf[nt][ks][1]);
+      }
+      const int jl = it.y * a.block + mt * 16 + r, jh = jl + 8;
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          cm[nt][e] = fmaxf(cm[nt][e], jl < L ? acc[nt][e] : ninf);
+          cm[nt][e] = fmaxf(cm[nt][e], jh < L ? acc[nt][2 + e] : ninf);
+        }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty0 + 8 * s);
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        float v = cm[nt][e];
+        v = warp_max_xor(v, 4);
+        v = warp_max_xor(v, 8);
+        v = warp_max_xor(v, 16);
+        const int g = nt * 8 + 2 * q + e;
+        if (r == 0 && g < a.h) a.scores[((int64_t)it.x * a.h + g) * a.nblk + it.y] = v;
+      }
+  }
+  if (a.fill_tail) {
+    // blocks past each sequence's end: -inf, spread over every consumer thread
+    const int nthr = (int)gridDim.x * NW * 32;
+    const int gt = (int)blockIdx.x * NW * 32 + (int)threadIdx.x;
+    for (int b = 0; b < a.batch; ++b)
+      for (int beta = seq_blocks(a, b) + gt; beta < a.nblk; beta += nthr)
+        for (int g = 0; g < a.h; ++g) a.scores[((int64_t)b * a.h + g) * a.nblk + beta] = ninf;
+  }
+}
+
+template <int DI, int NT>
+cudaError_t run_stream_scan(const Shape& s, const uint16_t* k_idx, StreamScanArgs& a,
+                            cudaStream_t stream, bool& done) {
+  done = false;
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return cudaSuccess;
+  // contiguous [d_idx, token, batch], or a page pool [d_idx, token in page, page];
+  // one box is 64 dims x one block of tokens
+  const bool paged = s.pages.table != nullptr;
+  cuuint64_t dims[3] = {(cuuint64_t)DI, (cuuint64_t)(paged ? s.block : s.max_kv),
+                        (cuuint64_t)(paged ? s.pages.pages : s.batch)};
+  cuuint64_t str[2] = {(cuuint64_t)s.ki_s[1] * 2, (cuuint64_t)s.ki_s[0] * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)s.block, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUtensorMap tmk;
+  if (enc(&tmk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<uint16_t*>(k_idx), dims, str,
+          box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaSuccess;  // not expressible as a tensor map: the direct-load scan runs
+  a.stage_bytes = (uint32_t)DI * 2u * (uint32_t)s.block;
+  const size_t fixed = 1024 + 64;
+  const size_t cap = (size_t)max_smem_optin();
+  // Consumer warp w takes items w, w + NW, ... and item k uses stage k % S.  With
+  // S a multiple of NW every stage is only ever consumed by one warp, which has
+  // consumed the stage's previous fill itself before it waits on the next: a
+  // parity wait then never meets a phase two fills behind (a stage shared by
+  // several warps would let one warp pass the parity test on a fill that
+  // another warp's item has not completed).
+  const size_t fit = (cap - fixed) / (a.stage_bytes + 24);
+  const int nw = kStreamScanWarps;
+  a.stages = (int)(fit >= 2 * (size_t)nw ? 2 * nw : (fit >= (size_t)nw ? nw : 0));
+  if (a.stages == 0) return cudaSuccess;  // too few stages fit: the direct-load scan runs
+  const size_t smem = fixed + (size_t)a.stages * (a.stage_bytes + 24);
+  cudaError_t err = cudaFuncSetAttribute(index_scan_stream_kernel<DI, NT>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  done = true;
+  return launch_pdl(index_scan_stream_kernel<DI, NT>, dim3(num_sms()),
+                    dim3((kStreamScanWarps + 1) * 32), smem, stream, tmk, a);
+}
+
+// Decode scans that the streaming kernel covers; `done` is false when the
+// direct-load kernel must run instead.
+cudaError_t launch_stream_scan(const Shape& s, const uint16_t* q_idx, const uint16_t* k_idx,
+                               float* scores, bool fill_tail, DeviceStatus* st,
+                               cudaStream_t stream, bool& done) {
+  done = false;
+  if (s.n_q != 1 || s.h > 16 || (s.d_idx != 64 && s.d_idx != 128) || s.block < 16 ||
+      s.block > 128 || s.block % 16 != 0 || (int64_t)s.batch * s.nblk >= (1LL << 31))
+    return cudaSuccess;
+  StreamScanArgs a;
+  a.q_idx = q_idx;
+  a.qi_s0 = s.qi_s[0];
+  a.qi_s2 = s.qi_s[2];
+  a.seq_lens = s.seq_lens;
+  a.batch = s.batch;
+  a.max_kv = s.max_kv;
+  a.h = s.h;
+  a.block = s.block;
+  a.nblk = s.nblk;
+  a.scores = scores;
+  a.fill_tail = fill_tail ? 1 : 0;
+  a.st = st;
+  a.wait_ns = 4000000000ull;
+  a.pg = s.pages;
+  const bool two = s.h > 8;
+  if (s.d_idx == 128)
+    return two ? run_stream_scan<128, 2>(s, k_idx, a, stream, done)
+               : run_stream_scan<128, 1>(s, k_idx, a, stream, done);
+  return two ? run_stream_scan<64, 2>(s, k_idx, a, stream, done)
+             : run_stream_scan<64, 1>(s, k_idx, a, stream, done);
+}
+
 }  // namespace
 
 cudaError_t launch_index_scores(const Shape& s, const uint16_t* q_idx, const uint16_t* k_idx,
                                 float* scores, bool fill_tail, DeviceStatus* st,
                                 cudaStream_t stream) {
+  bool done = false;
+  const cudaError_t e = launch_stream_scan(s, q_idx, k_idx, scores, fill_tail, st, stream, done);
+  if (e != cudaSuccess || done) return e;
   ScanArgs a;
   a.q_idx = q_idx;
   a.k_idx = k_idx;

@@ -77,4 +77,11 @@ cudaError_t launch_wait_timeout_probe(DeviceStatus* st, uint64_t wait_ns, cudaSt
 int num_sms();
 int max_smem_optin();
 
+// cuTensorMapEncodeTiled from the driver (nullptr when the driver lacks it).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_fn();
+
 }  // namespace msa

@@ -279,14 +279,6 @@ __device__ __forceinline__ void consumer_sync(int nthreads) {
   asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
 }
 
-// Named barrier `id` over `nthreads` threads: arrive without waiting, or wait.
-__device__ __forceinline__ void named_arrive(int id, int nthreads) {
-  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-__device__ __forceinline__ void named_sync(int id, int nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-
 // Producer: streams the K and V tiles of list entries [0, n) into the stage ring.
 // Each entry is (block id in the low 16 bits, row offset in the high bits); the
 // row supplies the sequence and the KV head.  Waits are bounded; before leaving,
@@ -703,24 +695,6 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1)
 }
 
 // ------------------------------------------------------------ host helpers
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (fn == nullptr) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault,
-                                         &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(ptr);
-  }
-  return fn;
-}
-
 // K or V as a 4-D tensor [batch][token][kv head][dim], or for a paged cache
 // [page][token in page][kv head][dim]; one box is 64 dims x 1 head x `block`
 // tokens (128 bytes per row, 128-byte swizzle).

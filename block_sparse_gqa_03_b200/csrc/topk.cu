@@ -245,17 +245,23 @@ __global__ void __launch_bounds__(256, 3) topk_warp_kernel(TopkArgs a) {
   for (int i = m + lane; i < a.topk; i += 32) out[i] = -1;
 }
 
-// Sum over the CTA (NW warps); `buf` alternates between calls so one barrier
-// per call suffices.  Each warp reads the NW partial sums with one load per lane.
-template <int NW>
-__device__ __forceinline__ unsigned cta_sum(unsigned v, unsigned (*red)[32], int& buf) {
+// Sums over the CTA (NW warps) of W words per thread; `buf` alternates between
+// calls so one barrier per call suffices.  Each warp reads the NW partial sums
+// of a word with one load per lane.
+template <int NW, int W>
+__device__ __forceinline__ void cta_sums(unsigned (&v)[W], unsigned (*red)[2][32], int& buf) {
   const int lane = threadIdx.x & 31;
-  v = __reduce_add_sync(0xffffffffu, v);
-  if (lane == 0) red[buf][threadIdx.x >> 5] = v;
+#pragma unroll
+  for (int k = 0; k < W; ++k) v[k] = __reduce_add_sync(0xffffffffu, v[k]);
+  if (lane == 0) {
+#pragma unroll
+    for (int k = 0; k < W; ++k) red[buf][k][threadIdx.x >> 5] = v[k];
+  }
   __syncthreads();
-  const unsigned tot = __reduce_add_sync(0xffffffffu, lane < NW ? red[buf][lane] : 0u);
+#pragma unroll
+  for (int k = 0; k < W; ++k)
+    v[k] = __reduce_add_sync(0xffffffffu, lane < NW ? red[buf][k][lane] : 0u);
   buf ^= 1;
-  return tot;
 }
 
 // Exclusive prefix over the CTA in thread order.
@@ -276,16 +282,22 @@ __device__ __forceinline__ unsigned cta_exclusive_scan(unsigned v, unsigned* wsu
   return before + inc - v;
 }
 
-// One CTA of NT threads per row; thread i holds elements [i*E, i*E + E).  Counts
-// are CTA sums; warp 0 ranks the last bucket.
+// One CTA of NT threads per row; thread i holds elements [i*E, i*E + E), read
+// with 16-byte loads.  Each search step is one CTA sum (one barrier).  The last
+// bucket (at most 32 keys) is gathered in any order: T is a key value, so the
+// order among equal keys does not change it.  One more sum counts the keys above
+// and equal to T; only when some keys equal to T must be left out are they
+// ranked by id.
 template <int NT, int E>
 __global__ void __launch_bounds__(NT) topk_cta_kernel(TopkArgs a) {
+  static_assert(E % 4 == 0, "four keys per vector load");
   grid_dep_wait();
   grid_dep_launch();
   clear_words(a);
   constexpr int NW = NT / 32;
   __shared__ uint32_t cbuf[32];
-  __shared__ unsigned red[2][32];
+  __shared__ int ccount;
+  __shared__ unsigned red[2][2][32];
   __shared__ unsigned wsum[32];
   __shared__ uint32_t wmax[NW], wmin[NW];
   __shared__ uint32_t Ts;
@@ -299,16 +311,33 @@ __global__ void __launch_bounds__(NT) topk_cta_kernel(TopkArgs a) {
   if (m == ri.F) {
     for (int i = threadIdx.x; i < m; i += NT) out[i] = i;
   } else {
+    if (threadIdx.x == 0) ccount = 0;  // ordered before its use by the barriers below
     uint32_t key[E];
     uint32_t kmax = 0u, kmin = 0xffffffffu;
+    const bool vec = (reinterpret_cast<uintptr_t>(s) & 15u) == 0;
 #pragma unroll
-    for (int e = 0; e < E; ++e) {
-      const int i = i0 + e;
-      key[e] = i < ri.F ? order_key(s[i]) : 0u;
-      if (i == ri.own) key[e] = 0xffffffffu;
-      const bool vis = key[e] != 0u && key[e] != 0xffffffffu;
-      kmax = vis ? max(kmax, key[e]) : kmax;
-      kmin = vis ? min(kmin, key[e]) : kmin;
+    for (int v = 0; v < E / 4; ++v) {
+      const int i = i0 + 4 * v;
+      float f[4];
+      if (vec && i + 3 < a.nblk) {
+        const float4 x = __ldg(reinterpret_cast<const float4*>(s + i));
+        f[0] = x.x;
+        f[1] = x.y;
+        f[2] = x.z;
+        f[3] = x.w;
+      } else {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) f[u] = i + u < ri.F ? s[i + u] : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int e = 4 * v + u;
+        key[e] = i + u < ri.F ? order_key(f[u]) : 0u;
+        if (i + u == ri.own) key[e] = 0xffffffffu;
+        const bool vis = key[e] != 0u && key[e] != 0xffffffffu;
+        kmax = vis ? max(kmax, key[e]) : kmax;
+        kmin = vis ? min(kmin, key[e]) : kmin;
+      }
     }
     kmax = __reduce_max_sync(0xffffffffu, kmax);
     kmin = __reduce_min_sync(0xffffffffu, kmin);
@@ -327,21 +356,21 @@ __global__ void __launch_bounds__(NT) topk_cta_kernel(TopkArgs a) {
       Bucket r = bucket_start(kmax, kmin, ri.F - forced, forced);
       while (r.cnt > 32 && r.hi >= 0) {
         const uint32_t cand = r.prefix | (1u << r.hi);
-        unsigned c = 0;
+        unsigned c[1] = {0u};
 #pragma unroll
-        for (int e = 0; e < E; ++e) c += key[e] >= cand;
-        bucket_split(r, (int)cta_sum<NW>(c, red, buf), m);
+        for (int e = 0; e < E; ++e) c[0] += key[e] >= cand;
+        cta_sums<NW, 1>(c, red, buf);
+        bucket_split(r, (int)c[0], m);
       }
       if (r.cnt > 32) {
         T = r.prefix;  // every bit resolved: the remaining keys all equal T
       } else {
-        unsigned nu = 0;
-#pragma unroll
-        for (int e = 0; e < E; ++e) nu += in_bucket(key[e], r);
-        unsigned pos = cta_exclusive_scan<NW>(nu, wsum);
 #pragma unroll
         for (int e = 0; e < E; ++e)
-          if (in_bucket(key[e], r)) cbuf[pos++] = key[e];
+          if (in_bucket(key[e], r)) {
+            const int at = atomicAdd(&ccount, 1);
+            if (at < 32) cbuf[at] = key[e];  // r.cnt <= 32 keys are in the bucket
+          }
         __syncthreads();
         if (warp == 0) {
           const uint32_t ck = lane < r.cnt ? cbuf[lane] : 0u;
@@ -352,22 +381,35 @@ __global__ void __launch_bounds__(NT) topk_cta_kernel(TopkArgs a) {
         T = Ts;
       }
     }
-    unsigned gt = 0, eq = 0;
+    unsigned ge[2] = {0u, 0u};  // keys above T, keys equal to T
 #pragma unroll
     for (int e = 0; e < E; ++e) {
-      gt += key[e] > T;
-      eq += key[e] == T;
+      ge[0] += key[e] > T;
+      ge[1] += key[e] == T;
     }
-    const int need = m - (int)cta_sum<NW>(gt, red, buf);
-    unsigned eqr = cta_exclusive_scan<NW>(eq, wsum);
+    cta_sums<NW, 2>(ge, red, buf);
+    const int need = m - (int)ge[0];
     unsigned nsel = 0;
     bool sel[E];
+    if ((int)ge[1] <= need) {
+      // every key equal to T is taken (the usual case: T is unique)
 #pragma unroll
-    for (int e = 0; e < E; ++e) {
-      const bool is_eq = key[e] == T;
-      sel[e] = key[e] > T || (is_eq && (int)eqr < need);
-      eqr += is_eq;
-      nsel += sel[e];
+      for (int e = 0; e < E; ++e) {
+        sel[e] = key[e] >= T;
+        nsel += sel[e];
+      }
+    } else {
+      unsigned eq = 0;
+#pragma unroll
+      for (int e = 0; e < E; ++e) eq += key[e] == T;
+      unsigned eqr = cta_exclusive_scan<NW>(eq, wsum);
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        const bool is_eq = key[e] == T;
+        sel[e] = key[e] > T || (is_eq && (int)eqr < need);
+        eqr += is_eq;
+        nsel += sel[e];
+      }
     }
     unsigned pos = cta_exclusive_scan<NW>(nsel, wsum);
 #pragma unroll
