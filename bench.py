@@ -41,11 +41,11 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # Per-launch DRAM traffic (read + write bytes) of the dominant kernel, from one ncu
 # capture at batch 4 scaled by 4 to the batch of 16 (the work grows in proportion):
-# profiles/sparse_attn_stream_decode128k_b4.md (134.46 MB read + 3.49 MB written) and
-# profiles/index_scan_decode128k_b4.md (134.26 MB read + 3.81 MB written).  Absent
+# profiles/sparse_attn_stream_decode128k_b4.md (134.46 MB read + 3.43 MB written) and
+# profiles/index_scan_stream_decode128k_b4.md (134.27 MB read + 4.17 MB written).  Absent
 # entries report null; an entry is removed when its kernel changes.
-TRAFFIC = {("decode_128k", "attn"): 4 * (134.462208e6 + 3.493888e6),
-           ("decode_128k", "select"): 4 * (134.258176e6 + 3.808768e6)}
+TRAFFIC = {("decode_128k", "attn"): 4 * (134.456832e6 + 3.434752e6),
+           ("decode_128k", "select"): 4 * (134.271744e6 + 4.173568e6)}
 
 
 def load_peaks():
@@ -405,7 +405,7 @@ def run_ours(args, prob, world, rank, local):
     dom_ms = attn_ms if dom == "attn" else sel_ms
     if prob.is_decode:
         kernel = {"attn": "sparse_attn_stream_kernel",
-                  "select": "index_scan_decode_kernel (+topk)"}[dom]
+                  "select": "index_scan_stream_kernel (+topk)"}[dom]
     else:
         kernel = {"attn": "kv_attn_kernel (+count/scan/scatter, combine)",
                   "select": "index_score_tc_kernel (+topk)"}[dom]
