@@ -294,6 +294,7 @@ __global__ void __launch_bounds__((kStreamScanWarps + 1) * 32, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)S * a.stage_bytes);
   int2* info = reinterpret_cast<int2*>(bars + 2 * S);  // [S] (sequence, block) of a stage
   int* n_items = reinterpret_cast<int*>(info + S);
+  int4* coord = reinterpret_cast<int4*>(bars + 3 * S + 2);  // [32] next items: tok, plane, b, beta
   const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + S);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t box_bytes = (uint32_t)a.block * 128u;
@@ -341,29 +342,74 @@ __global__ void __launch_bounds__((kStreamScanWarps + 1) * 32, 1)
     if (lane == 0) *n_items = skip ? -1 : n;
     __syncwarp();
     named_arrive(2, (NW + 1) * 32);
-    if (lane != 0 || skip || n == 0) return;
-    int b = b0, beta = beta0, nb = seq_blocks(a, b0);
-    int issued = 0;
-    for (int k = 0; k < n; ++k) {
-      const int s = k % S;
-      if (k >= S && !mbar_wait_bounded(empty0 + 8 * s, ((k / S) - 1) & 1, a.st, 0x201u, a.wait_ns))
-        break;
-      info[s] = make_int2(b, beta);
-      int tok, plane;
-      kv_block_coords(a.pg, b, beta, a.block, a.st, tok, plane);
-      const uint32_t full = full0 + 8 * s, dst = sbase + (uint32_t)s * a.stage_bytes;
-      mbar_arrive_expect_tx(full, a.stage_bytes);
+    if (skip || n == 0) return;
+    int b = b0, beta = beta0, issued = 0;
+    bool failed = false;
+    if (a.pg.table == nullptr) {
+      // contiguous K_idx: lane 0 walks the items itself (no table loads)
+      if (lane != 0) return;
+      int nb = seq_blocks(a, b0);
+      for (int k = 0; k < n; ++k) {
+        const int s = k % S;
+        if (k >= S &&
+            !mbar_wait_bounded(empty0 + 8 * s, ((k / S) - 1) & 1, a.st, 0x201u, a.wait_ns))
+          break;
+        info[s] = make_int2(b, beta);
+        const uint32_t full = full0 + 8 * s, dst = sbase + (uint32_t)s * a.stage_bytes;
+        mbar_arrive_expect_tx(full, a.stage_bytes);
 #pragma unroll
-      for (int hh = 0; hh < DI / 64; ++hh) tma_load_3d(dst + hh * box_bytes, &tmk, full, hh * 64, tok, plane);
-      issued = k + 1;
-      if (++beta == nb) {
-        beta = 0;
-        do {
-          ++b;
-          nb = b < a.batch ? seq_blocks(a, b) : 1;
-        } while (nb == 0);
+        for (int hh = 0; hh < DI / 64; ++hh)
+          tma_load_3d(dst + hh * box_bytes, &tmk, full, hh * 64, beta * a.block, b);
+        issued = k + 1;
+        if (++beta == nb) {
+          beta = 0;
+          do {
+            ++b;
+            nb = b < a.batch ? seq_blocks(a, b) : 1;
+          } while (nb == 0);
+        }
       }
     }
+    // Paged K_idx, groups of 32 items: every lane resolves one item's sequence,
+    // block and page (the table loads run in parallel), and lane 0 streams the
+    // group from shared memory.
+    for (int k0 = 0; k0 < n && !failed && a.pg.table != nullptr; k0 += 32) {
+      if (k0 + lane < n) {
+        int bb = b, bt = beta + lane, nbb = seq_blocks(a, bb);
+        while (bt >= nbb) {  // the item exists, so bb stays below the batch
+          bt -= nbb;
+          nbb = seq_blocks(a, ++bb);
+        }
+        int tok, plane;
+        kv_block_coords(a.pg, bb, bt, a.block, a.st, tok, plane);
+        coord[lane] = make_int4(tok, plane, bb, bt);
+      }
+      __syncwarp();
+      if (lane == 0) {
+        for (int j = 0; j < 32 && k0 + j < n; ++j) {
+          const int k = k0 + j, s = k % S;
+          if (k >= S &&
+              !mbar_wait_bounded(empty0 + 8 * s, ((k / S) - 1) & 1, a.st, 0x201u, a.wait_ns)) {
+            failed = true;
+            break;
+          }
+          const int4 c = coord[j];
+          info[s] = make_int2(c.z, c.w);
+          const uint32_t full = full0 + 8 * s, dst = sbase + (uint32_t)s * a.stage_bytes;
+          mbar_arrive_expect_tx(full, a.stage_bytes);
+#pragma unroll
+          for (int hh = 0; hh < DI / 64; ++hh)
+            tma_load_3d(dst + hh * box_bytes, &tmk, full, hh * 64, c.x, c.y);
+          issued = k + 1;
+        }
+      }
+      failed = __shfl_sync(0xffffffffu, failed, 0);
+      const int4 last = coord[31];  // next group starts after this group's last item
+      b = last.z;
+      beta = last.w + 1;
+      __syncwarp();
+    }
+    if (lane != 0) return;
     // before leaving, wait (bounded) for the copies still in flight
     for (int k = max(0, issued - S); k < issued; ++k)
       mbar_wait_bounded(full0 + 8 * (k % S), (k / S) & 1, a.st, 0x203u, a.wait_ns);
@@ -458,7 +504,9 @@ cudaError_t run_stream_scan(const Shape& s, const uint16_t* k_idx, StreamScanArg
           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaSuccess;  // not expressible as a tensor map: the direct-load scan runs
   a.stage_bytes = (uint32_t)DI * 2u * (uint32_t)s.block;
-  const size_t fixed = 1024 + 64;
+  // alignment slack, the item count and the 32 resolved items after the stages'
+  // barriers and (sequence, block) words
+  const size_t fixed = 1024 + 16 + 32 * 16;
   const size_t cap = (size_t)max_smem_optin();
   // Consumer warp w takes items w, w + NW, ... and item k uses stage k % S.  With
   // S a multiple of NW every stage is only ever consumed by one warp, which has

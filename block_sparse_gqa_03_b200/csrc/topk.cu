@@ -459,6 +459,7 @@ cudaError_t launch_topk(const Shape& s, const float* scores, int32_t* ids, Devic
   if (n <= NT_ * E_) {                                             \
     return launch_pdl(topk_cta_kernel<NT_, E_>, grid, dim3(NT_), 0, stream, a); \
   }
+  MSA_TOPK_CTA(512, 4)
   MSA_TOPK_CTA(256, 8)
   MSA_TOPK_CTA(256, 16)
   MSA_TOPK_CTA(512, 16)

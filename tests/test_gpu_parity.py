@@ -23,8 +23,10 @@ def host(t):
     return None if t is None else t.cpu()
 
 
-def run_and_check(prob: Problem, rows=None, tail_fill=None, with_oracle_ids=True):
+def run_and_check(prob: Problem, rows=None, tail_fill=None, with_oracle_ids=True, lens=None):
     x = make_inputs(prob, device="cuda", tail_fill=tail_fill)
+    if lens is not None:
+        x["seq_lens"] = torch.tensor(lens, dtype=torch.int32, device="cuda")
     sl = x["seq_lens"]
     kw = dict(block=prob.block, causal=prob.causal, seq_lens=sl)
     ids_g, sc_g = msa.msa_index_select(x["q_idx"], x["k_idx"], topk=prob.topk,
@@ -100,6 +102,25 @@ SMALL_CASES = [
 @pytest.mark.parametrize("prob", SMALL_CASES, ids=lambda p: p.name)
 def test_small_problem_all_rows(prob):
     run_and_check(prob, tail_fill=float("nan") if prob.len_range else None)
+
+
+# Decode edge cases of the streaming index scan: empty and one-token sequences (no
+# items; every block -inf), fewer items than CTAs, 16 groups (two 8-column query
+# tiles), d_idx 64 with block 16 (a ring of sixteen 2 KB stages).
+DECODE_EDGE_CASES = [
+    (Problem("decode_edges_h8", batch=6, n_q=1, max_kv=3000, H=32, h=8, d=128, d_idx=128,
+             block=64, topk=8, seed=121), [0, 1, 63, 64, 65, 3000]),
+    (Problem("decode_h16_d64_b16", batch=3, n_q=1, max_kv=5000, H=16, h=16, d=64, d_idx=64,
+             block=16, topk=40, seed=122), [5000, 17, 2500]),
+    (Problem("decode_few_items", batch=1, n_q=1, max_kv=640, H=8, h=2, d=64, d_idx=128,
+             block=64, topk=4, seed=123), [640]),
+]
+
+
+@pytest.mark.parametrize("case", DECODE_EDGE_CASES, ids=lambda c: c[0].name)
+def test_decode_scan_edges(case):
+    prob, lens = case
+    run_and_check(prob, lens=lens)
 
 
 def test_workload_prefill_1k():

@@ -43,12 +43,12 @@ def periodic_k_idx(x, prob, period):
 
 
 CASES = [
-    # 2500 blocks per row: 256 threads x 16 keys; T shared by ~350 blocks
+    # 2500 blocks per row (256 threads x 16 keys); T shared by ~350 blocks
     (Problem("ties_p7", batch=3, n_q=1, max_kv=40000, H=8, h=2, d=64, d_idx=32, block=16,
              topk=128, seed=301), 7, [40000, 23456, 1600]),
-    # every full block scores the same
-    (Problem("ties_all", batch=2, n_q=1, max_kv=33000, H=8, h=2, d=64, d_idx=32, block=16,
-             topk=100, seed=302), 1, [33000, 20000]),
+    # every full block scores the same; 2048 blocks (512 threads x 4 keys)
+    (Problem("ties_all", batch=2, n_q=1, max_kv=32768, H=8, h=2, d=64, d_idx=32, block=16,
+             topk=100, seed=302), 1, [32760, 20000]),
     # own block forced, 5000 blocks (512 threads x 16 keys)
     (Problem("ties_own", batch=2, n_q=1, max_kv=80000, H=4, h=1, d=64, d_idx=64, block=16,
              topk=300, force_own=True, seed=303), 13, [80000, 77777]),
