@@ -41,11 +41,11 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # Per-launch DRAM traffic (read + write bytes) of the dominant kernel, from one ncu
 # capture at batch 4 scaled by 4 to the batch of 16 (the work grows in proportion):
-# profiles/sparse_attn_stream_decode128k_b4.md (134.46 MB read + 3.43 MB written) and
-# profiles/index_scan_stream_decode128k_b4.md (134.27 MB read + 4.17 MB written).  Absent
-# entries report null; an entry is removed when its kernel changes.
-TRAFFIC = {("decode_128k", "attn"): 4 * (134.456832e6 + 3.434752e6),
-           ("decode_128k", "select"): 4 * (134.271744e6 + 4.173568e6)}
+# profiles/sparse_attn_stream_decode128k_b4.md (134.46 MB read + 3.43 MB written).  The
+# index scan's capture (profiles/index_scan_stream_decode128k_b4.md, 134.27 MB read + 4.17 MB
+# written) predates its paged producer path, so its entry is absent until it is re-captured.
+# Absent entries report null; an entry is removed when its kernel changes.
+TRAFFIC = {("decode_128k", "attn"): 4 * (134.456832e6 + 3.434752e6)}
 
 
 def load_peaks():
