@@ -18,7 +18,7 @@ CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libmsa.so")
 BUILD_DIR = os.path.join(ROOT, "_build")
 SOURCES = ["msa_api.cu", "index_scores.cu", "index_scores_tc.cu", "topk.cu", "sparse_attn.cu",
-           "sparse_attn_kv.cu", "append_kv.cu"]
+           "sparse_attn_kv.cu", "append_kv.cu", "shard.cu"]
 HEADERS = ["common.cuh", "kernels.h", "sm100.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",

@@ -34,8 +34,31 @@ cudaError_t launch_index_scores_tc(const Shape& s, const uint16_t* q_idx, const 
 // Stage 1c: top-k block ids, int32 [batch, n_q, h, topk], from the scores.  When
 // `zero` is given, the kernel also clears zero[0, nzero) (the attention's merge
 // counters, so that a fused forward needs no separate memset between the stages).
+// `kept` (nullable) receives the score of each kept id, -inf for padding.
 cudaError_t launch_topk(const Shape& s, const float* scores, int32_t* ids, DeviceStatus* st,
-                        cudaStream_t stream, int* zero = nullptr, int nzero = 0);
+                        cudaStream_t stream, int* zero = nullptr, int nzero = 0,
+                        float* kept = nullptr);
+
+// Global top-k from the candidate lists of KV shards (sequence-sharded decode):
+// cscores / cids [nlists, rows, len], list r ascending ids local to the shard
+// starting at block r * shard_blocks; writes global ids and/or the ids local to
+// the shard [base, base + nloc) (-1 elsewhere).  nlists * len <= 16384.
+cudaError_t launch_candidates_topk(const Shape& s, int nlists, int len, int shard_blocks,
+                                   const float* cscores, const int32_t* cids, int base, int nloc,
+                                   int32_t* ids, int32_t* local, DeviceStatus* st,
+                                   cudaStream_t stream);
+
+// LSE merge of `nparts` partial results of the same rows: part_out bf16
+// [nparts, rows * H, d] (dense), part_lse fp32 [nparts, rows * H]; out with the
+// shape's output strides, lse (nullable) dense [rows * H].
+cudaError_t launch_merge_partials(const Shape& s, int nparts, const uint16_t* part_out,
+                                  const float* part_lse, uint16_t* out, float* lse,
+                                  cudaStream_t stream);
+
+// Token lengths of the shard [base, base + len) of each sequence:
+// out[b] = clamp(L_b - base, 0, len).
+cudaError_t launch_shard_lengths(const int32_t* seq_lens, int batch, int max_kv, int64_t base,
+                                 int64_t len, int32_t* out, DeviceStatus* st, cudaStream_t stream);
 
 // Decode-step cache write: the n_q new tokens of every sequence (dense
 // [batch, n_q, h, d] K and V, [batch, n_q, d_idx] K_idx; any may be null) go to

@@ -4,6 +4,9 @@
 #include <math.h>
 #include <string.h>
 
+#include <atomic>
+#include <mutex>
+
 #include "../../include/msa.h"
 #include "kernels.h"
 
@@ -182,7 +185,7 @@ Layout layout(const Shape& s, msa_op_t op) {
   size_t off = msa::kStatusBytes;
   l.scores_off = l.ids_off = l.part_off = 0;
   l.part_bytes = 0;
-  if (op == MSA_OP_INDEX_SELECT || op == MSA_OP_FORWARD) {
+  if (op == MSA_OP_INDEX_SELECT || op == MSA_OP_INDEX_CANDIDATES || op == MSA_OP_FORWARD) {
     l.scores_off = off;
     off = align_up(off + scores_bytes(s));
   }
@@ -199,10 +202,16 @@ Layout layout(const Shape& s, msa_op_t op) {
   return l;
 }
 
+// Operations whose workspace holds the status word only.
+bool status_only(msa_op_t op) {
+  return op == MSA_OP_APPEND_KV || op == MSA_OP_BLOCK_SCORES || op == MSA_OP_SELECT_CANDIDATES ||
+         op == MSA_OP_SHARD_LENGTHS;
+}
+
 msa_status_t check_ws(const Shape& s, msa_op_t op, void* ws, size_t bytes) {
   if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) != 0)
     return MSA_ERR_WORKSPACE;
-  if (bytes < (op == MSA_OP_APPEND_KV ? msa::kStatusBytes : layout(s, op).total))
+  if (bytes < (status_only(op) ? msa::kStatusBytes : layout(s, op).total))
     return MSA_ERR_WORKSPACE;
   return MSA_OK;
 }
@@ -211,18 +220,23 @@ msa_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MSA_OK : MSA
 
 uint8_t* at(void* ws, size_t off) { return reinterpret_cast<uint8_t*>(ws) + off; }
 
+cudaError_t run_scores(const Shape& s, const msa_bf16_t* q_idx, const msa_bf16_t* k_idx,
+                       float* scores, bool fill_tail, msa::DeviceStatus* st,
+                       cudaStream_t stream) {
+  return msa::index_scores_tc_supported(s)
+             ? msa::launch_index_scores_tc(s, q_idx, k_idx, scores, fill_tail, st, stream)
+             : msa::launch_index_scores(s, q_idx, k_idx, scores, fill_tail, st, stream);
+}
+
 msa_status_t run_select(const Shape& s, const msa_bf16_t* q_idx, const msa_bf16_t* k_idx,
                         int32_t* ids, float* user_scores, void* ws, const Layout& l,
-                        cudaStream_t stream, int* zero = nullptr, int nzero = 0) {
+                        cudaStream_t stream, int* zero = nullptr, int nzero = 0,
+                        float* kept = nullptr) {
   msa::DeviceStatus* st = reinterpret_cast<msa::DeviceStatus*>(ws);
   float* scores = user_scores ? user_scores : reinterpret_cast<float*>(at(ws, l.scores_off));
-  cudaError_t e = msa::index_scores_tc_supported(s)
-                      ? msa::launch_index_scores_tc(s, q_idx, k_idx, scores,
-                                                    user_scores != nullptr, st, stream)
-                      : msa::launch_index_scores(s, q_idx, k_idx, scores, user_scores != nullptr,
-                                                 st, stream);
-  if (e != cudaSuccess) return MSA_ERR_CUDA;
-  return cuda_status(msa::launch_topk(s, scores, ids, st, stream, zero, nzero));
+  if (run_scores(s, q_idx, k_idx, scores, user_scores != nullptr, st, stream) != cudaSuccess)
+    return MSA_ERR_CUDA;
+  return cuda_status(msa::launch_topk(s, scores, ids, st, stream, zero, nzero, kept));
 }
 
 }  // namespace
@@ -232,9 +246,92 @@ extern "C" {
 size_t msa_workspace_size(const msa_params_t* params, msa_op_t op) {
   Shape s;
   if (make_shape(params, &s) != MSA_OK) return 0;
-  if (op == MSA_OP_APPEND_KV) return msa::kStatusBytes;
-  if (op != MSA_OP_INDEX_SELECT && op != MSA_OP_SPARSE_ATTN && op != MSA_OP_FORWARD) return 0;
+  if (status_only(op)) return msa::kStatusBytes;
+  if (op != MSA_OP_INDEX_SELECT && op != MSA_OP_SPARSE_ATTN && op != MSA_OP_FORWARD &&
+      op != MSA_OP_INDEX_CANDIDATES)
+    return 0;
   return layout(s, op).total;
+}
+
+msa_status_t msa_block_scores(const msa_params_t* params, const msa_bf16_t* q_idx,
+                              const msa_bf16_t* k_idx, float* block_scores, void* workspace,
+                              size_t workspace_bytes, msa_stream_t stream) {
+  Shape s;
+  msa_status_t rc = make_shape(params, &s);
+  if (rc != MSA_OK) return rc;
+  if ((rc = check_select_args(s, q_idx, k_idx)) != MSA_OK) return rc;
+  if (block_scores == nullptr) return MSA_ERR_INVALID_ARG;
+  if ((rc = check_ws(s, MSA_OP_BLOCK_SCORES, workspace, workspace_bytes)) != MSA_OK) return rc;
+  return cuda_status(run_scores(s, q_idx, k_idx, block_scores, true,
+                                reinterpret_cast<msa::DeviceStatus*>(workspace),
+                                reinterpret_cast<cudaStream_t>(stream)));
+}
+
+msa_status_t msa_index_candidates(const msa_params_t* params, const msa_bf16_t* q_idx,
+                                  const msa_bf16_t* k_idx, int32_t* block_ids,
+                                  float* kept_scores, void* workspace, size_t workspace_bytes,
+                                  msa_stream_t stream) {
+  Shape s;
+  msa_status_t rc = make_shape(params, &s);
+  if (rc != MSA_OK) return rc;
+  if ((rc = check_select_args(s, q_idx, k_idx)) != MSA_OK) return rc;
+  if (block_ids == nullptr || kept_scores == nullptr) return MSA_ERR_INVALID_ARG;
+  if ((rc = check_ws(s, MSA_OP_INDEX_CANDIDATES, workspace, workspace_bytes)) != MSA_OK)
+    return rc;
+  return run_select(s, q_idx, k_idx, block_ids, nullptr, workspace,
+                    layout(s, MSA_OP_INDEX_CANDIDATES), reinterpret_cast<cudaStream_t>(stream),
+                    nullptr, 0, kept_scores);
+}
+
+msa_status_t msa_select_candidates(const msa_params_t* params, int32_t nlists, int32_t list_len,
+                                   int32_t shard_blocks, const float* cand_scores,
+                                   const int32_t* cand_ids, int32_t block_base,
+                                   int32_t nblk_local, int32_t* block_ids, int32_t* local_ids,
+                                   void* workspace, size_t workspace_bytes, msa_stream_t stream) {
+  Shape s;
+  msa_status_t rc = make_shape(params, &s);
+  if (rc != MSA_OK) return rc;
+  if (!cand_scores || !cand_ids || (!block_ids && !local_ids)) return MSA_ERR_INVALID_ARG;
+  if (nlists < 1 || list_len < 1 || shard_blocks < 0 || block_base < 0 || nblk_local < 0)
+    return MSA_ERR_INVALID_ARG;
+  if ((int64_t)nlists * list_len > 16384) return MSA_ERR_UNSUPPORTED;
+  if ((int64_t)(nlists - 1) * shard_blocks >= (int64_t)INT32_MAX / 2) return MSA_ERR_INVALID_ARG;
+  if ((rc = check_ws(s, MSA_OP_SELECT_CANDIDATES, workspace, workspace_bytes)) != MSA_OK)
+    return rc;
+  return cuda_status(msa::launch_candidates_topk(
+      s, nlists, list_len, shard_blocks, cand_scores, cand_ids, block_base, nblk_local, block_ids,
+      local_ids, reinterpret_cast<msa::DeviceStatus*>(workspace),
+      reinterpret_cast<cudaStream_t>(stream)));
+}
+
+msa_status_t msa_merge_partials(const msa_params_t* params, int32_t nparts,
+                                const msa_bf16_t* part_out, const float* part_lse,
+                                msa_bf16_t* out, float* lse, msa_stream_t stream) {
+  Shape s;
+  msa_status_t rc = make_shape(params, &s);
+  if (rc != MSA_OK) return rc;
+  if (!part_out || !part_lse || !out || !aligned16(part_out) || !aligned16(out) ||
+      (reinterpret_cast<uintptr_t>(part_lse) & 3u) != 0)
+    return MSA_ERR_INVALID_ARG;
+  if (nparts < 1 || nparts > 1024) return MSA_ERR_INVALID_ARG;
+  if (check_strides3(s.o_s) != MSA_OK || s.o_s[2] < s.d) return MSA_ERR_INVALID_ARG;
+  return cuda_status(msa::launch_merge_partials(s, nparts, part_out, part_lse, out, lse,
+                                                reinterpret_cast<cudaStream_t>(stream)));
+}
+
+msa_status_t msa_shard_lengths(const msa_params_t* params, int64_t token_base,
+                               int64_t token_count, int32_t* shard_lens, void* workspace,
+                               size_t workspace_bytes, msa_stream_t stream) {
+  Shape s;
+  msa_status_t rc = make_shape(params, &s);
+  if (rc != MSA_OK) return rc;
+  if (shard_lens == nullptr || token_base < 0 || token_count < 0 ||
+      token_base > (int64_t)INT32_MAX || token_count > (int64_t)INT32_MAX)
+    return MSA_ERR_INVALID_ARG;
+  if ((rc = check_ws(s, MSA_OP_SHARD_LENGTHS, workspace, workspace_bytes)) != MSA_OK) return rc;
+  return cuda_status(msa::launch_shard_lengths(
+      s.seq_lens, s.batch, s.max_kv, token_base, token_count, shard_lens,
+      reinterpret_cast<msa::DeviceStatus*>(workspace), reinterpret_cast<cudaStream_t>(stream)));
 }
 
 msa_status_t msa_index_select(const msa_params_t* params, const msa_bf16_t* q_idx,
@@ -354,6 +451,10 @@ int msa_launch_count(const msa_params_t* params, msa_op_t op) {
     case MSA_OP_SPARSE_ATTN: return msa::attn_launches(s);
     case MSA_OP_FORWARD: return 2 + msa::attn_launches(s);
     case MSA_OP_APPEND_KV: return 1;
+    case MSA_OP_BLOCK_SCORES: return 1;
+    case MSA_OP_INDEX_CANDIDATES: return 2;
+    case MSA_OP_SELECT_CANDIDATES: return 1;
+    case MSA_OP_SHARD_LENGTHS: return 1;
   }
   return -1;
 }
@@ -386,19 +487,26 @@ __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 // Device address of g_noalloc_scratch per device.  In host code the array's
 // name is only a host-side stand-in, so the address is looked up once per
-// device (with that device current) and cached.
-void* g_noalloc_ptr[64] = {nullptr};
+// device (with that device current) and kept.  Host threads may call at the
+// same time: the entries are atomics and the lookup itself runs under a lock
+// (a failed lookup leaves the entry empty, so a later call tries again).
+std::atomic<void*> g_noalloc_ptr[64];
+std::mutex g_noalloc_lock;
 
 msa_status_t noalloc_scratch(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MSA_ERR_CUDA;
-  if (g_noalloc_ptr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
-      return MSA_ERR_CUDA;
-    g_noalloc_ptr[dev] = p;
+  void* p = g_noalloc_ptr[dev].load(std::memory_order_acquire);
+  if (p == nullptr) {
+    std::lock_guard<std::mutex> guard(g_noalloc_lock);
+    p = g_noalloc_ptr[dev].load(std::memory_order_acquire);
+    if (p == nullptr) {
+      if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+        return MSA_ERR_CUDA;
+      g_noalloc_ptr[dev].store(p, std::memory_order_release);
+    }
   }
-  *out = g_noalloc_ptr[dev];
+  *out = p;
   return MSA_OK;
 }
 
@@ -417,9 +525,10 @@ extern "C" msa_status_t msa_sparse_attn_noalloc(const msa_params_t* params, cons
   if (need > kNoAllocScratchBytes) return MSA_ERR_WORKSPACE;
   void* scratch = nullptr;
   if ((rc = noalloc_scratch(&scratch)) != MSA_OK) return rc;
-  // The per-row merge counters inside the scratch are zeroed on the stream before
-  // every launch; the partials themselves are always written before they are
-  // read.  No status word: device-side errors are skipped, not recorded.
+  // What must start at zero inside the scratch (the decode kernel's per-row merge
+  // counters, the KV-major kernel's per-block counts) is cleared on the stream by
+  // every call; the partials themselves are always written before they are read.
+  // No status word: device-side errors are skipped, not recorded.
   return cuda_status(msa::launch_sparse_attn(s, q, k, v, block_ids, out, lse, scratch,
                                              kNoAllocScratchBytes, nullptr,
                                              reinterpret_cast<cudaStream_t>(stream)));

@@ -27,6 +27,7 @@ namespace {
 struct TopkArgs {
   const float* scores;
   int32_t* ids;
+  float* kept;  // when not null: the score of each kept id (-inf for padding)
   const int32_t* seq_lens;
   int rows, n_q, max_kv, h, block, nblk, topk, causal, force_own;
   DeviceStatus* st;
@@ -243,6 +244,12 @@ __global__ void __launch_bounds__(256, 3) topk_warp_kernel(TopkArgs a) {
     warp_row_topk<E>(s, out, ri, lane, cbuf[w]);
   }
   for (int i = m + lane; i < a.topk; i += 32) out[i] = -1;
+  if (a.kept != nullptr) {
+    __syncwarp();
+    float* kp = a.kept + (int64_t)row * a.topk;
+    for (int i = lane; i < a.topk; i += 32)
+      kp[i] = i < m ? s[out[i]] : -__int_as_float(0x7f800000);
+  }
 }
 
 // Sums over the CTA (NW warps) of W words per thread; `buf` alternates between
@@ -417,12 +424,177 @@ __global__ void __launch_bounds__(NT) topk_cta_kernel(TopkArgs a) {
       if (sel[e]) out[pos++] = i0 + e;
   }
   for (int i = m + threadIdx.x; i < a.topk; i += NT) out[i] = -1;
+  if (a.kept != nullptr) {
+    __syncthreads();
+    float* kp = a.kept + (int64_t)row * a.topk;
+    for (int i = threadIdx.x; i < a.topk; i += NT)
+      kp[i] = i < m ? s[out[i]] : -__int_as_float(0x7f800000);
+  }
+}
+
+// ------------------------------------------------ merge of candidate lists
+// Global top-k of a row from the candidate lists of several KV shards (each
+// shard's own top-k of its blocks, with their scores): the same order as the
+// single-device top-k (score descending, block id ascending, the own block first
+// when forced), because a row's global top-k blocks are each in the top-k of the
+// shard that holds them.  The lists arrive as an all-gather leaves them, list
+// after list ([nlists, rows, len]); list r holds ascending ids local to shard r,
+// whose blocks start at r * shard_blocks, so a row's valid candidates, taken
+// list by list, come in ascending global id order and position order breaks
+// ties by id.  A forced own block needs no score: it is taken first even when no
+// shard listed it.
+struct CandArgs {
+  const float* cscores;  // [nlists, rows, len]
+  const int32_t* cids;   // [nlists, rows, len], -1 = empty
+  int32_t* ids;          // [rows, topk] global ids (nullable)
+  int32_t* local;        // [rows, topk] id - base inside [base, base + nloc), else -1 (nullable)
+  const int32_t* seq_lens;
+  int rows, nlists, len, shard_blocks, n_q, max_kv, h, block, topk, force_own, base, nloc;
+  DeviceStatus* st;
+};
+
+template <int NT, int E>
+__global__ void __launch_bounds__(NT) candidates_topk_kernel(CandArgs a) {
+  grid_dep_wait();
+  grid_dep_launch();
+  constexpr int NW = NT / 32;
+  __shared__ uint32_t cbuf[32];
+  __shared__ int ccount;
+  __shared__ unsigned red[2][2][32];
+  __shared__ unsigned wsum[32];
+  __shared__ uint32_t Ts;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int row = blockIdx.x;
+  const int bt = row / a.h;
+  const int t = bt % a.n_q, b = bt / a.n_q;
+  const int L = kv_length(a.seq_lens, b, a.max_kv, a.st);
+  const int p = L - a.n_q + t;
+  const int own = (a.force_own && p >= 0) ? p / a.block : -1;
+  const int ncand = a.nlists * a.len;
+  const int i0 = threadIdx.x * E;
+  if (threadIdx.x == 0) ccount = 0;
+  uint32_t key[E];
+  int id[E];
+  unsigned cnt[2] = {0u, 0u};  // valid candidates (the own block excluded), own present
+  uint32_t kmax = 0u, kmin = 0xffffffffu;
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const int i = i0 + e;
+    const int li = i / a.len;  // list (shard) of candidate i
+    const int64_t at = ((int64_t)li * a.rows + row) * a.len + (i - li * a.len);
+    id[e] = i < ncand ? __ldg(a.cids + at) : -1;
+    key[e] = id[e] >= 0 ? order_key(__ldg(a.cscores + at)) : 0u;
+    if (id[e] >= 0) id[e] += li * a.shard_blocks;
+    if (id[e] >= 0 && id[e] == own) key[e] = 0xffffffffu;
+    const bool vis = key[e] != 0u && key[e] != 0xffffffffu;
+    cnt[0] += vis;
+    cnt[1] += key[e] == 0xffffffffu;
+    kmax = vis ? max(kmax, key[e]) : kmax;
+    kmin = vis ? min(kmin, key[e]) : kmin;
+  }
+  int buf = 0;
+  cta_sums<NW, 2>(cnt, red, buf);
+  kmax = __reduce_max_sync(0xffffffffu, kmax);
+  kmin = __reduce_min_sync(0xffffffffu, kmin);
+  __shared__ uint32_t wmax[NW], wmin[NW];
+  if (lane == 0) {
+    wmax[warp] = kmax;
+    wmin[warp] = kmin;
+  }
+  __syncthreads();
+  kmax = __reduce_max_sync(0xffffffffu, lane < NW ? wmax[lane] : 0u);
+  kmin = __reduce_min_sync(0xffffffffu, lane < NW ? wmin[lane] : 0xffffffffu);
+  const int forced = own >= 0 ? 1 : 0;
+  const bool virt = forced && cnt[1] == 0u;  // forced own block listed by no shard
+  const int m = min(a.topk, (int)cnt[0] + forced);
+  uint32_t T;
+  if (m <= forced || kmax < kmin) {
+    T = 0xffffffffu;
+  } else {
+    Bucket r = bucket_start(kmax, kmin, (int)cnt[0], forced);
+    while (r.cnt > 32 && r.hi >= 0) {
+      const uint32_t cand = r.prefix | (1u << r.hi);
+      unsigned c[1] = {0u};
+#pragma unroll
+      for (int e = 0; e < E; ++e) c[0] += key[e] >= cand;
+      if (virt && threadIdx.x == 0) c[0] += 1u;  // the unlisted forced block, counted once
+      cta_sums<NW, 1>(c, red, buf);
+      bucket_split(r, (int)c[0], m);
+    }
+    if (r.cnt > 32) {
+      T = r.prefix;
+    } else {
+#pragma unroll
+      for (int e = 0; e < E; ++e)
+        if (in_bucket(key[e], r)) {
+          const int at = atomicAdd(&ccount, 1);
+          if (at < 32) cbuf[at] = key[e];
+        }
+      __syncthreads();
+      if (warp == 0) {
+        const uint32_t ck = lane < r.cnt ? cbuf[lane] : 0u;
+        const uint32_t tt = rank_pick(ck, r.cnt, m - r.above, lane);
+        if (lane == 0) Ts = tt;
+      }
+      __syncthreads();
+      T = Ts;
+    }
+  }
+  unsigned ge[2] = {0u, 0u};
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    ge[0] += key[e] > T;
+    ge[1] += key[e] == T;
+  }
+  if (virt && threadIdx.x == 0) ge[T == 0xffffffffu ? 1 : 0] += 1u;
+  cta_sums<NW, 2>(ge, red, buf);
+  const int need = m - (int)ge[0];
+  unsigned eq = 0;
+#pragma unroll
+  for (int e = 0; e < E; ++e) eq += key[e] == T;
+  // a virtual own block (key T only when T is the forced key) ranks before all
+  unsigned eqr = cta_exclusive_scan<NW>(eq, wsum) + ((virt && T == 0xffffffffu) ? 1u : 0u);
+  bool sel[E];
+  unsigned nsel = 0;
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const bool is_eq = key[e] == T;
+    sel[e] = key[e] != 0u && (key[e] > T || (is_eq && (int)eqr < need));
+    eqr += is_eq;
+    nsel += sel[e];
+  }
+  // output slots in ascending id order: position order, with a virtual own
+  // block placed before the first selected id above it
+  unsigned pos = cta_exclusive_scan<NW>(nsel, wsum);
+  unsigned below_own = 0;
+  if (virt) {
+#pragma unroll
+    for (int e = 0; e < E; ++e) below_own += sel[e] && id[e] < own;
+    unsigned tmp[1] = {below_own};
+    cta_sums<NW, 1>(tmp, red, buf);
+    below_own = tmp[0];
+  }
+  int32_t* og = a.ids ? a.ids + (int64_t)row * a.topk : nullptr;
+  int32_t* ol = a.local ? a.local + (int64_t)row * a.topk : nullptr;
+  auto emit = [&](int slot, int gid) {
+    if (og) og[slot] = gid;
+    if (ol) ol[slot] = (gid >= a.base && gid < a.base + a.nloc) ? gid - a.base : -1;
+  };
+#pragma unroll
+  for (int e = 0; e < E; ++e)
+    if (sel[e]) {
+      const int slot = (int)pos + ((virt && id[e] > own) ? 1 : 0);
+      ++pos;
+      if (slot < a.topk) emit(slot, id[e]);
+    }
+  if (virt && threadIdx.x == 0 && (int)below_own < a.topk) emit((int)below_own, own);
+  for (int i = m + threadIdx.x; i < a.topk; i += NT) emit(i, -1);
 }
 
 }  // namespace
 
 cudaError_t launch_topk(const Shape& s, const float* scores, int32_t* ids, DeviceStatus* st,
-                        cudaStream_t stream, int* zero, int nzero) {
+                        cudaStream_t stream, int* zero, int nzero, float* kept) {
   TopkArgs a;
   a.scores = scores;
   a.ids = ids;
@@ -439,6 +611,7 @@ cudaError_t launch_topk(const Shape& s, const float* scores, int32_t* ids, Devic
   a.st = st;
   a.zero = zero;
   a.nzero = nzero;
+  a.kept = kept;
   const int n = s.nblk;
   if (n <= 1024) {
     const dim3 grid((a.rows + 7) / 8);
@@ -467,6 +640,42 @@ cudaError_t launch_topk(const Shape& s, const float* scores, int32_t* ids, Devic
   MSA_TOPK_CTA(1024, 32)
   MSA_TOPK_CTA(1024, 64)
 #undef MSA_TOPK_CTA
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_candidates_topk(const Shape& s, int nlists, int len, int shard_blocks,
+                                   const float* cscores, const int32_t* cids, int base, int nloc,
+                                   int32_t* ids, int32_t* local, DeviceStatus* st,
+                                   cudaStream_t stream) {
+  CandArgs a;
+  a.cscores = cscores;
+  a.cids = cids;
+  a.ids = ids;
+  a.local = local;
+  a.seq_lens = s.seq_lens;
+  a.rows = s.batch * s.n_q * s.h;
+  a.nlists = nlists;
+  a.len = len;
+  a.shard_blocks = shard_blocks;
+  const int ncand = nlists * len;
+  a.n_q = s.n_q;
+  a.max_kv = s.max_kv;
+  a.h = s.h;
+  a.block = s.block;
+  a.topk = s.topk;
+  a.force_own = s.force_own;
+  a.base = base;
+  a.nloc = nloc;
+  a.st = st;
+  const dim3 grid(a.rows);
+#define MSA_CAND_CTA(NT_, E_)                                            \
+  if (ncand <= NT_ * E_) {                                               \
+    return launch_pdl(candidates_topk_kernel<NT_, E_>, grid, dim3(NT_), 0, stream, a); \
+  }
+  MSA_CAND_CTA(256, 4)
+  MSA_CAND_CTA(256, 16)
+  MSA_CAND_CTA(1024, 16)
+#undef MSA_CAND_CTA
   return cudaErrorInvalidValue;
 }
 

@@ -33,10 +33,16 @@ MSA_OP_INDEX_SELECT = 0
 MSA_OP_SPARSE_ATTN = 1
 MSA_OP_FORWARD = 2
 MSA_OP_APPEND_KV = 3
+MSA_OP_BLOCK_SCORES = 4
+MSA_OP_INDEX_CANDIDATES = 5
+MSA_OP_SELECT_CANDIDATES = 6
+MSA_OP_SHARD_LENGTHS = 7
 
 EXPORTED = ("msa_workspace_size", "msa_index_select", "msa_sparse_attn", "msa_forward",
             "msa_get_device_status", "msa_workspace_init", "msa_selftest_wait_timeout",
-            "msa_launch_count", "msa_sparse_attn_noalloc", "msa_status_string", "msa_append_kv")
+            "msa_launch_count", "msa_sparse_attn_noalloc", "msa_status_string", "msa_append_kv",
+            "msa_block_scores", "msa_index_candidates", "msa_select_candidates",
+            "msa_merge_partials", "msa_shard_lengths")
 
 
 class MsaError(RuntimeError):
@@ -97,6 +103,17 @@ def load_library():
             lib.msa_selftest_wait_timeout.restype = I
             lib.msa_sparse_attn_noalloc.argtypes = [P, P, P, P, P, P, P, P]
             lib.msa_sparse_attn_noalloc.restype = I
+            lib.msa_block_scores.argtypes = [P, P, P, P, P, S, P]
+            lib.msa_block_scores.restype = I
+            lib.msa_index_candidates.argtypes = [P, P, P, P, P, P, S, P]
+            lib.msa_index_candidates.restype = I
+            i32 = ctypes.c_int32
+            lib.msa_select_candidates.argtypes = [P, i32, i32, i32, P, P, i32, i32, P, P, P, S, P]
+            lib.msa_select_candidates.restype = I
+            lib.msa_merge_partials.argtypes = [P, ctypes.c_int32, P, P, P, P, P]
+            lib.msa_merge_partials.restype = I
+            lib.msa_shard_lengths.argtypes = [P, ctypes.c_int64, ctypes.c_int64, P, P, S, P]
+            lib.msa_shard_lengths.restype = I
             lib.msa_launch_count.argtypes = [P, I]
             lib.msa_launch_count.restype = I
             lib.msa_status_string.argtypes = [I]
@@ -364,3 +381,106 @@ def msa_forward(q, k, v, q_idx, k_idx, *, block, topk, causal=True, force_own_bl
     if return_lse:
         res.append(lse)
     return res[0] if len(res) == 1 else tuple(res)
+
+
+def msa_block_scores(q_idx, k_idx, *, block, causal=True, seq_lens=None, block_scores=None,
+                     block_table=None, max_kv=None, workspace: Workspace | None = None,
+                     stream=None):
+    """Stage 1, first half: fp32 block scores [b, n_q, h, nblk] (-inf past the frontier)."""
+    b, n_q, h, d_idx = q_idx.shape
+    max_kv, num_pages = _kv_extent(k_idx, block_table, max_kv)
+    nblk = (max_kv + block - 1) // block
+    p = make_params(batch=b, n_q=n_q, max_kv=max_kv, H=h, h=h, d=64, d_idx=d_idx, block=block,
+                    topk=1, causal=causal, seq_lens=seq_lens, q_idx=q_idx, k_idx=k_idx,
+                    block_table=block_table, num_pages=num_pages)
+    if block_scores is None:
+        block_scores = torch.empty((b, n_q, h, nblk), dtype=torch.float32, device=q_idx.device)
+    ws = _workspace(workspace, q_idx.device).get(msa_workspace_size(p, MSA_OP_BLOCK_SCORES))
+    _check(load_library().msa_block_scores(ctypes.byref(p), _ptr(q_idx), _ptr(k_idx),
+                                           _ptr(block_scores), ws.data_ptr(), ws.numel(),
+                                           _stream(stream)), "msa_block_scores")
+    return block_scores
+
+
+def msa_index_candidates(q_idx, k_idx, *, block, topk, causal=True, force_own_block=False,
+                         seq_lens=None, block_ids=None, kept_scores=None, block_table=None,
+                         max_kv=None, workspace: Workspace | None = None, stream=None):
+    """msa_index_select plus the kept blocks' scores: (ids, scores), both [b, n_q, h, topk]."""
+    b, n_q, h, d_idx = q_idx.shape
+    max_kv, num_pages = _kv_extent(k_idx, block_table, max_kv)
+    p = make_params(batch=b, n_q=n_q, max_kv=max_kv, H=h, h=h, d=64, d_idx=d_idx, block=block,
+                    topk=topk, causal=causal, force_own_block=force_own_block,
+                    seq_lens=seq_lens, q_idx=q_idx, k_idx=k_idx, block_table=block_table,
+                    num_pages=num_pages)
+    dev = q_idx.device
+    if block_ids is None:
+        block_ids = torch.empty((b, n_q, h, topk), dtype=torch.int32, device=dev)
+    if kept_scores is None:
+        kept_scores = torch.empty((b, n_q, h, topk), dtype=torch.float32, device=dev)
+    need = msa_workspace_size(p, MSA_OP_INDEX_CANDIDATES)
+    if need == 0:
+        raise MsaError(MSA_ERR_INVALID_ARG, "msa_workspace_size")
+    ws = _workspace(workspace, dev).get(need)
+    _check(load_library().msa_index_candidates(ctypes.byref(p), _ptr(q_idx), _ptr(k_idx),
+                                               _ptr(block_ids), _ptr(kept_scores), ws.data_ptr(),
+                                               ws.numel(), _stream(stream)),
+           "msa_index_candidates")
+    return block_ids, kept_scores
+
+
+def msa_select_candidates(cand_scores, cand_ids, *, max_kv, block, topk, shard_blocks=0,
+                          causal=True, force_own_block=False, seq_lens=None, block_base=0,
+                          nblk_local=0, block_ids=None, local_ids=None, want_global=True,
+                          want_local=False, workspace: Workspace | None = None, stream=None):
+    """Global top-k from gathered candidate lists [nlists, b, n_q, h, len] (list r's ids
+    local to the shard starting at block r * shard_blocks); returns the global ids and/or
+    the ids local to the shard [block_base, block_base + nblk_local)."""
+    nlists, b, n_q, h, llen = cand_ids.shape
+    if not (cand_ids.is_contiguous() and cand_scores.is_contiguous()):
+        raise ValueError("candidate lists must be dense")
+    p = make_params(batch=b, n_q=n_q, max_kv=max_kv, H=h, h=h, d=64, d_idx=32, block=block,
+                    topk=topk, causal=causal, force_own_block=force_own_block,
+                    seq_lens=seq_lens)
+    dev = cand_ids.device
+    if want_global and block_ids is None:
+        block_ids = torch.empty((b, n_q, h, topk), dtype=torch.int32, device=dev)
+    if want_local and local_ids is None:
+        local_ids = torch.empty((b, n_q, h, topk), dtype=torch.int32, device=dev)
+    ws = _workspace(workspace, dev).get(msa_workspace_size(p, MSA_OP_SELECT_CANDIDATES))
+    _check(load_library().msa_select_candidates(
+        ctypes.byref(p), int(nlists), int(llen), int(shard_blocks), _ptr(cand_scores),
+        _ptr(cand_ids), int(block_base), int(nblk_local),
+        _ptr(block_ids if want_global else None), _ptr(local_ids if want_local else None),
+        ws.data_ptr(), ws.numel(), _stream(stream)), "msa_select_candidates")
+    return block_ids, local_ids
+
+
+def msa_merge_partials(part_out, part_lse, *, out=None, lse=None, stream=None):
+    """LSE merge of part_out bf16 [P, b, n_q, H, d] with part_lse fp32 [P, b, n_q, H]."""
+    P, b, n_q, H, d = part_out.shape
+    if not (part_out.is_contiguous() and part_lse.is_contiguous()):
+        raise ValueError("partials must be dense")
+    if out is None:
+        out = torch.empty((b, n_q, H, d), dtype=part_out.dtype, device=part_out.device)
+    p = make_params(batch=b, n_q=n_q, max_kv=max(n_q, 1), H=H, h=H, d=d, d_idx=32, block=64,
+                    topk=1, out=out)
+    _check(load_library().msa_merge_partials(ctypes.byref(p), int(P), _ptr(part_out),
+                                             _ptr(part_lse), _ptr(out), _ptr(lse),
+                                             _stream(stream)), "msa_merge_partials")
+    return out
+
+
+def msa_shard_lengths(seq_lens, *, batch, max_kv, token_base, token_count, out=None,
+                      workspace: Workspace | None = None, stream=None, device=None):
+    """Per-sequence token counts inside the shard [token_base, token_base + token_count)."""
+    dev = seq_lens.device if seq_lens is not None else torch.device(device or "cuda")
+    if out is None:
+        out = torch.empty((batch,), dtype=torch.int32, device=dev)
+    p = make_params(batch=batch, n_q=1, max_kv=max_kv, H=1, h=1, d=64, d_idx=32, block=64,
+                    topk=1, seq_lens=seq_lens)
+    ws = _workspace(workspace, dev).get(msa_workspace_size(p, MSA_OP_SHARD_LENGTHS))
+    _check(load_library().msa_shard_lengths(ctypes.byref(p), int(token_base), int(token_count),
+                                            _ptr(out), ws.data_ptr(), ws.numel(),
+                                            _stream(stream)), "msa_shard_lengths")
+    return out
+

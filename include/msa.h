@@ -52,7 +52,9 @@
  *
  * Ownership and execution
  *   The caller owns every buffer, the workspace included; the library allocates
- *   no memory and keeps no state between calls.  All pointers except `params`
+ *   no memory and keeps no state between calls (one exception:
+ *   msa_sparse_attn_noalloc below uses a fixed array in the library's own device
+ *   memory and remembers that array's address per device).  All pointers except `params`
  *   are device pointers.  Calls are asynchronous on `stream`: argument errors
  *   return before anything is launched, launch failures return MSA_ERR_CUDA, and
  *   errors found on the device (a bounded wait that ran out, an id out of range)
@@ -93,7 +95,11 @@ typedef enum msa_op {
   MSA_OP_INDEX_SELECT = 0,
   MSA_OP_SPARSE_ATTN = 1,
   MSA_OP_FORWARD = 2,
-  MSA_OP_APPEND_KV = 3
+  MSA_OP_APPEND_KV = 3,
+  MSA_OP_BLOCK_SCORES = 4,
+  MSA_OP_INDEX_CANDIDATES = 5,
+  MSA_OP_SELECT_CANDIDATES = 6,
+  MSA_OP_SHARD_LENGTHS = 7
 } msa_op_t;
 
 typedef struct msa_params {
@@ -175,6 +181,87 @@ MSA_API msa_status_t msa_append_kv(const msa_params_t* params, const msa_bf16_t*
                                    msa_bf16_t* k, msa_bf16_t* v, msa_bf16_t* k_idx,
                                    void* workspace, size_t workspace_bytes, msa_stream_t stream);
 
+/* Stage 1, first half: the block scores alone (the index scan with its fused
+ * causal block max pool, no top-k).  block_scores fp32 [batch, n_q, h, nblk]
+ * receives S for every block, -inf past each row's frontier, exactly as
+ * msa_index_select's optional output.  The workspace holds the status word only
+ * (msa_workspace_size(params, MSA_OP_BLOCK_SCORES)).
+ * Sources: "MiniMax goes sparse" section 1 step 1 (Q_idx . K_idx^T and the Block
+ * Max Pool); "MiniMax M3 的 MSA ..." first layer. */
+MSA_API msa_status_t msa_block_scores(const msa_params_t* params, const msa_bf16_t* q_idx,
+                                      const msa_bf16_t* k_idx, float* block_scores,
+                                      void* workspace, size_t workspace_bytes,
+                                      msa_stream_t stream);
+
+/* Sequence-sharded decode.  The KV cache of every sequence is split into
+ * contiguous token shards of a whole number of blocks, one per GPU; shard r holds
+ * tokens [base_r, base_r + len_r) of every sequence.  The pages do not shard MSA;
+ * these four calls split one decode step (n_q = 1) so that the result equals the
+ * single-device result ("MiniMax goes sparse" section 1, steps 1 and 2):
+ *   1. msa_shard_lengths: each sequence's token count inside this shard.
+ *   2. msa_index_candidates on this shard's cache (params with the shard's
+ *      lengths and capacity, force_own_block = 0): the shard's own top-k block ids
+ *      (shard-local numbering) and their scores.  The lists of all shards are
+ *      gathered in shard order and
+ *   3. msa_select_candidates with the whole problem's params: the global top-k of
+ *      each row (the global top-k blocks are each in the top-k of their shard),
+ *      and the ids of the winners inside this shard in shard-local numbering.
+ *   4. msa_sparse_attn on this shard with those local ids (a row with no winner
+ *      here gets out = 0, lse = -inf), then the (out, lse) pairs of all shards are
+ *      gathered and msa_merge_partials weights them by their log-sum-exps.
+ * block_sparse_gqa_03_b200/seqshard.py runs these steps with NCCL all-gathers. */
+
+/* shard_lens[b] = clamp(L_b - token_base, 0, token_count) (device int32 [batch]),
+ * L_b from params->seq_lens (NULL: max_kv).  Workspace: the status word
+ * (msa_workspace_size(params, MSA_OP_SHARD_LENGTHS)). */
+MSA_API msa_status_t msa_shard_lengths(const msa_params_t* params, int64_t token_base,
+                                       int64_t token_count, int32_t* shard_lens,
+                                       void* workspace, size_t workspace_bytes,
+                                       msa_stream_t stream);
+
+/* msa_index_select plus the score of every kept block: block_ids int32 [batch,
+ * n_q, h, topk] as msa_index_select writes them (ascending, -1 padding) and
+ * kept_scores fp32 [batch, n_q, h, topk] = S[block_ids] (-inf for padding).
+ * Workspace: msa_workspace_size(params, MSA_OP_INDEX_CANDIDATES) bytes. */
+MSA_API msa_status_t msa_index_candidates(const msa_params_t* params, const msa_bf16_t* q_idx,
+                                          const msa_bf16_t* k_idx, int32_t* block_ids,
+                                          float* kept_scores, void* workspace,
+                                          size_t workspace_bytes, msa_stream_t stream);
+
+/* Top-k of each row (b, t, g) from candidate blocks, in msa_index_select's order:
+ * score descending, block id ascending, and with params->force_own_block the
+ * block holding position p = L_b - n_q + t first (also when no list holds it).
+ *   cand_scores fp32 / cand_ids int32 [nlists, batch, n_q, h, list_len]: the
+ *     lists of the shards in shard order, as an all-gather of every shard's
+ *     msa_index_candidates output leaves them.  List r holds ascending ids local
+ *     to shard r (global id = id + r * shard_blocks), -1 for empty entries;
+ *     1 <= nlists * list_len <= 16384.
+ *   block_ids (nullable) int32 [batch, n_q, h, topk]: the global winners,
+ *     ascending, -1 padded (m = min(topk, listed candidates plus the forced block)).
+ *   local_ids (nullable) int32 [batch, n_q, h, topk]: slot by slot, id -
+ *     block_base when block_base <= id < block_base + nblk_local, else -1.
+ * params: the whole problem (global seq_lens and max_kv, h, block, topk,
+ * force_own_block).  Workspace: the status word
+ * (msa_workspace_size(params, MSA_OP_SELECT_CANDIDATES)). */
+MSA_API msa_status_t msa_select_candidates(const msa_params_t* params, int32_t nlists,
+                                           int32_t list_len, int32_t shard_blocks,
+                                           const float* cand_scores, const int32_t* cand_ids,
+                                           int32_t block_base, int32_t nblk_local,
+                                           int32_t* block_ids, int32_t* local_ids,
+                                           void* workspace, size_t workspace_bytes,
+                                           msa_stream_t stream);
+
+/* Merge of nparts attention results over disjoint key sets of the same rows:
+ *   part_out bf16 [nparts, batch, n_q, H, d] and part_lse fp32 [nparts, batch,
+ *   n_q, H] (dense; a part with lse = -inf saw no key of the row);
+ *   out = sum_r e^(lse_r - M) out_r / sum_r e^(lse_r - M), M = max_r lse_r,
+ *   written with params->o_strides; lse (nullable, dense [batch, n_q, H]) =
+ *   M + log sum_r e^(lse_r - M).  Rows no part saw: out = 0, lse = -inf.
+ * Uses params batch, n_q, H, d and o_strides; no workspace. */
+MSA_API msa_status_t msa_merge_partials(const msa_params_t* params, int32_t nparts,
+                                        const msa_bf16_t* part_out, const float* part_lse,
+                                        msa_bf16_t* out, float* lse, msa_stream_t stream);
+
 /* Synchronises `stream`, returns the first error a kernel recorded in this
  * workspace since the last reset (MSA_OK if none) and clears it. */
 MSA_API msa_status_t msa_get_device_status(void* workspace, msa_stream_t stream);
@@ -195,17 +282,24 @@ MSA_API msa_status_t msa_selftest_wait_timeout(void* workspace, size_t workspace
  * memory: code running where an allocation is forbidden or would stall the GPU
  * (an inference engine's enqueue path, a real-time loop, a host framework that
  * owns every allocation), which therefore cannot provide the workspace that
- * msa_sparse_attn needs for its split-KV partial results.  This entry point has
- * no counterpart in the pages; it is a deployment convenience.
+ * msa_sparse_attn needs for its intermediate results.  This entry point has no
+ * counterpart in the pages; it is a deployment convenience.
  *   - Same arguments and results as msa_sparse_attn, minus the workspace.  The
  *     caller still passes inputs and outputs.
- *   - The partials live in one fixed 8 MiB array in the library's own device
- *     memory (every GPU that loads libmsa.so holds it until the process exits).
- *     Shapes whose partials do not fit (batch * n_q * H * splits * (d + 1) * 4
- *     bytes) return MSA_ERR_WORKSPACE; problems that run in one split (prefill)
- *     need none.
- *   - All calls share that array: calls whose work overlaps on the GPU (two
- *     streams, or two host threads) race and must be serialised by the caller.
+ *   - The intermediates live in one fixed 8 MiB array in the library's own
+ *     device memory (every GPU that loads libmsa.so holds it until the process
+ *     exits): the split-KV partials of decode-like shapes (batch * n_q * H *
+ *     splits * (d + 1) * 4 bytes) and, for prefill with d 64/128 and block
+ *     64/128, the inverted index and the per-block partial outputs of the
+ *     KV-major kernel (about n_q * h * topk * (G * (2 * d + 4) + 13) bytes per
+ *     sequence, plus 2 * d * 128 bytes per (group, block)), so only small
+ *     prefills fit.  Prefill with block 16/32 needs none.  Whatever does not
+ *     fit returns MSA_ERR_WORKSPACE before anything is launched
+ *     (msa_workspace_size(params, MSA_OP_SPARSE_ATTN) minus 256 is the need).
+ *   - All calls share that array and it keeps the last call's contents (the
+ *     parts that must start at zero are cleared on the stream by every call):
+ *     calls whose work overlaps on the GPU (two streams, or two host threads)
+ *     race and must be serialised by the caller.
  *   - The first call on a device looks up the array's device address; make that
  *     first call before any stream capture.
  *   - Device-side precondition failures (ids >= nblk, lengths outside

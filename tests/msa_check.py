@@ -152,3 +152,75 @@ def sample_rows(p, n_rows: int, seed: int = 0):
     while len(rows) < n_rows:
         rows.add((int(rng.integers(p.batch)), int(rng.integers(p.n_q))))
     return sorted(rows)
+
+
+def kv_chunk_rows(p) -> int:
+    """Query rows (flattened (b, t)) per chunk of the KV-major prefill attention.
+
+    Restates the library's chunk plan: a chunk's partial tiles and per-slot
+    records must fit a 6 GiB budget, next to one spare tile per (sequence,
+    group, block) list; chunk-relative slot positions stay below 2^30.  A CPU
+    test checks the resulting chunk count against msa_launch_count.
+    """
+    rows = p.batch * p.n_q
+    row_bytes = 2 * p.d
+    nj = p.batch * p.h * p.nblk
+    qpt = 128 // p.G
+    fixed = (nj + 1) * 128 * row_bytes
+    per_bt = p.h * p.topk * (12 + p.G * 4 + (128 * row_bytes) // qpt + 1)
+    budget = 6 << 30
+    cr = (budget - fixed) // per_bt if fixed < budget else 1
+    cr = max(cr, 1)
+    if cr * p.h * p.topk > (1 << 30):
+        cr = (1 << 30) // (p.h * p.topk)
+    return min(cr, rows)
+
+
+def sample_rows_chunked(p, n_rows: int, seed: int = 0, per_chunk_min: int = 64):
+    """Query rows for sampled prefill checks, stratified over the KV-major query
+    chunks: every chunk gets its first and last query, at least ``per_chunk_min``
+    rows and an equal share of ``n_rows``; the special rows of ``sample_rows``
+    (first blocks, partial own blocks, the last queries) are always included."""
+    rng = np.random.default_rng(seed)
+    rows = set(sample_rows(p, 0, seed))
+    total = p.batch * p.n_q
+    cr = kv_chunk_rows(p)
+    nch = (total + cr - 1) // cr
+    share = max(per_chunk_min, (n_rows - len(rows)) // nch)
+    for c in range(nch):
+        lo, hi = c * cr, min(total, (c + 1) * cr)
+        chosen = {lo, hi - 1}
+        want = min(share, hi - lo)
+        while len(chosen) < want:
+            chosen.add(int(rng.integers(lo, hi)))
+        for bt in chosen:
+            rows.add((bt // p.n_q, bt % p.n_q))
+    return sorted(rows)
+
+
+def page_pools(x, prob, spare: int = 5, seed: int = 0):
+    """Scatters the contiguous k, v and k_idx of ``x`` into shuffled page pools of
+    one block per page (plus ``spare`` unused pages of noise) on the tensors'
+    device; returns (pools, block table int32 [batch, nblk])."""
+    B, nb = prob.block, (prob.max_kv + prob.block - 1) // prob.block
+    n_pages = prob.batch * nb + spare
+    dev = x["k"].device
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    perm = torch.randperm(n_pages, generator=g)
+    table = perm[:prob.batch * nb].view(prob.batch, nb).to(torch.int32).to(dev)
+    unused = perm[prob.batch * nb:].to(dev)
+    gd = torch.Generator(device=dev).manual_seed(seed + 1)
+    pools = {}
+    for name in ("k", "v", "k_idx"):
+        t = x[name]
+        tail = tuple(t.shape[2:])
+        pool = torch.empty((n_pages, B) + tail, dtype=t.dtype, device=dev)
+        if spare:
+            pool[unused] = torch.randn((spare, B) + tail, generator=gd, device=dev).to(t.dtype)
+        for b in range(prob.batch):  # one sequence at a time bounds the staging memory
+            padded = torch.zeros((nb * B,) + tail, dtype=t.dtype, device=dev)
+            padded[:t.shape[1]] = t[b]
+            pool[table[b].long()] = padded.view((nb, B) + tail)
+            del padded
+        pools[name] = pool
+    return pools, table

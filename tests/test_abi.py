@@ -62,7 +62,45 @@ def test_workspace_size_host_only(lib):
     # status word + fp32 block scores [1, 1024, 2, 16] (+ ids for forward)
     assert sel >= 256 + 1024 * 2 * 16 * 4
     assert fwd >= sel + 1024 * 2 * 4 * 4
-    assert msa.msa_workspace_size(p, 7) == 0
+    assert msa.msa_workspace_size(p, 99) == 0
+    # the index scan alone, the candidate merge and the shard lengths need the
+    # status word only; the candidates call needs what index select needs
+    for op in (msa.MSA_OP_BLOCK_SCORES, msa.MSA_OP_SELECT_CANDIDATES, msa.MSA_OP_SHARD_LENGTHS,
+               msa.MSA_OP_APPEND_KV):
+        assert msa.msa_workspace_size(p, op) == 256
+    assert msa.msa_workspace_size(p, msa.MSA_OP_INDEX_CANDIDATES) == sel
+
+
+def test_sharded_decode_calls_validate_on_the_host(lib):
+    p = valid_params(n_q=1)
+    fake = 1 << 20  # never dereferenced: validation fails first
+    ws_small = 128
+    # candidate merge: empty or oversized lists, negative base, no output
+    sc = lib.msa_select_candidates
+    assert sc(ctypes.byref(p), 0, 4, 0, fake, fake, 0, 4, fake, None, fake, 4096,
+              None) == msa.MSA_ERR_INVALID_ARG
+    assert sc(ctypes.byref(p), 8, 4096, 0, fake, fake, 0, 4, fake, None, fake, 4096,
+              None) == msa.MSA_ERR_UNSUPPORTED
+    assert sc(ctypes.byref(p), 2, 4, 16, fake, fake, -1, 4, fake, None, fake, 4096,
+              None) == msa.MSA_ERR_INVALID_ARG
+    assert sc(ctypes.byref(p), 2, 4, 16, fake, fake, 0, 4, None, None, fake, 4096,
+              None) == msa.MSA_ERR_INVALID_ARG
+    assert sc(ctypes.byref(p), 2, 4, 16, fake, fake, 0, 4, fake, None, fake, ws_small,
+              None) == msa.MSA_ERR_WORKSPACE
+    # merge of partials: part count and alignment
+    assert lib.msa_merge_partials(ctypes.byref(p), 0, fake, fake, fake, None,
+                                  None) == msa.MSA_ERR_INVALID_ARG
+    assert lib.msa_merge_partials(ctypes.byref(p), 2, fake + 8, fake, fake, None,
+                                  None) == msa.MSA_ERR_INVALID_ARG
+    # shard lengths and the candidates call
+    assert lib.msa_shard_lengths(ctypes.byref(p), -1, 10, fake, fake, 4096,
+                                 None) == msa.MSA_ERR_INVALID_ARG
+    assert lib.msa_index_candidates(ctypes.byref(p), fake, fake, fake, None, fake, 1 << 30,
+                                    None) == msa.MSA_ERR_INVALID_ARG
+    assert lib.msa_block_scores(ctypes.byref(p), fake, fake, None, fake, 4096,
+                                None) == msa.MSA_ERR_INVALID_ARG
+    assert msa.msa_launch_count(p, msa.MSA_OP_INDEX_CANDIDATES) == 2
+    assert msa.msa_launch_count(p, msa.MSA_OP_SELECT_CANDIDATES) == 1
 
 
 @pytest.mark.parametrize("bad,code", [
@@ -145,3 +183,20 @@ def test_binding_fails_loudly_without_library(monkeypatch):
     monkeypatch.setattr(msa, "_lib", None)
     with pytest.raises(RuntimeError, match="not built"):
         msa.load_library()
+
+
+def test_prefill_chunk_plan_matches_the_library(lib):
+    # the parity tests stratify their sampled prefill rows by the KV-major query
+    # chunks; their restatement of the chunk plan must give the library's count
+    # (five kernels per chunk)
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.abspath(__file__)))
+    from msa_check import kv_chunk_rows
+    from block_sparse_gqa_03_b200.inputs import WORKLOADS
+    for name in ("prefill_1k", "prefill_32k", "prefill_128k"):
+        pr = WORKLOADS[name]
+        p = msa.make_params(batch=pr.batch, n_q=pr.n_q, max_kv=pr.max_kv, H=pr.H, h=pr.h,
+                            d=pr.d, d_idx=pr.d_idx, block=pr.block, topk=pr.topk)
+        rows = pr.batch * pr.n_q
+        nch = -(-rows // kv_chunk_rows(pr))
+        assert msa.msa_launch_count(p, msa.MSA_OP_SPARSE_ATTN) == 5 * nch, name

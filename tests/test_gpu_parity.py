@@ -13,8 +13,8 @@ import torch
 import oracle
 from block_sparse_gqa_03_b200 import msa
 from block_sparse_gqa_03_b200.inputs import WORKLOADS, Problem, make_inputs
-from msa_check import (check_attn, check_ids, check_scores, oracle_cfg, row_geometry,
-                       sample_rows, take_rows)
+from msa_check import (check_attn, check_ids, check_scores, oracle_cfg, page_pools,
+                       row_geometry, sample_rows_chunked, take_rows)
 
 pytestmark = pytest.mark.gpu
 
@@ -23,16 +23,31 @@ def host(t):
     return None if t is None else t.cpu()
 
 
-def run_and_check(prob: Problem, rows=None, tail_fill=None, with_oracle_ids=True, lens=None):
+def run_and_check(prob: Problem, rows=None, tail_fill=None, with_oracle_ids=True, lens=None,
+                  paged=False):
+    """Runs msa_index_select, msa_sparse_attn and msa_forward on the seeded inputs
+    of ``prob`` and checks every stage against the oracle on ``rows`` (default: all).
+    With ``paged`` the GPU reads K, V and K_idx from shuffled page pools through a
+    block table; the oracle always reads the contiguous tensors."""
     x = make_inputs(prob, device="cuda", tail_fill=tail_fill)
     if lens is not None:
         x["seq_lens"] = torch.tensor(lens, dtype=torch.int32, device="cuda")
     sl = x["seq_lens"]
     kw = dict(block=prob.block, causal=prob.causal, seq_lens=sl)
-    ids_g, sc_g = msa.msa_index_select(x["q_idx"], x["k_idx"], topk=prob.topk,
+    # host copies for the oracle before the cache is paged
+    q_h, k_h, v_h = host(x["q"]), host(x["k"]), host(x["v"])
+    qi_h, ki_h = host(x["q_idx"]), host(x["k_idx"])
+    dk, dv, dki = x["k"], x["v"], x["k_idx"]
+    if paged:
+        pools, table = page_pools(x, prob, seed=prob.seed)
+        dk, dv, dki = pools["k"], pools["v"], pools["k_idx"]
+        del x["k"], x["v"], x["k_idx"]
+        torch.cuda.empty_cache()
+        kw.update(block_table=table, max_kv=prob.max_kv)
+    ids_g, sc_g = msa.msa_index_select(x["q_idx"], dki, topk=prob.topk,
                                        force_own_block=prob.force_own, return_scores=True, **kw)
-    out_g, lse_g = msa.msa_sparse_attn(x["q"], x["k"], x["v"], ids_g, return_lse=True, **kw)
-    out_f, ids_f, lse_f = msa.msa_forward(x["q"], x["k"], x["v"], x["q_idx"], x["k_idx"],
+    out_g, lse_g = msa.msa_sparse_attn(x["q"], dk, dv, ids_g, return_lse=True, **kw)
+    out_f, ids_f, lse_f = msa.msa_forward(x["q"], dk, dv, x["q_idx"], dki,
                                           topk=prob.topk, force_own_block=prob.force_own,
                                           return_ids=True, return_lse=True, **kw)
     torch.cuda.synchronize()
@@ -45,7 +60,6 @@ def run_and_check(prob: Problem, rows=None, tail_fill=None, with_oracle_ids=True
         rows = [(b, t) for b in range(prob.batch) for t in range(prob.n_q)]
     cfg = oracle_cfg(prob)
     sl_h = host(sl)
-    qi_h, ki_h = host(x["q_idx"]), host(x["k_idx"])
     ora_sc = oracle.block_scores(cfg, qi_h, ki_h, seq_lens=sl_h, rows=rows)
     ora_ids = oracle.select(cfg, ora_sc, seq_lens=sl_h, rows=rows)
     gpu_sc = take_rows(sc_g, rows)
@@ -54,7 +68,6 @@ def run_and_check(prob: Problem, rows=None, tail_fill=None, with_oracle_ids=True
     check_scores(gpu_sc, ora_sc, F_rows)
     _, near = check_ids(prob, rows, sl_h, gpu_ids, ora_ids, ora_sc, gpu_sc)
 
-    q_h, k_h, v_h = host(x["q"]), host(x["k"]), host(x["v"])
     ora_out, ora_lse = oracle.sparse_attn(cfg, q_h, k_h, v_h, gpu_ids, seq_lens=sl_h, rows=rows)
     stats = check_attn(take_rows(out_g.float(), rows), take_rows(lse_g, rows), ora_out, ora_lse)
 
@@ -62,7 +75,7 @@ def run_and_check(prob: Problem, rows=None, tail_fill=None, with_oracle_ids=True
         # stage 2 in isolation on the oracle's own selection
         ids_o = torch.as_tensor(ora_ids.reshape(prob.batch, prob.n_q, prob.h, prob.topk),
                                 device="cuda")
-        out_o, lse_o = msa.msa_sparse_attn(x["q"], x["k"], x["v"], ids_o, return_lse=True, **kw)
+        out_o, lse_o = msa.msa_sparse_attn(x["q"], dk, dv, ids_o, return_lse=True, **kw)
         o2, l2 = oracle.sparse_attn(cfg, q_h, k_h, v_h, ora_ids, seq_lens=sl_h, rows=rows)
         check_attn(take_rows(out_o.float(), rows), take_rows(lse_o, rows), o2, l2)
     return x, ids_g, near, stats
@@ -141,14 +154,48 @@ def test_workload_decode_1m_varlen():
     run_and_check(WORKLOADS["decode_1m"], with_oracle_ids=False)
 
 
+# Prefill workloads: 2048 sampled query rows each, stratified over the KV-major
+# query chunks (3 at 32K, 18 at 128K) so that every chunk, its first and last
+# query included, is checked on at least 64 rows.
 def test_workload_prefill_32k_sampled():
     prob = WORKLOADS["prefill_32k"]
-    run_and_check(prob, rows=sample_rows(prob, 160, seed=3))
+    run_and_check(prob, rows=sample_rows_chunked(prob, 2048, seed=3))
 
 
 def test_workload_prefill_128k_sampled():
     prob = WORKLOADS["prefill_128k"]
-    run_and_check(prob, rows=sample_rows(prob, 48, seed=4))
+    run_and_check(prob, rows=sample_rows_chunked(prob, 2048, seed=4))
+
+
+# Paged KV cache against the oracle: the decode workloads' shapes (shuffled page
+# pools; the 1M lengths vary per sequence) and a prefill case on every row.
+def test_paged_decode_128k_against_oracle():
+    prob = WORKLOADS["decode_128k"].with_(batch=4)
+    x, ids_g, _, _ = run_and_check(prob, with_oracle_ids=False, paged=True)
+    ids = ids_g.cpu()
+    for b in range(prob.batch):
+        for g in range(prob.h):
+            assert set(x["planted"][b, g].tolist()) <= set(ids[b, 0, g].tolist())
+
+
+def test_paged_decode_1m_varlen_against_oracle():
+    run_and_check(WORKLOADS["decode_1m"], with_oracle_ids=False, paged=True)
+
+
+PAGED_PREFILL = [
+    # tcgen05 index GEMM (one page per 128-key tile), KV-major attention, block 128
+    Problem("paged_prefill_b128_oracle", batch=1, n_q=700, max_kv=2000, H=12, h=2, d=128,
+            d_idx=128, block=128, topk=5, causal=True, seed=211),
+    # two pages per index key tile, block-64 KV-major attention, own block forced,
+    # variable lengths
+    Problem("paged_prefill_b64_oracle", batch=2, n_q=400, max_kv=1100, H=8, h=2, d=64, d_idx=64,
+            block=64, topk=6, causal=True, force_own=True, seed=212, len_range=(600, 1100)),
+]
+
+
+@pytest.mark.parametrize("prob", PAGED_PREFILL, ids=lambda p: p.name)
+def test_paged_prefill_all_rows_against_oracle(prob):
+    run_and_check(prob, paged=True, tail_fill=float("nan") if prob.len_range else None)
 
 
 def test_ids_any_order_with_empty_slots():
