@@ -39,13 +39,15 @@ DEFAULT_WORKLOAD = "decode_128k"
 L2_BYTES = 126 * 2**20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
-# Per-launch DRAM traffic (read + write bytes) of the dominant kernel, from one ncu
-# capture at batch 4 scaled by 4 to the batch of 16 (the work grows in proportion):
-# profiles/sparse_attn_stream_decode128k_b4.md (134.46 MB read + 3.43 MB written).  The
-# index scan's capture (profiles/index_scan_stream_decode128k_b4.md, 134.27 MB read + 4.17 MB
-# written) predates its paged producer path, so its entry is absent until it is re-captured.
-# Absent entries report null; an entry is removed when its kernel changes.
-TRAFFIC = {("decode_128k", "attn"): 4 * (134.456832e6 + 3.434752e6)}
+# Per-launch DRAM traffic (read + write bytes) of a kernel, from one ncu capture
+# at batch 4 scaled by 4 to the workload's batch of 16 (the work grows in
+# proportion).  An entry is removed when its kernel changes; absent entries
+# report null.
+TRAFFIC = {
+    ("decode_128k", "attn"): 4 * (134.456832e6 + 3.434752e6),
+    ("decode_128k", "scan"): 4 * (134.275584e6 + 4.156672e6),
+}
+L2_FLUSH_BYTES = 256 * 2**20
 
 
 def load_peaks():
@@ -191,9 +193,10 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------- oracle arm
-def oracle_sample(prob, x, budget_s: float, max_rows: int | None = None):
+def oracle_sample(prob, x, budget_s: float, max_rows: int | None = None, collect=None):
     """Times the float64 oracle on a bounded sample: whole sequences for decode,
-    query rows for prefill.  Returns (units processed, seconds, description)."""
+    query rows for prefill.  Returns (units processed, seconds, description); with
+    ``collect`` (a list), appends (b, rows, ids, out) of every sampled sequence."""
     import numpy as np
     import oracle
 
@@ -210,9 +213,11 @@ def oracle_sample(prob, x, budget_s: float, max_rows: int | None = None):
             n = max_rows or 64
             rows = [(0, int(t)) for t in sorted(rng.choice(prob.n_q, size=n, replace=False))]
         t0 = time.perf_counter()
-        ids, _, _ = oracle.forward(cfg1, hb["q"], hb["k"], hb["v"], hb["q_idx"], hb["k_idx"],
-                                   seq_lens=sl, rows=rows)
+        ids, _, _lse = oracle.forward(cfg1, hb["q"], hb["k"], hb["v"], hb["q_idx"], hb["k_idx"],
+                                      seq_lens=sl, rows=rows)
         secs += time.perf_counter() - t0
+        if collect is not None:
+            collect.append((b, rows, ids, _))
         # work of the sampled rows, counted like the GPU's
         sub = prob.with_(batch=1)
         ids_t = torch.as_tensor(ids)
@@ -237,6 +242,48 @@ def oracle_sample(prob, x, budget_s: float, max_rows: int | None = None):
         desc = "%d query rows (%d per sequence, %d sequences), all groups and heads" % (
             nrows, nrows // max(1, nseq), nseq)
     return units, secs, desc
+
+
+def parity_stats(prob, x, ids, out, got, desc):
+    """The GPU's ids and outputs of the last timed step against the oracle's on the
+    CPU-baseline sample: rows whose ids are equal, rows that differ on a near tie
+    (the oracle's k-th and (k+1)-th block scores within 1e-3 relative), and the
+    output errors on rows with equal ids."""
+    import numpy as np
+    import oracle
+    rows_n = same = near = 0
+    errs = []
+    ids_h = ids.cpu().numpy()
+    out_h = out.float().cpu().numpy()
+    for b, rows, oid, oout in got:
+        tt = [t for _, t in rows]
+        gi = ids_h[b, tt]                      # [nrows, h, topk]
+        go = out_h[b, tt].reshape(oout.shape)  # [nrows, H, d]
+        eq = (gi == oid).all(axis=-1)          # [nrows, h]
+        rows_n += eq.size
+        same += int(eq.sum())
+        if not eq.all():
+            sub = prob.with_(batch=1)
+            cfg1 = oracle.Config(1, sub.n_q, sub.max_kv, sub.H, sub.h, sub.d, sub.d_idx,
+                                 sub.block, sub.topk, causal=sub.causal, force_own=sub.force_own)
+            sl = x["seq_lens"][b:b + 1].cpu() if x["seq_lens"] is not None else None
+            sc = oracle.block_scores(cfg1, x["q_idx"][b:b + 1].cpu(), x["k_idx"][b:b + 1].cpu(),
+                                     seq_lens=sl, rows=[(0, t) for t in tt])
+            for i, g in zip(*np.nonzero(~eq)):
+                v = np.sort(sc[i, g][np.isfinite(sc[i, g])])[::-1]
+                k = min(prob.topk, len(v))
+                if k < len(v) and (v[k - 1] - v[k]) / max(abs(v[k - 1]), abs(v[k]), 1e-6) < 1e-3:
+                    near += 1
+        for i in range(len(tt)):
+            for g in range(prob.h):
+                if eq[i, g]:
+                    errs.append(np.abs(go[i, g * prob.G:(g + 1) * prob.G] -
+                                       oout[i, g * prob.G:(g + 1) * prob.G]))
+    e = np.concatenate([a.ravel() for a in errs]) if errs else np.zeros(1)
+    return {"rows": rows_n, "ids_equal": same, "near_tie_rows": near,
+            "other_mismatch_rows": rows_n - same - near, "max_abs": float(e.max()),
+            "mean_abs": float(e.mean()), "tolerance": {"max_abs": 2e-2, "mean_abs": 2e-3},
+            "oracle": "float64", "sample": desc}
 
 
 def unit_of(prob):
@@ -352,40 +399,104 @@ def run_ours(args, prob, world, rank, local):
     touched = units["select"] + units["attn"] if prob.is_decode else None
 
     K = args.steps
-    t_start = torch.cuda.Event(enable_timing=True)
-    t_end = torch.cuda.Event(enable_timing=True)
     props = torch.cuda.get_device_properties(dev)
     uuid = str(getattr(props, "uuid", "")) or None
     if uuid and not uuid.startswith("GPU-"):
         uuid = "GPU-" + uuid
-    barrier(world)
-    torch.cuda.synchronize(dev)
+    flush_buf = (torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+                 if args.l2_flush else None)
+
+    def timed_loop():
+        """K steps bracketed by a barrier and a synchronize on both sides; returns the
+        per-step device times (ms) of the loop: one figure (loop / K) when the steps
+        run back to back, K figures when the L2 is flushed before every step."""
+        barrier(world)
+        torch.cuda.synchronize(dev)
+        if flush_buf is None:
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(K):
+                step()
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            times = [e0.elapsed_time(e1) / K]
+        else:
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(K)]
+            for e0, e1 in ev:
+                flush_buf.fill_(1.0)  # a write larger than L2, outside the timed span
+                e0.record(stream)
+                step()
+                e1.record(stream)
+            torch.cuda.synchronize(dev)
+            times = [e0.elapsed_time(e1) for e0, e1 in ev]
+        barrier(world)
+        return times
+
+    # the K-step loop is repeated until at least --min-ms of device time is timed,
+    # so that the clock samples fall inside it and the spread is measured
+    # (every rank must run the same number of loops: the largest calibration rules)
+    calib = max_over_ranks(sum(timed_loop()) * (K if flush_buf is None else 1), world)
+    repeats = max(1, min(args.max_repeats, -(-int(args.min_ms) // max(1, int(calib)))))
+    step_times = []
     with ClockSampler(uuid) as clk:
         h0 = time.perf_counter()
-        t_start.record(stream)
-        for i in range(K):
-            step()
-        t_end.record(stream)
-        torch.cuda.synchronize(dev)
+        for _ in range(repeats):
+            step_times.extend(timed_loop())
         clk.mark(h0, time.perf_counter())
-    barrier(world)
-    total_ms = max_over_ranks(t_start.elapsed_time(t_end), world)
-    # per-stage times (for the stage split and the roofline of the dominant stage):
-    # the two calls apart, events between them, outside the timed region
-    ks = min(K, 20)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(ks)]
-    for i in range(ks):
-        ev[i][0].record(stream)
-        msa.msa_index_select(x["q_idx"], x["k_idx"], topk=prob.topk,
-                             force_own_block=prob.force_own, block_ids=ids, workspace=ws, **kw)
-        ev[i][1].record(stream)
-        msa.msa_sparse_attn(x["q"], x["k"], x["v"], ids, out=out, workspace=ws, **kw)
-        ev[i][2].record(stream)
-    torch.cuda.synchronize(dev)
-    sel_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
-    attn_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+    step_times.sort()
+
+    def pct(q):
+        return step_times[min(len(step_times) - 1, int(q * (len(step_times) - 1) + 0.5))]
+
+    med_ms = max_over_ranks(statistics.median(step_times), world)
+    step_stats = {"median_ms": med_ms, "p10_ms": max_over_ranks(pct(0.1), world),
+                  "p90_ms": max_over_ranks(pct(0.9), world),
+                  "mean_ms": max_over_ranks(statistics.mean(step_times), world),
+                  "repeats": repeats, "steps_per_repeat": K,
+                  "timed_ms": max_over_ranks(sum(step_times) * (K if flush_buf is None else 1),
+                                             world),
+                  "per": "K-step loop / K" if flush_buf is None else "step"}
+
+    # per-kernel times (for the roofline of the dominant kernel), measured apart
+    # from the timed region with events around each call: the index scan alone
+    # (msa_block_scores), scan + top-k (msa_index_select) and the attention call
+    # (msa_sparse_attn: its merge-counter memset and kernel; prefill: the whole
+    # KV-major stage)
+    scores_buf = torch.empty((prob.batch, prob.n_q, prob.h, prob.nblk), dtype=torch.float32,
+                             device=dev)
+    ks = max(5, min(20, int(200.0 / max(med_ms, 1e-3))))
+    calls = {
+        "scan": lambda: msa.msa_block_scores(x["q_idx"], x["k_idx"], block=prob.block,
+                                             causal=prob.causal, seq_lens=sl,
+                                             block_scores=scores_buf, workspace=ws,
+                                             **{k: kw[k] for k in ("block_table", "max_kv")
+                                                if k in kw}),
+        "select": lambda: msa.msa_index_select(x["q_idx"], x["k_idx"], topk=prob.topk,
+                                               force_own_block=prob.force_own, block_ids=ids,
+                                               workspace=ws, **kw),
+        "attn": lambda: msa.msa_sparse_attn(x["q"], x["k"], x["v"], ids, out=out, workspace=ws,
+                                            **kw),
+    }
+    stage = {}
+    for name, fn in calls.items():
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(ks)]
+        fn()
+        for e0, e1 in ev:
+            if flush_buf is not None:
+                flush_buf.fill_(1.0)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
+        stage[name] = statistics.median(e0.elapsed_time(e1) for e0, e1 in ev)
     assert msa.msa_get_device_status(ws) == msa.MSA_OK
-    ms_per_step = total_ms / K
+    sel_ms, attn_ms = stage["select"], stage["attn"]
+    kern_ms = {"scan": stage["scan"], "topk": max(0.0, stage["select"] - stage["scan"]),
+               "attn": stage["attn"]}
+    ms_per_step = med_ms
     unit, scale = unit_of(prob)
     total_units = (units["select"] + units["attn"]) * world
     value = total_units / (ms_per_step * 1e-3) / scale
@@ -401,25 +512,44 @@ def run_ours(args, prob, world, rank, local):
     launches_per_step = msa.msa_launch_count(p_sel, msa.MSA_OP_FORWARD)
 
     peaks, peak_kind = load_peaks()
-    dom = "attn" if attn_ms >= sel_ms else "select"
-    dom_ms = attn_ms if dom == "attn" else sel_ms
     if prob.is_decode:
-        kernel = {"attn": "sparse_attn_stream_kernel",
-                  "select": "index_scan_stream_kernel (+topk)"}[dom]
+        names = {"scan": "index_scan_stream_kernel", "attn": "sparse_attn_stream_kernel"}
+        work = {"scan": units["select"], "attn": units["attn"]}
     else:
-        kernel = {"attn": "kv_attn_kernel (+count/scan/scatter, combine)",
-                  "select": "index_score_tc_kernel (+topk)"}[dom]
-    if prob.is_decode:
-        roof = {"bound": "hbm", "achieved": units[dom] / (dom_ms * 1e-3) / 1e9,
-                "peak": peaks["hbm_gbs"], "unit": "GB/s"}
-    else:
-        key = "bf16_tflops_sustained" if ms_per_step > 50 else "bf16_tflops"
-        roof = {"bound": "tensor", "achieved": units[dom] / (dom_ms * 1e-3) / 1e12,
-                "peak": peaks.get(key, FALLBACK_PEAKS[key]), "unit": "TFLOP/s"}
-    roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = TRAFFIC.get((prob.name, dom))
-    roof["kernel"] = kernel
-    roof["peak_source"] = "of %s" % peak_kind
+        names = {"scan": "index_score_tc_kernel",
+                 "attn": "sparse attention stage (inverted index, kv_attn_kernel, combine)"}
+        work = {"scan": units["select"], "attn": units["attn"]}
+    dom = "attn" if kern_ms["attn"] >= kern_ms["scan"] else "scan"
+
+    def roof_of(k):
+        if prob.is_decode:
+            r = {"bound": "hbm", "achieved": work[k] / (kern_ms[k] * 1e-3) / 1e9,
+                 "peak": peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]), "unit": "GB/s"}
+        else:
+            r = {"bound": "tensor", "achieved": work[k] / (kern_ms[k] * 1e-3) / 1e12,
+                 "peak": peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]),
+                 "unit": "TFLOP/s"}
+            sus = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+            r["frac_of_sustained_peak"] = r["achieved"] / sus
+        r["frac"] = r["achieved"] / r["peak"]
+        r["kernel"] = names[k]
+        r["ms"] = kern_ms[k]
+        return r
+
+    # the captured traffic holds for the workload as defined (not for overridden sizes)
+    stock = prob == WORKLOADS.get(prob.name) and not args.paged
+    roof = roof_of(dom)
+    roof["traffic"] = TRAFFIC.get((prob.name, dom)) if stock else None
+    roof["peak_source"] = "of %s (%s)" % (peak_kind, "copy" if prob.is_decode else "burst bf16")
+    other = "scan" if dom == "attn" else "attn"
+    o = roof_of(other)
+    o["traffic"] = TRAFFIC.get((prob.name, other)) if stock else None
+    roof["other_kernels"] = [o, {"kernel": "topk_%s_kernel" % ("cta" if prob.nblk > 1024
+                                                               else "warp"),
+                                 "ms": kern_ms["topk"]}]
+    if not prob.is_decode:
+        # the whole step against the dense bf16 peak (the prefill target)
+        roof["step_frac_of_peak"] = value / roof["peak"]
 
     line = {
         "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": K,
@@ -429,14 +559,18 @@ def run_ours(args, prob, world, rank, local):
         "config": {"workload": prob.name, **workload_config(prob),
                    "kv_cache": "paged (one block per page, shuffled pool)" if args.paged
                    else "contiguous",
-                   "l2": ("inputs larger than L2 (%.2f GB touched per step)" % (touched / 1e9)
-                          if touched else "inputs larger than L2"),
+                   "l2": ("flushed before every step (%d MiB written), each step timed alone"
+                          % (L2_FLUSH_BYTES >> 20) if args.l2_flush else
+                          "no flush: inputs larger than L2 (%.2f GB touched per step)"
+                          % (touched / 1e9) if touched else
+                          "no flush: inputs larger than L2"),
                    "parallelism": "replicas" if world > 1 else "single GPU"},
         "us_per_step": 1e3 * ms_per_step,
-        "stage_ms": {"index_select": sel_ms, "sparse_attn": attn_ms},
+        "step_ms": step_stats,
+        "stage_ms": {"index_scan": stage["scan"], "index_select": sel_ms, "sparse_attn": attn_ms},
         "roofline": roof,
         "e2e": e2e,
-        "gpu_launches": launches_per_step * K,
+        "gpu_launches": launches_per_step * K * repeats,
     }
     if prob.is_decode:
         line["tokens_per_s"] = prob.batch * world / (ms_per_step * 1e-3)
@@ -444,10 +578,13 @@ def run_ours(args, prob, world, rank, local):
         line["clocks"] = clk.summary()
         if world == 1 and not args.no_cpu_baseline and not args.paged:
             import oracle
-            u, s, desc = oracle_sample(prob, {k: v for k, v in x.items()}, args.cpu_budget)
+            got = []
+            u, s, desc = oracle_sample(prob, {k: v for k, v in x.items()}, args.cpu_budget,
+                                       collect=got)
             line["cpu_baseline"] = {"value": u / s / scale, "unit": unit,
                                     "cores": oracle.num_threads(), "kind": "oracle",
                                     "sample": desc}
+            line["parity"] = parity_stats(prob, x, ids, out, got, desc)
         print(json.dumps(line), flush=True)
 
 
@@ -574,6 +711,12 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default=DEFAULT_WORKLOAD)
     ap.add_argument("--cpu-budget", type=float, default=10.0)
+    ap.add_argument("--min-ms", type=float, default=200.0,
+                    help="repeat the K-step loop until this much device time is timed")
+    ap.add_argument("--max-repeats", type=int, default=400)
+    ap.add_argument("--l2-flush", action="store_true",
+                    help="write a buffer larger than L2 before every step and time each step "
+                         "alone")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--batch", type=int, default=0,

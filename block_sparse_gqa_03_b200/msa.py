@@ -455,14 +455,17 @@ def msa_select_candidates(cand_scores, cand_ids, *, max_kv, block, topk, shard_b
     return block_ids, local_ids
 
 
-def msa_merge_partials(part_out, part_lse, *, out=None, lse=None, stream=None):
-    """LSE merge of part_out bf16 [P, b, n_q, H, d] with part_lse fp32 [P, b, n_q, H]."""
+def msa_merge_partials(part_out, part_lse, *, out=None, lse=None, h=None, stream=None):
+    """LSE merge of part_out bf16 [P, b, n_q, H, d] with part_lse fp32 [P, b, n_q, H].
+    ``h`` (the KV heads) only has to make a valid head grouping of H."""
     P, b, n_q, H, d = part_out.shape
     if not (part_out.is_contiguous() and part_lse.is_contiguous()):
         raise ValueError("partials must be dense")
     if out is None:
         out = torch.empty((b, n_q, H, d), dtype=part_out.dtype, device=part_out.device)
-    p = make_params(batch=b, n_q=n_q, max_kv=max(n_q, 1), H=H, h=H, d=d, d_idx=32, block=64,
+    if h is None:
+        h = next((c for c in range(1, 17) if H % c == 0 and H // c <= 16), 1)
+    p = make_params(batch=b, n_q=n_q, max_kv=max(n_q, 1), H=H, h=h, d=d, d_idx=32, block=64,
                     topk=1, out=out)
     _check(load_library().msa_merge_partials(ctypes.byref(p), int(P), _ptr(part_out),
                                              _ptr(part_lse), _ptr(out), _ptr(lse),
