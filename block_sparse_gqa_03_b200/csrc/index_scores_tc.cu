@@ -21,6 +21,17 @@
 // Accumulators are double-buffered (2 x 2 groups x 128 columns = 512 columns), so
 // the epilogue of one key tile overlaps the MMAs of the next.  Every mbarrier wait
 // is bounded and records an error instead of hanging.
+//
+// Streaming top-k (the TOPK instantiation): the block scores need not reach HBM
+// at all.  Each epilogue thread owns one (query, group) row and keeps the row's
+// best blocks so far in a min-heap in shared memory (the root is the worst kept
+// block: lowest score, then highest id), laid out [entry][row] so that the 32
+// lanes of a warp touch 32 banks.  Blocks arrive in increasing id order, so a new
+// block enters exactly when its score beats the root's (on equal scores the kept,
+// lower id wins).  After the sweep the thread sorts its ids and writes them.  This
+// follows the FlashMoBA top-k kernel's idea ("混合块注意力机制(MoBA)原理与实现详解",
+// section 3.1, kernel 2: sorted top-k lists in SRAM instead of the score matrix in
+// HBM); the heap costs the key ring two of its stages at d_idx 128.
 #include "kernels.h"
 #include "sm100.cuh"
 
@@ -42,9 +53,34 @@ struct TcArgs {
   DeviceStatus* st;
   uint64_t wait_ns;
   KvPages pg;  // table == nullptr: contiguous K_idx
+  // streaming top-k: ids [b, n_q, h, topk]; scores (above) optional
+  int32_t* ids;
+  int topk, force_own;
 };
 
-template <int DI, int BLK>
+constexpr int kHeapMax = 64;    // top-k the streaming variant takes
+constexpr int kHeapRows = kNG * kQT;  // rows (query, group) of a CTA
+
+// Sorts v[0..N) ascending (bitonic network, fully unrolled: v stays in registers).
+template <int N>
+__device__ __forceinline__ void bitonic_sort(uint32_t (&v)[N]) {
+#pragma unroll
+  for (int k = 2; k <= N; k <<= 1)
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1)
+#pragma unroll
+      for (int i = 0; i < N; ++i) {
+        const int l = i ^ j;
+        if (l > i) {
+          const bool up = (i & k) == 0;
+          const uint32_t x = v[i], y = v[l];
+          v[i] = up ? min(x, y) : max(x, y);
+          v[l] = up ? max(x, y) : min(x, y);
+        }
+      }
+}
+
+template <int DI, int BLK, bool TOPK>
 __global__ void __launch_bounds__(kTcThreads, 1)
     index_score_tc_kernel(const __grid_constant__ CUtensorMap tmq,
                           const __grid_constant__ CUtensorMap tmk, TcArgs a) {
@@ -60,7 +96,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                                              ~uintptr_t(1023));
   const uint32_t q_base = smem_u32(smem);
   const uint32_t k_base = q_base + kNG * Q_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kNG * Q_BYTES + a.stages * K_BYTES);
+  // streaming top-k heaps: scores [kHeapMax][kHeapRows] f32, ids [kHeapMax][kHeapRows] u16
+  float* heap_s = reinterpret_cast<float*>(smem + kNG * Q_BYTES + a.stages * K_BYTES);
+  uint16_t* heap_i = reinterpret_cast<uint16_t*>(heap_s + (TOPK ? kHeapMax * kHeapRows : 0));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(
+      smem + kNG * Q_BYTES + a.stages * K_BYTES + (TOPK ? kHeapMax * kHeapRows * 6 : 0));
   const uint32_t b_qfull = smem_u32(bars);
   const uint32_t b_kfull = b_qfull + 8;
   const uint32_t b_kempty = b_kfull + 8 * a.stages;
@@ -192,7 +232,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     constexpr int bpt = kKT / BLK;  // blocks per key tile
     const float ninf = -__int_as_float(0x7f800000);
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
-    float* srow = a.scores + (((int64_t)b * a.n_q + t) * a.h + gp * kNG + ng) * (int64_t)a.nblk;
+    const int64_t rowi = ((int64_t)b * a.n_q + t) * a.h + gp * kNG + ng;
+    float* srow = a.scores ? a.scores + rowi * (int64_t)a.nblk : nullptr;
+    // streaming top-k state: the heap holds `cap` entries (the forced own block is
+    // kept aside), `root` caches the heap root's score
+    const int hr = ng * kQT + row;  // this thread's heap column
+    const int nb_row = (L + BLK - 1) / BLK;
+    const int F = row_ok ? (a.causal ? (p < 0 ? 0 : min(nb_row, p / BLK + 1)) : nb_row) : 0;
+    const int own = (TOPK && a.force_own && row_ok && p >= 0 && p / BLK < F) ? p / BLK : -1;
+    const int cap = TOPK ? a.topk - (own >= 0 ? 1 : 0) : 0;
+    float root = ninf;
+    if (TOPK) {
+      for (int i = 0; i < cap; ++i) {
+        heap_s[i * kHeapRows + hr] = ninf;
+        heap_i[i * kHeapRows + hr] = 0xffffu;
+      }
+    }
     for (int kt = 0; kt < n_kt && ng < ng_valid; ++kt) {
       const int buf = kt & 1;
       if (!mbar_wait_warp(b_afull + 8 * buf, (kt >> 1) & 1, a.st, 0x106u, a.wait_ns)) break;
@@ -227,13 +282,68 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           bm[col / BLK] = fmaxf(bm[col / BLK], col < vis ? v[col] : ninf);
       }
       if (row_ok) {
+        if (srow != nullptr) {
 #pragma unroll
-        for (int k = 0; k < bpt; ++k)
-          if (j0 / BLK + k < a.nblk) srow[j0 / BLK + k] = bm[k];
+          for (int k = 0; k < bpt; ++k)
+            if (j0 / BLK + k < a.nblk) srow[j0 / BLK + k] = bm[k];
+        }
+        if constexpr (TOPK) {
+#pragma unroll
+          for (int k = 0; k < bpt; ++k) {
+            const int beta = j0 / BLK + k;
+            const float sc = bm[k];
+            if (sc > root && beta != own && cap > 0) {
+              // replace the root, sift the new entry down (worse children move up)
+              int pos = 0;
+              for (;;) {
+                int c = 2 * pos + 1;
+                if (c >= cap) break;
+                float cs = heap_s[c * kHeapRows + hr];
+                uint32_t ci = heap_i[c * kHeapRows + hr];
+                if (c + 1 < cap) {
+                  const float s2 = heap_s[(c + 1) * kHeapRows + hr];
+                  const uint32_t i2 = heap_i[(c + 1) * kHeapRows + hr];
+                  if (s2 < cs || (s2 == cs && i2 > ci)) {
+                    c = c + 1;
+                    cs = s2;
+                    ci = i2;
+                  }
+                }
+                if (cs < sc || (cs == sc && ci > (uint32_t)beta)) {
+                  heap_s[pos * kHeapRows + hr] = cs;
+                  heap_i[pos * kHeapRows + hr] = (uint16_t)ci;
+                  pos = c;
+                } else {
+                  break;
+                }
+              }
+              heap_s[pos * kHeapRows + hr] = sc;
+              heap_i[pos * kHeapRows + hr] = (uint16_t)beta;
+              root = heap_s[hr];
+            }
+          }
+        }
       }
     }
-    if (a.fill_tail && row_ok && ng < ng_valid)
+    if (srow != nullptr && a.fill_tail && row_ok && ng < ng_valid)
       for (int beta = n_kt * bpt; beta < a.nblk; ++beta) srow[beta] = ninf;
+    if constexpr (TOPK) {
+      if (row_ok && ng < ng_valid) {
+        // the kept ids (empty entries are 0xffff and sort last) and the forced own
+        // block, in ascending order, then -1 padding
+        uint32_t v[kHeapMax];
+#pragma unroll
+        for (int i = 0; i < kHeapMax; ++i)
+          v[i] = i < cap ? (uint32_t)heap_i[i * kHeapRows + hr]
+                         : (i == cap && own >= 0 ? (uint32_t)own : 0xffffu);
+        bitonic_sort<kHeapMax>(v);
+        const int m = min(a.topk, F);
+        int32_t* out = a.ids + rowi * a.topk;
+#pragma unroll
+        for (int i = 0; i < kHeapMax; ++i)
+          if (i < a.topk) out[i] = i < m ? (int32_t)v[i] : -1;
+      }
+    }
   }
   tc::fence_before_sync();
   __syncthreads();
@@ -243,7 +353,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   }
 }
 
-template <int DI, int BLK>
+template <int DI, int BLK, bool TOPK>
 cudaError_t run_tc(const Shape& s, const uint16_t* q_idx, const uint16_t* k_idx, TcArgs& a,
                    cudaStream_t stream) {
   EncodeTiledFn enc = encode_fn();
@@ -276,14 +386,19 @@ cudaError_t run_tc(const Shape& s, const uint16_t* q_idx, const uint16_t* k_idx,
       return cudaErrorInvalidValue;
   }
   constexpr uint32_t tile = (DI / 64) * 128u * 128u;
+  constexpr size_t heap = TOPK ? (size_t)kHeapMax * kHeapRows * 6 : 0;
   a.stages = DI == 128 ? 4 : 8;
-  const size_t smem = 1024 + kNG * tile + (size_t)a.stages * tile + 8 * (1 + 2 * a.stages + 5) + 16;
-  cudaError_t err = cudaFuncSetAttribute(index_score_tc_kernel<DI, BLK>,
+  auto bytes = [&](int st) {
+    return 1024 + kNG * tile + (size_t)st * tile + heap + 8 * (1 + 2 * st + 5) + 16;
+  };
+  while (a.stages > 2 && bytes(a.stages) > (size_t)max_smem_optin()) --a.stages;
+  const size_t smem = bytes(a.stages);
+  cudaError_t err = cudaFuncSetAttribute(index_score_tc_kernel<DI, BLK, TOPK>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   const unsigned grid = (unsigned)((int64_t)s.batch * a.n_gpairs * a.n_mtiles);
-  return launch_pdl(index_score_tc_kernel<DI, BLK>, dim3(grid), dim3(kTcThreads), smem, stream,
-                    tmq, tmk, a);
+  return launch_pdl(index_score_tc_kernel<DI, BLK, TOPK>, dim3(grid), dim3(kTcThreads), smem,
+                    stream, tmq, tmk, a);
 }
 
 }  // namespace
@@ -311,8 +426,11 @@ cudaError_t launch_index_scores_tc(const Shape& s, const uint16_t* q_idx, const 
   a.st = st;
   a.wait_ns = 4000000000ull;
   a.pg = s.pages;
+  a.ids = nullptr;
+  a.topk = s.topk;
+  a.force_own = s.force_own;
 #define MSA_TC_CASE(DI_, BLK_) \
-  if (s.d_idx == DI_ && s.block == BLK_) return run_tc<DI_, BLK_>(s, q_idx, k_idx, a, stream);
+  if (s.d_idx == DI_ && s.block == BLK_) return run_tc<DI_, BLK_, false>(s, q_idx, k_idx, a, stream);
   MSA_TC_CASE(128, 16)
   MSA_TC_CASE(128, 32)
   MSA_TC_CASE(128, 64)
@@ -322,6 +440,41 @@ cudaError_t launch_index_scores_tc(const Shape& s, const uint16_t* q_idx, const 
   MSA_TC_CASE(64, 64)
   MSA_TC_CASE(64, 128)
 #undef MSA_TC_CASE
+  return cudaErrorInvalidValue;
+}
+
+bool index_topk_tc_supported(const Shape& s) {
+  return index_scores_tc_supported(s) && (s.block == 64 || s.block == 128) &&
+         s.topk <= kHeapMax && s.nblk <= 0xffff;
+}
+
+cudaError_t launch_index_topk_tc(const Shape& s, const uint16_t* q_idx, const uint16_t* k_idx,
+                                 int32_t* ids, float* scores, DeviceStatus* st,
+                                 cudaStream_t stream) {
+  if (!index_topk_tc_supported(s)) return cudaErrorInvalidValue;
+  TcArgs a;
+  a.batch = s.batch;
+  a.n_q = s.n_q;
+  a.max_kv = s.max_kv;
+  a.h = s.h;
+  a.block = s.block;
+  a.nblk = s.nblk;
+  a.causal = s.causal;
+  a.seq_lens = s.seq_lens;
+  a.n_mtiles = (s.n_q + kQT - 1) / kQT;
+  a.n_gpairs = (s.h + kNG - 1) / kNG;
+  a.scores = scores;
+  a.fill_tail = 1;
+  a.st = st;
+  a.wait_ns = 4000000000ull;
+  a.pg = s.pages;
+  a.ids = ids;
+  a.topk = s.topk;
+  a.force_own = s.force_own;
+  if (s.d_idx == 128 && s.block == 128) return run_tc<128, 128, true>(s, q_idx, k_idx, a, stream);
+  if (s.d_idx == 128 && s.block == 64) return run_tc<128, 64, true>(s, q_idx, k_idx, a, stream);
+  if (s.d_idx == 64 && s.block == 128) return run_tc<64, 128, true>(s, q_idx, k_idx, a, stream);
+  if (s.d_idx == 64 && s.block == 64) return run_tc<64, 64, true>(s, q_idx, k_idx, a, stream);
   return cudaErrorInvalidValue;
 }
 

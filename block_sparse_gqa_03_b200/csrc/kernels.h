@@ -31,6 +31,14 @@ cudaError_t launch_index_scores_tc(const Shape& s, const uint16_t* q_idx, const 
                                    float* scores, bool fill_tail, DeviceStatus* st,
                                    cudaStream_t stream);
 
+// Stage 1 in one kernel for prefill (d_idx 64/128, block 64/128, topk <= 64): the
+// index GEMM keeps a per-row top-k in shared memory; block scores written only
+// when `scores` is given (every block, -inf past the frontier).
+bool index_topk_tc_supported(const Shape& s);
+cudaError_t launch_index_topk_tc(const Shape& s, const uint16_t* q_idx, const uint16_t* k_idx,
+                                 int32_t* ids, float* scores, DeviceStatus* st,
+                                 cudaStream_t stream);
+
 // Stage 1c: top-k block ids, int32 [batch, n_q, h, topk], from the scores.  When
 // `zero` is given, the kernel also clears zero[0, nzero) (the attention's merge
 // counters, so that a fused forward needs no separate memset between the stages).

@@ -205,7 +205,7 @@ Layout layout(const Shape& s, msa_op_t op) {
 // Operations whose workspace holds the status word only.
 bool status_only(msa_op_t op) {
   return op == MSA_OP_APPEND_KV || op == MSA_OP_BLOCK_SCORES || op == MSA_OP_SELECT_CANDIDATES ||
-         op == MSA_OP_SHARD_LENGTHS;
+         op == MSA_OP_SHARD_LENGTHS || op == MSA_OP_INDEX_TOPK;
 }
 
 msa_status_t check_ws(const Shape& s, msa_op_t op, void* ws, size_t bytes) {
@@ -265,6 +265,21 @@ msa_status_t msa_block_scores(const msa_params_t* params, const msa_bf16_t* q_id
   return cuda_status(run_scores(s, q_idx, k_idx, block_scores, true,
                                 reinterpret_cast<msa::DeviceStatus*>(workspace),
                                 reinterpret_cast<cudaStream_t>(stream)));
+}
+
+msa_status_t msa_index_topk(const msa_params_t* params, const msa_bf16_t* q_idx,
+                            const msa_bf16_t* k_idx, int32_t* block_ids, float* block_scores,
+                            void* workspace, size_t workspace_bytes, msa_stream_t stream) {
+  Shape s;
+  msa_status_t rc = make_shape(params, &s);
+  if (rc != MSA_OK) return rc;
+  if ((rc = check_select_args(s, q_idx, k_idx)) != MSA_OK) return rc;
+  if (block_ids == nullptr) return MSA_ERR_INVALID_ARG;
+  if (!msa::index_topk_tc_supported(s)) return MSA_ERR_UNSUPPORTED;
+  if ((rc = check_ws(s, MSA_OP_INDEX_TOPK, workspace, workspace_bytes)) != MSA_OK) return rc;
+  return cuda_status(msa::launch_index_topk_tc(s, q_idx, k_idx, block_ids, block_scores,
+                                               reinterpret_cast<msa::DeviceStatus*>(workspace),
+                                               reinterpret_cast<cudaStream_t>(stream)));
 }
 
 msa_status_t msa_index_candidates(const msa_params_t* params, const msa_bf16_t* q_idx,
@@ -455,6 +470,7 @@ int msa_launch_count(const msa_params_t* params, msa_op_t op) {
     case MSA_OP_INDEX_CANDIDATES: return 2;
     case MSA_OP_SELECT_CANDIDATES: return 1;
     case MSA_OP_SHARD_LENGTHS: return 1;
+    case MSA_OP_INDEX_TOPK: return 1;
   }
   return -1;
 }

@@ -37,12 +37,13 @@ MSA_OP_BLOCK_SCORES = 4
 MSA_OP_INDEX_CANDIDATES = 5
 MSA_OP_SELECT_CANDIDATES = 6
 MSA_OP_SHARD_LENGTHS = 7
+MSA_OP_INDEX_TOPK = 8
 
 EXPORTED = ("msa_workspace_size", "msa_index_select", "msa_sparse_attn", "msa_forward",
             "msa_get_device_status", "msa_workspace_init", "msa_selftest_wait_timeout",
             "msa_launch_count", "msa_sparse_attn_noalloc", "msa_status_string", "msa_append_kv",
             "msa_block_scores", "msa_index_candidates", "msa_select_candidates",
-            "msa_merge_partials", "msa_shard_lengths")
+            "msa_merge_partials", "msa_shard_lengths", "msa_index_topk")
 
 
 class MsaError(RuntimeError):
@@ -103,6 +104,8 @@ def load_library():
             lib.msa_selftest_wait_timeout.restype = I
             lib.msa_sparse_attn_noalloc.argtypes = [P, P, P, P, P, P, P, P]
             lib.msa_sparse_attn_noalloc.restype = I
+            lib.msa_index_topk.argtypes = [P, P, P, P, P, P, S, P]
+            lib.msa_index_topk.restype = I
             lib.msa_block_scores.argtypes = [P, P, P, P, P, S, P]
             lib.msa_block_scores.restype = I
             lib.msa_index_candidates.argtypes = [P, P, P, P, P, P, S, P]
@@ -486,4 +489,29 @@ def msa_shard_lengths(seq_lens, *, batch, max_kv, token_base, token_count, out=N
                                             _ptr(out), ws.data_ptr(), ws.numel(),
                                             _stream(stream)), "msa_shard_lengths")
     return out
+
+
+def msa_index_topk(q_idx, k_idx, *, block, topk, causal=True, force_own_block=False,
+                   seq_lens=None, return_scores=False, block_ids=None, block_scores=None,
+                   block_table=None, max_kv=None, workspace: Workspace | None = None,
+                   stream=None):
+    """Stage 1 for prefill in one kernel (the top-k kept in the index GEMM's epilogue):
+    the ids of msa_index_select, and the block scores only if asked."""
+    b, n_q, h, d_idx = q_idx.shape
+    max_kv, num_pages = _kv_extent(k_idx, block_table, max_kv)
+    nblk = (max_kv + block - 1) // block
+    p = make_params(batch=b, n_q=n_q, max_kv=max_kv, H=h, h=h, d=64, d_idx=d_idx, block=block,
+                    topk=topk, causal=causal, force_own_block=force_own_block,
+                    seq_lens=seq_lens, q_idx=q_idx, k_idx=k_idx, block_table=block_table,
+                    num_pages=num_pages)
+    dev = q_idx.device
+    if block_ids is None:
+        block_ids = torch.empty((b, n_q, h, topk), dtype=torch.int32, device=dev)
+    if return_scores and block_scores is None:
+        block_scores = torch.empty((b, n_q, h, nblk), dtype=torch.float32, device=dev)
+    ws = _workspace(workspace, dev).get(msa_workspace_size(p, MSA_OP_INDEX_TOPK))
+    _check(load_library().msa_index_topk(ctypes.byref(p), _ptr(q_idx), _ptr(k_idx),
+                                         _ptr(block_ids), _ptr(block_scores), ws.data_ptr(),
+                                         ws.numel(), _stream(stream)), "msa_index_topk")
+    return (block_ids, block_scores) if return_scores else block_ids
 

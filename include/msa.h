@@ -99,7 +99,8 @@ typedef enum msa_op {
   MSA_OP_BLOCK_SCORES = 4,
   MSA_OP_INDEX_CANDIDATES = 5,
   MSA_OP_SELECT_CANDIDATES = 6,
-  MSA_OP_SHARD_LENGTHS = 7
+  MSA_OP_SHARD_LENGTHS = 7,
+  MSA_OP_INDEX_TOPK = 8
 } msa_op_t;
 
 typedef struct msa_params {
@@ -192,6 +193,21 @@ MSA_API msa_status_t msa_block_scores(const msa_params_t* params, const msa_bf16
                                       const msa_bf16_t* k_idx, float* block_scores,
                                       void* workspace, size_t workspace_bytes,
                                       msa_stream_t stream);
+
+/* Stage 1 in one kernel for prefill: msa_index_select's ids (same order, same
+ * ties, same padding) with the top-k kept in the index GEMM's epilogue, so that
+ * the block scores need not be written at all (block_scores, nullable, still
+ * receives them when given).  Each (query, group) row keeps its best blocks in a
+ * heap in shared memory while the key tiles stream past.  Supported: n_q > 1,
+ * d_idx 64 or 128, block 64 or 128, topk <= 64, else MSA_ERR_UNSUPPORTED.  The
+ * workspace holds the status word only (msa_workspace_size(params,
+ * MSA_OP_INDEX_TOPK)).  Sources: "MiniMax goes sparse" section 1 step 1; the
+ * streaming top-k is the idea of "混合块注意力机制(MoBA)原理与实现详解" section
+ * 3.1, kernel 2 (top-k lists in on-chip memory instead of the score matrix in HBM). */
+MSA_API msa_status_t msa_index_topk(const msa_params_t* params, const msa_bf16_t* q_idx,
+                                    const msa_bf16_t* k_idx, int32_t* block_ids,
+                                    float* block_scores, void* workspace, size_t workspace_bytes,
+                                    msa_stream_t stream);
 
 /* Sequence-sharded decode.  The KV cache of every sequence is split into
  * contiguous token shards of a whole number of blocks, one per GPU; shard r holds
