@@ -385,11 +385,22 @@ def run_ours(args, prob, world, rank, local):
     stream = torch.cuda.current_stream(dev)
 
     # One step is one fused call (both stages, the kernels chained as programmatic
-    # dependents); the per-stage times are measured in a separate pass.
+    # dependents); the per-stage times are measured in a separate pass.  With
+    # --fused-select (prefill) the step is msa_index_topk (the top-k kept in the
+    # index GEMM's epilogue) followed by msa_sparse_attn.
+    if args.fused_select and prob.is_decode:
+        raise SystemExit("--fused-select is a prefill option")
+
     def step():
-        msa.msa_forward(x["q"], x["k"], x["v"], x["q_idx"], x["k_idx"], topk=prob.topk,
-                        force_own_block=prob.force_own, out=out, block_ids=ids, workspace=ws,
-                        **kw)
+        if args.fused_select:
+            msa.msa_index_topk(x["q_idx"], x["k_idx"], topk=prob.topk,
+                               force_own_block=prob.force_own, block_ids=ids, workspace=ws,
+                               **kw)
+            msa.msa_sparse_attn(x["q"], x["k"], x["v"], ids, out=out, workspace=ws, **kw)
+        else:
+            msa.msa_forward(x["q"], x["k"], x["v"], x["q_idx"], x["k_idx"], topk=prob.topk,
+                            force_own_block=prob.force_own, out=out, block_ids=ids,
+                            workspace=ws, **kw)
 
     for _ in range(args.warmup):
         step()
@@ -513,7 +524,10 @@ def run_ours(args, prob, world, rank, local):
                             h=prob.h, d=prob.d, d_idx=prob.d_idx, block=prob.block,
                             topk=prob.topk, causal=prob.causal, q=x["q"], k=x["k"], v=x["v"],
                             q_idx=x["q_idx"], k_idx=x["k_idx"], out=out)
-    launches_per_step = msa.msa_launch_count(p_sel, msa.MSA_OP_FORWARD)
+    launches_per_step = (msa.msa_launch_count(p_sel, msa.MSA_OP_INDEX_TOPK) +
+                         msa.msa_launch_count(p_sel, msa.MSA_OP_SPARSE_ATTN)
+                         if args.fused_select else
+                         msa.msa_launch_count(p_sel, msa.MSA_OP_FORWARD))
 
     peaks, peak_kind = load_peaks()
     if prob.is_decode:
@@ -568,7 +582,9 @@ def run_ours(args, prob, world, rank, local):
                           "no flush: inputs larger than L2 (%.2f GB touched per step)"
                           % (touched / 1e9) if touched else
                           "no flush: inputs larger than L2"),
-                   "parallelism": "replicas" if world > 1 else "single GPU"},
+                   "parallelism": "replicas" if world > 1 else "single GPU",
+                   "select": "msa_index_topk (streaming top-k)" if args.fused_select
+                   else "index GEMM/scan + top-k kernel"},
         "us_per_step": 1e3 * ms_per_step,
         "step_ms": step_stats,
         "stage_ms": {"index_scan": stage["scan"], "index_select": sel_ms, "sparse_attn": attn_ms},
@@ -718,6 +734,9 @@ def main():
     ap.add_argument("--min-ms", type=float, default=200.0,
                     help="repeat the K-step loop until this much device time is timed")
     ap.add_argument("--max-repeats", type=int, default=400)
+    ap.add_argument("--fused-select", action="store_true",
+                    help="prefill: select with msa_index_topk (top-k in the index GEMM's "
+                         "epilogue) instead of the GEMM + top-k kernels")
     ap.add_argument("--l2-flush", action="store_true",
                     help="write a buffer larger than L2 before every step and time each step "
                          "alone")

@@ -71,7 +71,9 @@ struct KvArgs {
   int* toffs;              // [batch * h * nblk + 1] tile offsets
   int2* entries;           // {chunk-relative slot position, query index t} of each
                            // entry, grouped by (b, g, block)
-  int* slot_row;           // [slot] partial row of a valid slot's query (head 0) in its tile
+  int* slot_row;           // [slot] partial row of a valid slot's query (head 0) in its
+                           // tile; -1 for an empty or invalid slot, whose log-sum-exps
+                           // are then -inf (both written by the scatter kernel)
   int qpt;                 // queries per tile
   int nj;                  // batch * h * nblk
   // partial outputs: 128 rows per tile, row = tile * 128 + query-in-tile * G +
@@ -196,6 +198,10 @@ __global__ void kv_scatter_kernel(KvArgs a, int BLK) {
       const int k = atomicAdd(&a.counts[j], 1);
       a.entries[a.offs[j] + k] = make_int2((int)pos, t);
       a.slot_row[pos] = (a.toffs[j] + k / a.qpt) * kRows + (k % a.qpt) * a.G;
+    } else {
+      // no partial for this slot: the merge reads the marks, not the ids
+      a.slot_row[pos] = -1;
+      for (int hh = 0; hh < a.G; ++hh) a.part_lse[pos * a.G + hh] = -__int_as_float(0x7f800000);
     }
   }
 }
@@ -769,25 +775,21 @@ __global__ void __launch_bounds__(256, 2) kv_combine_group_kernel(KvArgs a, int 
   const int bt_rel = (int)(wid / a.h);
   const int bt = (int)a.bt0 + bt_rel;
   const int b = bt / a.n_q, t = bt % a.n_q;
-  const int lim = visible_limit(a, b, t);
   constexpr int G = GC;
   const int rl = lane / LPR, c = lane % LPR;
-  const int32_t* row_ids = a.ids + ((int64_t)bt * a.h + g) * a.topk;
   const int64_t p0 = ((int64_t)bt_rel * a.h + g) * a.topk;
   const float ninf = -__int_as_float(0x7f800000);
-  // pass 1: per-head maximum of the valid slots' LSEs, slots spread over the lanes
+  // pass 1: per-head maximum of the slots' log-sum-exps (empty or invalid slots
+  // hold -inf), slots spread over the lanes; a slot's row is kept for pass 2
   float M[GC];
 #pragma unroll
   for (int h = 0; h < GC; ++h) M[h] = ninf;
   for (int s0 = 0; s0 < a.topk; s0 += 32) {
     const int s = s0 + lane;
     if (s < a.topk) {
-      const int beta = __ldg(row_ids + s);
-      if (beta >= 0 && beta < a.nblk && beta * BLK < lim) {
-        const float* l = a.part_lse + (p0 + s) * G;
+      const float* l = a.part_lse + (p0 + s) * G;
 #pragma unroll
-        for (int h = 0; h < GC; ++h) M[h] = fmaxf(M[h], __ldg(l + h));
-      }
+      for (int h = 0; h < GC; ++h) M[h] = fmaxf(M[h], __ldg(l + h));
     }
   }
 #pragma unroll
@@ -811,13 +813,8 @@ __global__ void __launch_bounds__(256, 2) kv_combine_group_kernel(KvArgs a, int 
   // so that whatever row 0 holds cannot leak into the sum
   for (int s0 = 0; s0 < a.topk; s0 += 32) {
     const int s = s0 + lane;
-    int prow = 0;
-    bool ok = false;
-    if (s < a.topk) {
-      const int beta = __ldg(row_ids + s);
-      ok = beta >= 0 && beta < a.nblk && beta * BLK < lim;
-      if (ok) prow = __ldg(a.slot_row + p0 + s);
-    }
+    const int prow = s < a.topk ? __ldg(a.slot_row + p0 + s) : -1;
+    const bool ok = prow >= 0;
     const int cnt = min(32, a.topk - s0);
     for (int j0 = 0; j0 < cnt; j0 += U) {
       uint4 u[U][MI];
@@ -827,7 +824,7 @@ __global__ void __launch_bounds__(256, 2) kv_combine_group_kernel(KvArgs a, int 
       for (int jj = 0; jj < U; ++jj) {
         const int j = min(j0 + jj, cnt - 1);
         use[jj] = j0 + jj < cnt && __shfl_sync(0xffffffffu, ok ? 1 : 0, j) != 0;
-        const int rj = __shfl_sync(0xffffffffu, prow, j);
+        const int rj = max(0, __shfl_sync(0xffffffffu, prow, j));
         const float* lp = a.part_lse + (p0 + s0 + j) * G;
 #pragma unroll
         for (int i = 0; i < MI; ++i) {
@@ -889,21 +886,32 @@ __global__ void __launch_bounds__(256) kv_combine_kernel(KvArgs a, int BLK) {
   const int g = hq / a.G, hi = hq - g * a.G;
   const int bt = (int)a.bt0 + bt_rel;
   const int b = bt / a.n_q, t = bt % a.n_q;
-  const int lim = visible_limit(a, b, t);
-  const int32_t* row_ids = a.ids + ((int64_t)bt * a.h + g) * a.topk;
   const int64_t p0 = ((int64_t)bt_rel * a.h + g) * a.topk;
   const float ninf = -__int_as_float(0x7f800000);
   constexpr int PER = D / 32;  // dims per lane
+  // pass 1: the slots' log-sum-exps and partial rows (empty or invalid slots hold
+  // -inf and row -1, written by the scatter kernel), both loaded at once; the
+  // first 64 slots stay in registers for pass 2
+  constexpr int KR = 2;  // slot groups of 32 kept in registers
+  float lk[KR];
+  int rk[KR];
   float M = ninf;
-  for (int s0 = 0; s0 < a.topk; s0 += 32) {
-    const int s = s0 + lane;
-    float l = ninf;
+#pragma unroll
+  for (int r = 0; r < KR; ++r) {
+    const int s = r * 32 + lane;
+    lk[r] = ninf;
+    rk[r] = -1;
     if (s < a.topk) {
-      const int beta = __ldg(row_ids + s);
-      if (beta >= 0 && beta < a.nblk && beta * BLK < lim) l = __ldg(a.part_lse + (p0 + s) * a.G + hi);
+      lk[r] = __ldg(a.part_lse + (p0 + s) * a.G + hi);
+      rk[r] = __ldg(a.slot_row + p0 + s);
     }
-    M = fmaxf(M, l);
   }
+  for (int s0 = KR * 32; s0 < a.topk; s0 += 32) {
+    const int s = s0 + lane;
+    if (s < a.topk) M = fmaxf(M, __ldg(a.part_lse + (p0 + s) * a.G + hi));
+  }
+#pragma unroll
+  for (int r = 0; r < KR; ++r) M = fmaxf(M, lk[r]);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
   float acc[PER];
@@ -913,15 +921,18 @@ __global__ void __launch_bounds__(256) kv_combine_kernel(KvArgs a, int BLK) {
   if (M != ninf) {
     for (int s0 = 0; s0 < a.topk; s0 += 32) {
       const int s = s0 + lane;
-      float wgt = 0.f;
-      int prow = 0;  // partial row of this lane's slot (row 0 stands in for none)
-      if (s < a.topk) {
-        const int beta = __ldg(row_ids + s);
-        if (beta >= 0 && beta < a.nblk && beta * BLK < lim) {
-          prow = __ldg(a.slot_row + p0 + s) + hi;
-          wgt = __expf(__ldg(a.part_lse + (p0 + s) * a.G + hi) - M);
-        }
+      const int r = s0 / 32;
+      float l = ninf;
+      int prow = -1;
+      if (r < KR) {
+        l = r == 0 ? lk[0] : lk[1];
+        prow = r == 0 ? rk[0] : rk[1];
+      } else if (s < a.topk) {
+        l = __ldg(a.part_lse + (p0 + s) * a.G + hi);
+        prow = __ldg(a.slot_row + p0 + s);
       }
+      const float wgt = (prow >= 0 && l != ninf) ? __expf(l - M) : 0.f;
+      prow = prow >= 0 ? prow + hi : 0;  // row 0 stands in for none
       den += wgt;
       // Loads are issued for every slot of the pass (a slot without a partial reads
       // row 0, which exists); such a slot contributes through a select, never a
