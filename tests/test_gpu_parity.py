@@ -127,6 +127,10 @@ DECODE_EDGE_CASES = [
              block=16, topk=40, seed=122), [5000, 17, 2500]),
     (Problem("decode_few_items", batch=1, n_q=1, max_kv=640, H=8, h=2, d=64, d_idx=128,
              block=64, topk=4, seed=123), [640]),
+    # forced own block, many rows per attention CTA (msa_forward's attention kernel
+    # then selects the blocks of its rows itself), a one-token and an empty sequence
+    (Problem("decode_own_forced", batch=6, n_q=1, max_kv=4000, H=16, h=4, d=64, d_idx=64,
+             block=32, topk=6, force_own=True, seed=124), [4000, 1, 0, 33, 2500, 3999]),
 ]
 
 
