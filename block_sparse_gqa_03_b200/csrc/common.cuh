@@ -127,6 +127,13 @@ inline cudaError_t launch_pdl(void (*kernel)(K...), dim3 grid, dim3 block, size_
   return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
+// Load with acquire semantics at GPU scope (pairs with a writer's fence + atomic).
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
 // Named barrier `id` over `nthreads` threads: arrive without waiting, or wait.
 __device__ __forceinline__ void named_arrive(int id, int nthreads) {
   asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");

@@ -27,7 +27,9 @@
 // one pipeline that never drains.  At each row boundary the consumers merge their
 // states; a row covered by several CTAs gets one fp32 partial per CTA, and the
 // last CTA to finish the row (a per-row counter, zeroed before the launch)
-// merges them by log-sum-exp weights.
+// merges them by log-sum-exp weights.  The row's first CTA, which reaches the
+// row at the end of its range, usually finds the others' partials already
+// published and merges them into its own state without writing its own.
 #include "kernels.h"
 
 namespace msa {
@@ -546,29 +548,81 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1)
   // Ends the segment of row `cur` held by this CTA: merge the warps, then write
   // the output (row entirely in this CTA) or a partial (and merge the row's
   // partials if this CTA is the last of the row to finish).
+  //
+  // A row's first CTA reaches it at the end of its range, while the row's other
+  // CTAs start their ranges with it, so their partials are usually published
+  // long before.  The first CTA reads the row's counter as it arrives: if every
+  // other segment is in, it merges them straight into its own state (its own
+  // partial is never written, and no atomic is taken; no other CTA can then be
+  // the last, since the count never reaches nseg).  Otherwise it publishes like
+  // the others.
   auto flush = [&]() {
-    ws.stash(mo, mm, ml, warp, lane, a.G);
-    consumer_sync(NC * 32);
     const int64_t c_first = (cur * a.topk) / a.per;
     const int64_t c_last = ((cur + 1) * a.topk - 1) / a.per;
     const int nseg = (int)(c_last - c_first + 1);
     const int seg = (int)(c - c_first);
+    const bool first = nseg > 1 && seg == 0;
+    if (first && tid == 0) {
+      *flag = ld_acquire_gpu(a.counters + cur);
+      __threadfence();
+    }
+    ws.stash(mo, mm, ml, warp, lane, a.G);
+    consumer_sync(NC * 32);
+    const bool fast = first && *flag == nseg - 1;
     for (int x = tid; x < a.G * (D / 4); x += NC * 32) {
       const int row = x / (D / 4), dim = (x % (D / 4)) * 4;
+      const int hq = rg.g * a.G + row;
+      const int64_t pr0 = ((int64_t)rg.bt * a.H + hq) * a.smax;
+      // the second segment's partial, loaded before the warps' merge
+      float l1 = neg_inf();
+      float4 o1 = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (fast) {
+        l1 = __ldcg(a.part_lse + pr0 + 1);
+        o1 = __ldcg(reinterpret_cast<const float4*>(a.part_o + (pr0 + 1) * D + dim));
+      }
       float4 val;
       float lsev;
       merge_warps4<D, NC>(mo, mm, ml, a.G, row, dim, val, lsev);
-      const int hq = rg.g * a.G + row;
-      if (nseg == 1) {
+      if (fast) {
+        // the same operations in the same order as the last CTA's merge below,
+        // so that the result does not depend on which of the two ran
+        const float ninf = neg_inf();
+        float M = fmaxf(fmaxf(ninf, lsev), l1);
+        for (int sp = 2; sp < nseg; ++sp) M = fmaxf(M, __ldcg(a.part_lse + pr0 + sp));
+        float4 res = make_float4(0.f, 0.f, 0.f, 0.f);
+        float lres = ninf;
+        if (M != ninf) {
+          float den = 0.f;
+          float4 acc = res;
+          auto add = [&](float l, const float4& o) {
+            const float w = exp2f((l - M) * kLog2e);
+            den += w;
+            acc.x += w * o.x;
+            acc.y += w * o.y;
+            acc.z += w * o.z;
+            acc.w += w * o.w;
+          };
+          add(lsev, val);
+          add(l1, o1);
+          for (int sp = 2; sp < nseg; ++sp)
+            add(__ldcg(a.part_lse + pr0 + sp),
+                __ldcg(reinterpret_cast<const float4*>(a.part_o + (pr0 + sp) * D + dim)));
+          res = make_float4(acc.x / den, acc.y / den, acc.z / den, acc.w / den);
+          lres = M + log2f(den) * kLn2;
+        }
+        val = res;
+        lsev = lres;
+      }
+      if (nseg == 1 || fast) {
         store_out4(a, rg, hq, dim, val);
         if (dim == 0 && a.lse) a.lse[(int64_t)rg.bt * a.H + hq] = lsev;
       } else {
-        const int64_t pr = ((int64_t)rg.bt * a.H + hq) * a.smax + seg;
+        const int64_t pr = pr0 + seg;
         *reinterpret_cast<float4*>(a.part_o + pr * D + dim) = val;
         if (dim == 0) a.part_lse[pr] = lsev;
       }
     }
-    if (nseg > 1) {
+    if (nseg > 1 && !fast) {
       // One thread publishes the CTA's partial (its stores ordered before the
       // fence by the barrier) and learns whether it is the row's last; its
       // second fence orders the other CTAs' partials before the loads below.
