@@ -233,6 +233,146 @@ struct WarpState {
   }
 };
 
+// The same state for groups of at most 8 heads with the MMA operands swapped:
+// S^T = K Q^T puts a slice's 16 tokens on the MMA rows and the G heads on the
+// n8 columns, and O^T = V^T P^T puts 16 output dims on the rows, so no MMA row
+// is spent on padding (half as many MMAs and exponentials as the layout above
+// at G = 8).  The K and V tiles feed the A operands through the same ldmatrix
+// loads (K as stored, V transposed); P^T reaches the B layout of the second MMA
+// through an in-register 8x8 transpose.  Each thread keeps heads 2 (lane % 4)
+// and 2 (lane % 4) + 1: running max (shared by the 8 lanes of those heads) and
+// its own part of the running sum.
+template <int D>
+struct WarpStateT {
+  uint32_t qb[D / 16][2];  // B fragments of Q^T: dims 16kk + 2 (lane % 4) (+8), head lane / 4
+  float o[D / 16][4];      // O^T tile mt: dims 16mt + lane / 4 (+8), heads 2 (lane % 4) (+1)
+  float m0, m1, l0, l1;
+
+  __device__ __forceinline__ void reset() {
+#pragma unroll
+    for (int i = 0; i < D / 16; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+    m0 = m1 = neg_inf();
+    l0 = l1 = 0.f;
+  }
+
+  __device__ __forceinline__ void load_q(const AttnArgs& a, const RowGeo& rg, int lane) {
+    const int r = lane >> 2, q4 = lane & 3;
+    const bool valid = r < a.G;
+    const uint16_t* qh = a.q + rg.b * a.q_s0 + (int64_t)rg.t * a.q_s1 +
+                         (int64_t)(rg.g * a.G + r) * a.q_s2 + 2 * q4;
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      qb[kk][0] = valid ? ld_b32(qh + 16 * kk) : 0u;
+      qb[kk][1] = valid ? ld_b32(qh + 16 * kk + 8) : 0u;
+    }
+  }
+
+  __device__ __forceinline__ void attend(const AttnArgs& a, uint8_t* smem, uint32_t sbase,
+                                         uint32_t kbase, uint32_t vbase, uint32_t half_bytes,
+                                         int tok, int j0, int lim, int lane, bool& wrote_smem) {
+    constexpr int NH = D / 64;
+    const int r = lane >> 2;
+    const float ninf = neg_inf();
+    if (j0 + 16 > lim) {
+      // Tokens j >= lim of this slice may be uninitialised memory: zero their V rows
+      // so that a zero probability never meets a non-finite value.
+      const int r0 = lim - j0;
+      const int per_h = (16 - r0) * 8;
+      uint8_t* vrow = smem + (vbase - sbase);
+      for (int x = lane; x < per_h * NH; x += 32) {
+        const int hh = x / per_h, rem = x % per_h;
+        const int row = tok + r0 + rem / 8;
+        *reinterpret_cast<uint4*>(vrow + hh * half_bytes + row * 128 + (rem % 8) * 16) =
+            make_uint4(0, 0, 0, 0);
+      }
+      wrote_smem = true;
+      __syncwarp();
+    }
+    // S^T: tokens tok + r (s[0], s[1]) and tok + r + 8 (s[2], s[3]), heads 2q4, 2q4 + 1
+    float s[4] = {0.f, 0.f, 0.f, 0.f};
+    {
+      const int mi = lane >> 3, rr = lane & 7;
+      const uint32_t row = tok + (mi >> 1) * 8 + rr;
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t chunk = (kk & 3) * 2 + (mi & 1);
+        uint32_t k0, k1, k2, k3;  // tokens 0-7 / 8-15 x dims low / high of the k-step
+        ldmatrix_x4(kbase + (kk >> 2) * half_bytes + swz128(row, chunk), k0, k1, k2, k3);
+        mma_bf16_16816(s, k0, k2, k1, k3, qb[kk][0], qb[kk][1]);
+      }
+    }
+    const bool ok_lo = j0 + r < lim, ok_hi = j0 + r + 8 < lim;
+    s[0] = ok_lo ? s[0] * a.scale_log2 : ninf;
+    s[1] = ok_lo ? s[1] * a.scale_log2 : ninf;
+    s[2] = ok_hi ? s[2] * a.scale_log2 : ninf;
+    s[3] = ok_hi ? s[3] * a.scale_log2 : ninf;
+    float mx0 = fmaxf(s[0], s[2]), mx1 = fmaxf(s[1], s[3]);
+    mx0 = warp_max_xor(warp_max_xor(warp_max_xor(mx0, 4), 8), 16);
+    mx1 = warp_max_xor(warp_max_xor(warp_max_xor(mx1, 4), 8), 16);
+    const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+    const float c0 = exp2f(m0 - mn0), c1 = exp2f(m1 - mn1);
+    m0 = mn0;
+    m1 = mn1;
+    s[0] = exp2f(s[0] - mn0);
+    s[1] = exp2f(s[1] - mn1);
+    s[2] = exp2f(s[2] - mn0);
+    s[3] = exp2f(s[3] - mn1);
+    l0 = l0 * c0 + (s[0] + s[2]);
+    l1 = l1 * c1 + (s[1] + s[3]);
+#pragma unroll
+    for (int mt = 0; mt < D / 16; ++mt) {
+      o[mt][0] *= c0;
+      o[mt][1] *= c1;
+      o[mt][2] *= c0;
+      o[mt][3] *= c1;
+    }
+    // P^T as the B operand: tokens 2q4 (+1) (+8), head r
+    const uint32_t pb0 = movmatrix_trans(pack_bf16(s[0], s[1]));
+    const uint32_t pb1 = movmatrix_trans(pack_bf16(s[2], s[3]));
+    const int mi = lane >> 3, rr = lane & 7;
+    const uint32_t row = tok + (mi & 1) * 8 + rr;
+#pragma unroll
+    for (int mt = 0; mt < D / 16; ++mt) {
+      const uint32_t chunk = (mt & 3) * 2 + (mi >> 1);
+      uint32_t v0, v1, v2, v3;  // dims low / high x tokens 0-7 / 8-15, transposed
+      ldmatrix_x4_trans(vbase + (mt >> 2) * half_bytes + swz128(row, chunk), v0, v1, v2, v3);
+      mma_bf16_16816(o[mt], v0, v2, v1, v3, pb0, pb1);
+    }
+  }
+
+  // Same merge-buffer layout as WarpState::stash: O rows [warp][gr][D], running
+  // max and sum [warp][16].
+  __device__ __forceinline__ void stash(float* mo, float* mm, float* ml, int warp, int lane,
+                                        int gr) {
+    const int r = lane >> 2, h0 = 2 * (lane & 3), h1 = h0 + 1;
+    float s0 = l0, s1 = l1;
+#pragma unroll
+    for (int x = 4; x < 32; x <<= 1) {
+      s0 += __shfl_xor_sync(0xffffffffu, s0, x);
+      s1 += __shfl_xor_sync(0xffffffffu, s1, x);
+    }
+    float* mw = mo + warp * gr * D;
+#pragma unroll
+    for (int mt = 0; mt < D / 16; ++mt) {
+      const int dd = mt * 16 + r;
+      if (h0 < gr) {
+        mw[h0 * D + dd] = o[mt][0];
+        mw[h0 * D + dd + 8] = o[mt][2];
+      }
+      if (h1 < gr) {
+        mw[h1 * D + dd] = o[mt][1];
+        mw[h1 * D + dd + 8] = o[mt][3];
+      }
+    }
+    if (r == 0) {
+      mm[warp * 16 + h0] = m0;
+      mm[warp * 16 + h1] = m1;
+      ml[warp * 16 + h0] = s0;
+      ml[warp * 16 + h1] = s1;
+    }
+  }
+};
+
 // Merge of NC warp states for tile row `row`, dims [dim, dim + 4) (dim a
 // multiple of 4): normalised output and natural-log LSE (-inf and 0 when no key
 // was seen).  The warps' weights are computed once for the four dims.
@@ -484,7 +624,7 @@ __global__ void __launch_bounds__(5 * 32, 1)
 }
 
 // ----------------------------------------- persistent, balanced streaming
-template <int D, int NC>
+template <int D, int NC, class WS>
 __global__ void __launch_bounds__((NC + 1) * 32, 1)
     sparse_attn_stream_kernel(const __grid_constant__ CUtensorMap tmk,
                               const __grid_constant__ CUtensorMap tmv, AttnArgs a) {
@@ -535,7 +675,7 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1)
     return;
   }
   // the consumers load their first row's queries while the list is built
-  WarpState<D> ws;
+  WS ws;
   int64_t cur = r0;
   RowGeo rg = row_geo(a, cur);
   ws.reset();
@@ -970,20 +1110,18 @@ cudaError_t launch_sparse_attn(const Shape& s, const uint16_t* q, const uint16_t
   }
   const dim3 grid((unsigned)pl.ctas);
   constexpr int NT = (kStreamNC + 1) * 32;
-  if (s.d == 128) {
-    err = cudaFuncSetAttribute(sparse_attn_stream_kernel<128, kStreamNC>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem_bytes);
-    if (err != cudaSuccess) return err;
-    err = launch_pdl(sparse_attn_stream_kernel<128, kStreamNC>, grid, dim3(NT), pl.smem_bytes,
-                     stream, tmk, tmv, a);
-  } else {
-    err = cudaFuncSetAttribute(sparse_attn_stream_kernel<64, kStreamNC>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem_bytes);
-    if (err != cudaSuccess) return err;
-    err = launch_pdl(sparse_attn_stream_kernel<64, kStreamNC>, grid, dim3(NT), pl.smem_bytes,
-                     stream, tmk, tmv, a);
-  }
-  return err;
+  auto run = [&](auto kernel) {
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)pl.smem_bytes);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(kernel, grid, dim3(NT), pl.smem_bytes, stream, tmk, tmv, a);
+  };
+  // groups of up to 8 heads take the swapped MMA operands
+  if (s.d == 128)
+    return s.G <= 8 ? run(sparse_attn_stream_kernel<128, kStreamNC, WarpStateT<128>>)
+                    : run(sparse_attn_stream_kernel<128, kStreamNC, WarpState<128>>);
+  return s.G <= 8 ? run(sparse_attn_stream_kernel<64, kStreamNC, WarpStateT<64>>)
+                  : run(sparse_attn_stream_kernel<64, kStreamNC, WarpState<64>>);
 }
 
 }  // namespace msa
