@@ -44,7 +44,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # proportion).  An entry is removed when its kernel changes; absent entries
 # report null.
 TRAFFIC = {
-    ("decode_128k", "attn"): 4 * (134.456832e6 + 3.434752e6),
+    ("decode_128k", "attn"): 4 * (134.483968e6 + 3.917824e6),
     ("decode_128k", "scan"): 4 * (134.275584e6 + 4.156672e6),
 }
 L2_FLUSH_BYTES = 256 * 2**20
