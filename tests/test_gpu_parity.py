@@ -109,6 +109,12 @@ SMALL_CASES = [
             block=128, topk=3, causal=True, force_own=True, seed=115),
     Problem("decode_many_splits", batch=2, n_q=1, max_kv=65536, H=64, h=8, d=128, d_idx=128,
             block=64, topk=600, causal=True, seed=109, len_range=(40000, 65536)),
+    # groups of 7 and 5 heads in the decode attention (swapped MMA operands: heads
+    # past G are zero columns of the n8 tile)
+    Problem("decode_g7_d64", batch=3, n_q=1, max_kv=6000, H=14, h=2, d=64, d_idx=64, block=64,
+            topk=12, causal=True, seed=125, len_range=(1, 6000)),
+    Problem("decode_g5_b128", batch=2, n_q=1, max_kv=9000, H=20, h=4, d=128, d_idx=128,
+            block=128, topk=10, causal=True, force_own=True, seed=126),
 ]
 
 
@@ -127,8 +133,8 @@ DECODE_EDGE_CASES = [
              block=16, topk=40, seed=122), [5000, 17, 2500]),
     (Problem("decode_few_items", batch=1, n_q=1, max_kv=640, H=8, h=2, d=64, d_idx=128,
              block=64, topk=4, seed=123), [640]),
-    # forced own block, many rows per attention CTA (msa_forward's attention kernel
-    # then selects the blocks of its rows itself), a one-token and an empty sequence
+    # forced own block, many rows per attention CTA, a one-token and an empty
+    # sequence
     (Problem("decode_own_forced", batch=6, n_q=1, max_kv=4000, H=16, h=4, d=64, d_idx=64,
              block=32, topk=6, force_own=True, seed=124), [4000, 1, 0, 33, 2500, 3999]),
 ]
