@@ -611,7 +611,8 @@ def run_ours(args, prob, world, rank, local):
 def run_e2e(args, prob, x, dev, world, msa, kw):
     """Same metric through the public API with host buffers: pinned host -> device
     copies of the step's inputs, the calls, and the output read back, inside the
-    timed region."""
+    timed region (decode: the step replayed as a captured CUDA graph unless
+    --e2e-eager)."""
     stream = torch.cuda.current_stream(dev)
     out_dev = torch.empty_like(x["q"])
     out_host = torch.empty(out_dev.shape, dtype=out_dev.dtype, pin_memory=True)
@@ -623,6 +624,9 @@ def run_e2e(args, prob, x, dev, world, msa, kw):
         # packed in one pinned buffer, copied once, the rows written into the
         # resident cache at position L_b - 1 by msa_append_kv, then msa_forward.
         # (The rows are the cache's own, so the cache is unchanged step to step.)
+        # Copying the attention queries on a second stream beside msa_index_select,
+        # then msa_sparse_attn, measured slower (218 against 210 us at 128K): the
+        # extra dependency and the merge-counter memset cost more than the copy.
         L = (x["seq_lens"].cpu().tolist() if x["seq_lens"] is not None
              else [prob.max_kv] * prob.batch)
         parts = {"q": x["q"], "q_idx": x["q_idx"]}
@@ -704,12 +708,24 @@ def run_e2e(args, prob, x, dev, world, msa, kw):
 
     one()
     torch.cuda.synchronize(dev)
+    step, graphed = one, False
+    if prob.is_decode and not args.e2e_eager:
+        # A decode step as a serving loop runs it: captured once as a CUDA graph (the
+        # pinned-memory copies, msa_append_kv and msa_forward's kernels with their
+        # programmatic dependencies) and replayed every step; the copies stay inside.
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            one()
+        step, graphed = graph.replay, True
+        nsteps = max(1, min(args.steps, 400))
+        step()
+        torch.cuda.synchronize(dev)
     barrier(world)
     s0 = torch.cuda.Event(enable_timing=True)
     s1 = torch.cuda.Event(enable_timing=True)
     s0.record(stream)
     for _ in range(nsteps):
-        one()
+        step()
     s1.record(stream)
     torch.cuda.synchronize(dev)
     barrier(world)
@@ -720,7 +736,8 @@ def run_e2e(args, prob, x, dev, world, msa, kw):
     u = work_units(prob, x, ids)
     unit, scale = unit_of(prob)
     return {"value": (u["select"] + u["attn"]) * world / (ms * 1e-3) / scale, "unit": unit,
-            "ms_per_step": ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+            "ms_per_step": ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "steps": nsteps, "cuda_graph": graphed}
 
 
 def main():
@@ -742,6 +759,9 @@ def main():
                          "alone")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-eager", action="store_true",
+                    help="decode e2e: issue the step's calls one by one instead of replaying "
+                         "them as a captured CUDA graph")
     ap.add_argument("--batch", type=int, default=0,
                     help="override the workload's batch (for small profiling captures)")
     ap.add_argument("--seq", type=int, default=0,
