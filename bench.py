@@ -714,7 +714,9 @@ def run_e2e(args, prob, x, dev, world, msa, kw):
         # pinned-memory copies, msa_append_kv and msa_forward's kernels with their
         # programmatic dependencies) and replayed every step; the copies stay inside.
         graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph):
+        # thread-local capture: other threads (a process group's watchdog, the clock
+        # sampler) may use CUDA meanwhile
+        with torch.cuda.graph(graph, capture_error_mode="thread_local"):
             one()
         step, graphed = graph.replay, True
         nsteps = max(1, min(args.steps, 400))
