@@ -7,8 +7,9 @@
 // ("MiniMax M3 的 MSA ...", second layer).
 //
 // A "row" is one (sequence, query, group); its G query heads are the 16 rows of
-// a bf16 m16n8k16 tensor-core tile (rows >= G are zero).  Both kernels below
-// share the same engine:
+// a bf16 m16n8k16 tensor-core tile (rows >= G are zero), or, in the streaming
+// kernel for G <= 8, the 8 columns of the tile with the operands swapped
+// (WarpStateT).  Both kernels below share the same engine:
 //  * one producer warp streams each selected block's K and V tiles into a ring of
 //    shared-memory stages with TMA (4-D tensor maps over [batch, token, kv head,
 //    dim], 128-byte swizzle), completion tracked by mbarriers whose waits are
