@@ -21,7 +21,14 @@ struct DeviceStatus {
   uint32_t detail;  // kernel-specific detail of that error
 };
 
-constexpr size_t kStatusBytes = 256;  // reserved at the start of the workspace
+// Reserved at the start of the workspace: the status word, and from byte
+// kCounterOffset the decode attention's per-row merge counters.  The counters are
+// zero between calls: msa_workspace_init clears the region, every row's merging
+// CTA puts its counter back to zero, and msa_get_device_status clears the region
+// again after an error (a call that stopped early may leave counters set).
+constexpr size_t kStatusBytes = 4096;
+constexpr size_t kCounterOffset = 256;
+constexpr int kFixedCounters = (int)((kStatusBytes - kCounterOffset) / sizeof(int));
 
 __device__ __forceinline__ void record_error(DeviceStatus* st, uint32_t code, uint32_t detail) {
   if (st == nullptr) return;

@@ -81,12 +81,16 @@ int attn_launches(const Shape& s);
 // The streaming (decode) kernel's per-row merge counters inside `partials`, or
 // nullptr when the shape takes another kernel; *count receives their number.
 int* attn_merge_counters(const Shape& s, void* partials, int* count);
-// counters_zeroed: the merge counters were cleared on the stream already (by the
-// top-k kernel of the same forward), so no memset is issued.
+// Merge counters: `fixed_counters` (kFixedCounters words that are zero between
+// calls, nullable) when the shape needs no more of them; otherwise the ones in
+// `partials`, cleared by a memset unless `counters_zeroed` (the top-k kernel of
+// the same forward cleared them already).  The kernel puts every counter it uses
+// back to zero.
 cudaError_t launch_sparse_attn(const Shape& s, const uint16_t* q, const uint16_t* k,
                                const uint16_t* v, const int32_t* ids, uint16_t* out, float* lse,
                                void* partials, size_t partial_bytes, DeviceStatus* st,
-                               cudaStream_t stream, bool counters_zeroed = false);
+                               cudaStream_t stream, bool counters_zeroed = false,
+                               int* fixed_counters = nullptr);
 
 // Stage 2 for prefill, KV-major on tcgen05 (d 64/128, block 64/128, n_q > 1):
 // inverted index, tiles of gathered (query, head) rows per selected block,

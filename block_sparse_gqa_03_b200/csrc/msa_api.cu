@@ -175,7 +175,8 @@ size_t ids_bytes(const Shape& s) {
   return (size_t)s.batch * s.n_q * s.h * s.topk * sizeof(int32_t);
 }
 
-// Workspace layout: [status | scores | ids | attention partials], 256-aligned parts.
+// Workspace layout: [status region (status word, decode merge counters) | scores |
+// ids | attention partials], 256-aligned parts.
 struct Layout {
   size_t scores_off, ids_off, part_off, part_bytes, total;
 };
@@ -219,6 +220,9 @@ msa_status_t check_ws(const Shape& s, msa_op_t op, void* ws, size_t bytes) {
 msa_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MSA_OK : MSA_ERR_CUDA; }
 
 uint8_t* at(void* ws, size_t off) { return reinterpret_cast<uint8_t*>(ws) + off; }
+
+// The decode attention's merge counters in the workspace's status region.
+int* fixed_counters(void* ws) { return reinterpret_cast<int*>(at(ws, msa::kCounterOffset)); }
 
 cudaError_t run_scores(const Shape& s, const msa_bf16_t* q_idx, const msa_bf16_t* k_idx,
                        float* scores, bool fill_tail, msa::DeviceStatus* st,
@@ -375,7 +379,8 @@ msa_status_t msa_sparse_attn(const msa_params_t* params, const msa_bf16_t* q, co
   const Layout l = layout(s, MSA_OP_SPARSE_ATTN);
   return cuda_status(msa::launch_sparse_attn(
       s, q, k, v, block_ids, out, lse, at(workspace, l.part_off), l.part_bytes,
-      reinterpret_cast<msa::DeviceStatus*>(workspace), reinterpret_cast<cudaStream_t>(stream)));
+      reinterpret_cast<msa::DeviceStatus*>(workspace), reinterpret_cast<cudaStream_t>(stream),
+      false, fixed_counters(workspace)));
 }
 
 msa_status_t msa_forward(const msa_params_t* params, const msa_bf16_t* q, const msa_bf16_t* k,
@@ -391,17 +396,20 @@ msa_status_t msa_forward(const msa_params_t* params, const msa_bf16_t* q, const 
   const Layout l = layout(s, MSA_OP_FORWARD);
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   int32_t* ids = block_ids ? block_ids : reinterpret_cast<int32_t*>(at(workspace, l.ids_off));
-  // the top-k kernel clears the attention's merge counters, so that the two
-  // stages follow each other with no memset in between
+  // The attention's merge counters are the status region's (zero between calls)
+  // when the shape needs no more of them; otherwise the top-k kernel clears the
+  // ones in the partials, so that the two stages follow each other with no memset
+  // in between.
   int ncounters = 0;
   int* counters = msa::attn_merge_counters(s, at(workspace, l.part_off), &ncounters);
+  if (counters != nullptr && ncounters <= msa::kFixedCounters) counters = nullptr;
   if ((rc = run_select(s, q_idx, k_idx, ids, block_scores, workspace, l, cs, counters,
                        ncounters)) != MSA_OK)
     return rc;
   return cuda_status(msa::launch_sparse_attn(s, q, k, v, ids, out, lse, at(workspace, l.part_off),
                                              l.part_bytes,
                                              reinterpret_cast<msa::DeviceStatus*>(workspace), cs,
-                                             counters != nullptr));
+                                             counters != nullptr, fixed_counters(workspace)));
 }
 
 msa_status_t msa_append_kv(const msa_params_t* params, const msa_bf16_t* k_new,
@@ -433,7 +441,9 @@ msa_status_t msa_get_device_status(void* workspace, msa_stream_t stream) {
     return MSA_ERR_CUDA;
   if (cudaStreamSynchronize(cs) != cudaSuccess) return MSA_ERR_CUDA;
   if (h.code != 0) {
-    if (cudaMemsetAsync(workspace, 0, sizeof h, cs) != cudaSuccess) return MSA_ERR_CUDA;
+    // the whole status region: a call that stopped early may have left merge
+    // counters set
+    if (cudaMemsetAsync(workspace, 0, msa::kStatusBytes, cs) != cudaSuccess) return MSA_ERR_CUDA;
     if (cudaStreamSynchronize(cs) != cudaSuccess) return MSA_ERR_CUDA;
   }
   return static_cast<msa_status_t>(h.code);

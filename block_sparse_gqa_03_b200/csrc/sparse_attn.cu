@@ -27,8 +27,8 @@
 // equal contiguous ranges, so every SM streams the same number of blocks through
 // one pipeline that never drains.  At each row boundary the consumers merge their
 // states; a row covered by several CTAs gets one fp32 partial per CTA, and the
-// last CTA to finish the row (a per-row counter, zeroed before the launch)
-// merges them by log-sum-exp weights.  The row's first CTA, which reaches the
+// last CTA to finish the row (a per-row counter, zero before the launch and put
+// back to zero by the merging CTA) merges them by log-sum-exp weights.  The row's first CTA, which reaches the
 // row at the end of its range, usually finds the others' partials already
 // published and merges them into its own state without writing its own.
 #include "kernels.h"
@@ -845,6 +845,8 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1)
         }
       }
     }
+    // the row's merge is done: its counter goes back to zero for the next call
+    if (nseg > 1 && tid == 0 && *flag == nseg - 1) a.counters[cur] = 0;
     consumer_sync(NC * 32);  // the merge buffer is free again
   };
 
@@ -1034,7 +1036,7 @@ int* attn_merge_counters(const Shape& s, void* partials, int* count) {
 cudaError_t launch_sparse_attn(const Shape& s, const uint16_t* q, const uint16_t* k,
                                const uint16_t* v, const int32_t* ids, uint16_t* out, float* lse,
                                void* partials, size_t partial_bytes, DeviceStatus* st,
-                               cudaStream_t stream, bool counters_zeroed) {
+                               cudaStream_t stream, bool counters_zeroed, int* fixed_counters) {
   const AttnPlan pl = plan_attn(s);
   if (pl.smem_bytes > kSmemCap) return cudaErrorInvalidValue;
   CUtensorMap tmk, tmv;
@@ -1105,7 +1107,9 @@ cudaError_t launch_sparse_attn(const Shape& s, const uint16_t* q, const uint16_t
   a.part_lse = a.part_o + nrow_h * pl.smax * s.d;
   int ncounters = 0;
   a.counters = attn_merge_counters(s, partials, &ncounters);
-  if (!counters_zeroed) {
+  if (fixed_counters != nullptr && ncounters <= kFixedCounters) {
+    a.counters = fixed_counters;  // zero already, and left at zero
+  } else if (!counters_zeroed) {
     err = cudaMemsetAsync(a.counters, 0, (size_t)ncounters * sizeof(int), stream);
     if (err != cudaSuccess) return err;
   }

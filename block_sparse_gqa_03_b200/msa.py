@@ -20,6 +20,7 @@ import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmsa.so")
+STATUS_BYTES = 4096  # the workspace's status region (status word, decode merge counters)
 
 MSA_OK = 0
 MSA_ERR_INVALID_ARG = 1
@@ -184,7 +185,7 @@ class Workspace:
 
     def get(self, nbytes: int) -> torch.Tensor:
         if self.buf is None or self.buf.numel() < nbytes:
-            self.buf = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=self.device)
+            self.buf = torch.empty(max(nbytes, STATUS_BYTES), dtype=torch.uint8, device=self.device)
             rc = load_library().msa_workspace_init(self.buf.data_ptr(), self.buf.numel(), _stream())
             if rc != MSA_OK:
                 raise MsaError(rc, "msa_workspace_init")

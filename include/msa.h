@@ -122,9 +122,11 @@ typedef struct msa_params {
 } msa_params_t;
 
 /* Bytes of workspace `op` needs for these shapes (0 on invalid params).  The
- * workspace must be 256-byte aligned.  It holds the sticky device status word,
- * and, when the caller does not supply them, block scores and block ids, plus
- * the split-KV partial results of the attention. */
+ * workspace must be 256-byte aligned.  It starts with a 4096-byte status region
+ * (the sticky device status word and the decode attention's per-row merge
+ * counters, which are zero between calls) and holds, when the caller does not
+ * supply them, block scores and block ids, plus the split-KV partial results of
+ * the attention. */
 MSA_API size_t msa_workspace_size(const msa_params_t* params, msa_op_t op);
 
 /* Stage 1 (index branch).  For every (b, t, g):
@@ -173,7 +175,7 @@ MSA_API msa_status_t msa_forward(const msa_params_t* params, const msa_bf16_t* q
  * paged caches included (row pos % block of page block_table[b, pos / block]).
  * A position < 0 or a page id outside the pool is recorded as
  * MSA_ERR_DEVICE_ASSERT and that token is not written.  The workspace holds the
- * status word only (msa_workspace_size(params, MSA_OP_APPEND_KV) bytes).
+ * status region only (msa_workspace_size(params, MSA_OP_APPEND_KV) bytes).
  * The cache keeps the plain GQA layout ("MiniMax M3 的 MSA ...", section
  * "三条有意为之的减法", first item), one block per physical block ("深度解析M3多模态
  * 模型与Token Plan", list of MSA's innovations, first item). */
@@ -185,7 +187,7 @@ MSA_API msa_status_t msa_append_kv(const msa_params_t* params, const msa_bf16_t*
 /* Stage 1, first half: the block scores alone (the index scan with its fused
  * causal block max pool, no top-k).  block_scores fp32 [batch, n_q, h, nblk]
  * receives S for every block, -inf past each row's frontier, exactly as
- * msa_index_select's optional output.  The workspace holds the status word only
+ * msa_index_select's optional output.  The workspace holds the status region only
  * (msa_workspace_size(params, MSA_OP_BLOCK_SCORES)).
  * Sources: "MiniMax goes sparse" section 1 step 1 (Q_idx . K_idx^T and the Block
  * Max Pool); "MiniMax M3 的 MSA ..." first layer. */
@@ -200,7 +202,7 @@ MSA_API msa_status_t msa_block_scores(const msa_params_t* params, const msa_bf16
  * receives them when given).  Each (query, group) row keeps its best blocks in a
  * heap in shared memory while the key tiles stream past.  Supported: n_q > 1,
  * d_idx 64 or 128, block 64 or 128, topk <= 64, else MSA_ERR_UNSUPPORTED.  The
- * workspace holds the status word only (msa_workspace_size(params,
+ * workspace holds the status region only (msa_workspace_size(params,
  * MSA_OP_INDEX_TOPK)).  Sources: "MiniMax goes sparse" section 1 step 1; the
  * streaming top-k is the idea of "混合块注意力机制(MoBA)原理与实现详解" section
  * 3.1, kernel 2 (top-k lists in on-chip memory instead of the score matrix in HBM). */
@@ -228,7 +230,7 @@ MSA_API msa_status_t msa_index_topk(const msa_params_t* params, const msa_bf16_t
  * block_sparse_gqa_03_b200/seqshard.py runs these steps with NCCL all-gathers. */
 
 /* shard_lens[b] = clamp(L_b - token_base, 0, token_count) (device int32 [batch]),
- * L_b from params->seq_lens (NULL: max_kv).  Workspace: the status word
+ * L_b from params->seq_lens (NULL: max_kv).  Workspace: the status region
  * (msa_workspace_size(params, MSA_OP_SHARD_LENGTHS)). */
 MSA_API msa_status_t msa_shard_lengths(const msa_params_t* params, int64_t token_base,
                                        int64_t token_count, int32_t* shard_lens,
@@ -257,7 +259,7 @@ MSA_API msa_status_t msa_index_candidates(const msa_params_t* params, const msa_
  *   local_ids (nullable) int32 [batch, n_q, h, topk]: slot by slot, id -
  *     block_base when block_base <= id < block_base + nblk_local, else -1.
  * params: the whole problem (global seq_lens and max_kv, h, block, topk,
- * force_own_block).  Workspace: the status word
+ * force_own_block).  Workspace: the status region
  * (msa_workspace_size(params, MSA_OP_SELECT_CANDIDATES)). */
 MSA_API msa_status_t msa_select_candidates(const msa_params_t* params, int32_t nlists,
                                            int32_t list_len, int32_t shard_blocks,
@@ -279,12 +281,15 @@ MSA_API msa_status_t msa_merge_partials(const msa_params_t* params, int32_t npar
                                         msa_bf16_t* out, float* lse, msa_stream_t stream);
 
 /* Synchronises `stream`, returns the first error a kernel recorded in this
- * workspace since the last reset (MSA_OK if none) and clears it. */
+ * workspace since the last reset (MSA_OK if none) and, after an error, clears the
+ * workspace's 4096-byte status region (the word, and the merge counters that a
+ * call which stopped early may have left set). */
 MSA_API msa_status_t msa_get_device_status(void* workspace, msa_stream_t stream);
 
-/* Zeroes the workspace's status word, asynchronously on `stream`.  Call it once
- * on every new workspace before its first use (the word is sticky: kernels only
- * ever set it, msa_get_device_status() clears it). */
+/* Zeroes the workspace's 4096-byte status region, asynchronously on `stream`.
+ * Call it once on every new workspace before its first use.  The region holds the
+ * sticky status word (kernels only ever set it, msa_get_device_status() clears
+ * it) and the decode attention's merge counters (each call leaves them at zero). */
 MSA_API msa_status_t msa_workspace_init(void* workspace, size_t workspace_bytes, msa_stream_t stream);
 
 /* Self-test of the device error path: launches one tiny kernel that waits, with
@@ -311,7 +316,7 @@ MSA_API msa_status_t msa_selftest_wait_timeout(void* workspace, size_t workspace
  *     sequence, plus 2 * d * 128 bytes per (group, block)), so only small
  *     prefills fit.  Prefill with block 16/32 needs none.  Whatever does not
  *     fit returns MSA_ERR_WORKSPACE before anything is launched
- *     (msa_workspace_size(params, MSA_OP_SPARSE_ATTN) minus 256 is the need).
+ *     (msa_workspace_size(params, MSA_OP_SPARSE_ATTN) minus 4096 is the need).
  *   - All calls share that array and it keeps the last call's contents (the
  *     parts that must start at zero are cleared on the stream by every call):
  *     calls whose work overlaps on the GPU (two streams, or two host threads)

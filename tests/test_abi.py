@@ -59,15 +59,15 @@ def test_workspace_size_host_only(lib):
     p = valid_params()
     sel = msa.msa_workspace_size(p, msa.MSA_OP_INDEX_SELECT)
     fwd = msa.msa_workspace_size(p, msa.MSA_OP_FORWARD)
-    # status word + fp32 block scores [1, 1024, 2, 16] (+ ids for forward)
-    assert sel >= 256 + 1024 * 2 * 16 * 4
+    # status region + fp32 block scores [1, 1024, 2, 16] (+ ids for forward)
+    assert sel >= msa.STATUS_BYTES + 1024 * 2 * 16 * 4
     assert fwd >= sel + 1024 * 2 * 4 * 4
     assert msa.msa_workspace_size(p, 99) == 0
     # the index scan alone, the candidate merge and the shard lengths need the
-    # status word only; the candidates call needs what index select needs
+    # status region only; the candidates call needs what index select needs
     for op in (msa.MSA_OP_BLOCK_SCORES, msa.MSA_OP_SELECT_CANDIDATES, msa.MSA_OP_SHARD_LENGTHS,
                msa.MSA_OP_APPEND_KV):
-        assert msa.msa_workspace_size(p, op) == 256
+        assert msa.msa_workspace_size(p, op) == msa.STATUS_BYTES
     assert msa.msa_workspace_size(p, msa.MSA_OP_INDEX_CANDIDATES) == sel
 
 
@@ -163,18 +163,19 @@ def test_paged_params_validated(lib):
 def test_append_args_validated(lib):
     p = valid_params()
     fake = 1 << 20
-    assert msa.msa_workspace_size(p, msa.MSA_OP_APPEND_KV) == 256
+    assert msa.msa_workspace_size(p, msa.MSA_OP_APPEND_KV) == msa.STATUS_BYTES
     assert msa.msa_launch_count(p, msa.MSA_OP_APPEND_KV) == 1
     # new K rows without a K cache, misaligned new rows, a workspace without room
-    # for the status word
-    assert lib.msa_append_kv(ctypes.byref(p), fake, None, None, None, None, None, fake, 256,
+    # for the status region
+    sb = msa.STATUS_BYTES
+    assert lib.msa_append_kv(ctypes.byref(p), fake, None, None, None, None, None, fake, sb,
                              None) == msa.MSA_ERR_INVALID_ARG
-    assert lib.msa_append_kv(ctypes.byref(p), fake + 2, None, None, fake, None, None, fake, 256,
+    assert lib.msa_append_kv(ctypes.byref(p), fake + 2, None, None, fake, None, None, fake, sb,
                              None) == msa.MSA_ERR_INVALID_ARG
-    assert lib.msa_append_kv(ctypes.byref(p), fake, fake, fake, fake, fake, fake, fake, 128,
+    assert lib.msa_append_kv(ctypes.byref(p), fake, fake, fake, fake, fake, fake, fake, sb - 256,
                              None) == msa.MSA_ERR_WORKSPACE
     p.ki_strides[1] = 16  # index-key rows closer than d_idx
-    assert lib.msa_append_kv(ctypes.byref(p), None, None, fake, None, None, fake, fake, 256,
+    assert lib.msa_append_kv(ctypes.byref(p), None, None, fake, None, None, fake, fake, sb,
                              None) == msa.MSA_ERR_INVALID_ARG
 
 
