@@ -12,7 +12,8 @@
 // (counted with multiplicity), is found from the most significant bit down: the
 // visible keys share the high bits of the row's largest and smallest key, and
 // each step halves the bucket of keys that can still be T by counting the keys
-// at or above its midpoint.  Once at most 32 keys remain in the bucket they are
+// at or above its midpoint (the CTA kernel first narrows a large bucket eight bits
+// at a time with a shared histogram).  Once at most 32 keys remain in the bucket they are
 // gathered in id order and T is the one of the right rank among them (exact
 // ranks by key, ties by id), so the count steps stop long before the last bit.
 // Keys above T are all taken; keys equal to T are taken in ascending id order
@@ -289,8 +290,59 @@ __device__ __forceinline__ unsigned cta_exclusive_scan(unsigned v, unsigned* wsu
   return before + inc - v;
 }
 
+// One 8-bit step of the threshold search, for a bucket with at least 8 unresolved
+// bits: the bucket's keys are counted by their bits [hi - 7, hi] in a shared
+// histogram (hist[hb]; the other buffer is cleared for the next step) and the
+// digit holding the bucket key of rank need = m - above (counted from the top) is
+// found from suffix sums over the 256 bins, taken by the first 256 threads.  The
+// bucket becomes that digit's keys: eight bits resolved for three barriers.
+template <int NT, int E>
+__device__ __forceinline__ void bucket_radix8(Bucket& r, const uint32_t (&key)[E], int m,
+                                              unsigned (*hist)[256], int& hb, unsigned* wsum8,
+                                              int* res) {
+  static_assert(NT >= 256, "a thread per bin");
+  const int sh = r.hi - 7;
+  unsigned* h = hist[hb];
+  if (threadIdx.x < 256) hist[hb ^ 1][threadIdx.x] = 0u;
+#pragma unroll
+  for (int e = 0; e < E; ++e)
+    if (in_bucket(key[e], r)) atomicAdd(&h[(key[e] >> sh) & 255u], 1u);
+  __syncthreads();
+  const int t = threadIdx.x, lane = t & 31, w = t >> 5;
+  unsigned v = 0u, inc = 0u;
+  if (t < 256) {
+    v = h[255 - t];
+    inc = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const unsigned n = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += n;
+    }
+    if (lane == 31) wsum8[w] = inc;
+  }
+  __syncthreads();
+  if (t < 256) {
+    unsigned before = 0u;
+    for (int k = 0; k < w; ++k) before += wsum8[k];
+    const unsigned incl = before + inc, excl = incl - v, need = (unsigned)(m - r.above);
+    if (excl < need && need <= incl) {
+      res[0] = 255 - t;
+      res[1] = (int)excl;
+      res[2] = (int)v;
+    }
+  }
+  __syncthreads();
+  r.prefix |= (uint32_t)res[0] << sh;
+  r.above += res[1];
+  r.cnt = res[2];
+  r.hi = sh - 1;
+  hb ^= 1;
+}
+
 // One CTA of NT threads per row; thread i holds elements [i*E, i*E + E), read
-// with 16-byte loads.  Each search step is one CTA sum (one barrier).  The last
+// with 16-byte loads.  While the bucket holds more than 64 keys the search takes
+// eight bits per step (bucket_radix8, three barriers), then one bit per step (one
+// CTA sum, one barrier).  The last
 // bucket (at most 32 keys) is gathered in any order: T is a key value, so the
 // order among equal keys does not change it.  One more sum counts the keys above
 // and equal to T; only when some keys equal to T must be left out are they
@@ -308,6 +360,9 @@ __global__ void __launch_bounds__(NT) topk_cta_kernel(TopkArgs a) {
   __shared__ unsigned wsum[32];
   __shared__ uint32_t wmax[NW], wmin[NW];
   __shared__ uint32_t Ts;
+  __shared__ unsigned hist[2][256];
+  __shared__ unsigned wsum8[8];
+  __shared__ int rres[3];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int row = blockIdx.x;
   const RowInfo ri = row_info(a, row);
@@ -352,6 +407,7 @@ __global__ void __launch_bounds__(NT) topk_cta_kernel(TopkArgs a) {
       wmax[warp] = kmax;
       wmin[warp] = kmin;
     }
+    if (threadIdx.x < 256) hist[0][threadIdx.x] = 0u;
     __syncthreads();
     kmax = __reduce_max_sync(0xffffffffu, lane < NW ? wmax[lane] : 0u);
     kmin = __reduce_min_sync(0xffffffffu, lane < NW ? wmin[lane] : 0xffffffffu);
@@ -361,7 +417,12 @@ __global__ void __launch_bounds__(NT) topk_cta_kernel(TopkArgs a) {
       T = 0xffffffffu;  // only the forced block is taken
     } else {
       Bucket r = bucket_start(kmax, kmin, ri.F - forced, forced);
+      int hb = 0;
       while (r.cnt > 32 && r.hi >= 0) {
+        if (r.cnt > 64 && r.hi >= 7) {
+          bucket_radix8<NT, E>(r, key, m, hist, hb, wsum8, rres);
+          continue;
+        }
         const uint32_t cand = r.prefix | (1u << r.hi);
         unsigned c[1] = {0u};
 #pragma unroll
